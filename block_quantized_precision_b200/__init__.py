@@ -1,0 +1,172 @@
+"""Python binding of libqattn (block-quantized attention for B200, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/qattn.h. PyTorch provides device
+memory and streams. There is no fallback: if libqattn.so is missing or a call
+fails, an exception is raised.
+
+Function names follow the C ABI:
+    qattn_rotate_block_quant, qattn_prefill, qattn_decode_workspace_size,
+    qattn_decode_kvq, qattn_device_error, qattn_selftest_wait_timeout,
+    qattn_abi_version, qattn_status_string.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqattn.so")
+
+# Enumerations of include/qattn.h
+QATTN_OK = 0
+QATTN_ERR_INVALID_ARG = 1
+QATTN_ERR_UNSUPPORTED = 2
+QATTN_ERR_ALIGNMENT = 3
+QATTN_ERR_WORKSPACE = 4
+QATTN_ERR_CUDA = 5
+QATTN_ERR_TIMEOUT = 6
+
+QATTN_BNSD, QATTN_BSND = 0, 1
+QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 3, 4
+
+EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
+            "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_device_error",
+            "qattn_selftest_wait_timeout")
+
+_lib = None
+
+
+class QAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+def lib() -> C.CDLL:
+    """Loads libqattn.so from this package directory (raises if absent)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libqattn.so not built; run `python -m block_quantized_precision_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        P, i, f, z = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+        L.qattn_abi_version.restype = i
+        L.qattn_status_string.argtypes, L.qattn_status_string.restype = [i], C.c_char_p
+        L.qattn_rotate_block_quant.argtypes = [P, i, i, i, i, i, i, P, i, i, P, P, P]
+        L.qattn_rotate_block_quant.restype = i
+        L.qattn_prefill.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
+        L.qattn_prefill.restype = i
+        L.qattn_decode_workspace_size.argtypes, L.qattn_decode_workspace_size.restype = [i, i, i, i, i], z
+        L.qattn_decode_kvq.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, P, P, z, P]
+        L.qattn_decode_kvq.restype = i
+        L.qattn_device_error.argtypes, L.qattn_device_error.restype = [P], i
+        L.qattn_selftest_wait_timeout.argtypes, L.qattn_selftest_wait_timeout.restype = [i, P], i
+        _lib = L
+    return _lib
+
+
+def qattn_abi_version() -> int:
+    return int(lib().qattn_abi_version())
+
+
+def status_string(status: int) -> str:
+    return lib().qattn_status_string(int(status)).decode()
+
+
+qattn_status_string = status_string
+
+
+def _check(status: int, where: str):
+    if status != QATTN_OK:
+        raise QAttnError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dims(x, layout):
+    if layout == QATTN_BNSD:
+        B, H, N, D = x.shape
+    else:
+        B, N, H, D = x.shape
+    return B, H, N, D
+
+
+def qattn_rotate_block_quant(x, layout: int, rot, block_tokens: int, code_dtype: int,
+                             codes=None, scales=None, stream=None):
+    """Rotation (optional) + dynamic block quantization of one tensor.
+
+    x: CUDA bfloat16/float16 tensor in `layout`; rot: CUDA float32 [D, D] or
+    None. Returns (codes uint8 like x, scales float32 [B, H, nblk])."""
+    import torch
+    B, H, N, D = _dims(x, layout)
+    x_dtype = {torch.bfloat16: QATTN_BF16, torch.float16: QATTN_F16}[x.dtype]
+    nblk = -(-N // block_tokens)
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((B, H, nblk), dtype=torch.float32, device=x.device)
+    st = lib().qattn_rotate_block_quant(_ptr(x), x_dtype, layout, B, H, N, D, _ptr(rot), block_tokens,
+                                        code_dtype, _ptr(codes), _ptr(scales), _stream(stream))
+    _check(st, "qattn_rotate_block_quant")
+    return codes, scales
+
+
+def qattn_prefill(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, code_dtype: int, layout: int,
+                  causal: bool, softmax_scale: float = 0.0, out=None, lse=None, q_block: int = 128,
+                  kv_block: int = 256, stream=None):
+    """Quantized attention over codes; returns the bfloat16 output (layout of Q)."""
+    import torch
+    B, H, Nq, D = _dims(q_codes, layout)
+    Nkv = _dims(k_codes, layout)[2]
+    if out is None:
+        out = torch.empty(q_codes.shape, dtype=torch.bfloat16, device=q_codes.device)
+    st = lib().qattn_prefill(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                             _ptr(v_scales), code_dtype, layout, B, H, Nq, Nkv, D, q_block, kv_block,
+                             int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "qattn_prefill")
+    return out
+
+
+def qattn_decode_workspace_size(B: int, H_q: int, H_kv: int, L: int, D: int) -> int:
+    return int(lib().qattn_decode_workspace_size(B, H_q, H_kv, L, D))
+
+
+def qattn_decode_kvq(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: int, kv_block: int = 256,
+                     group: int = 128, softmax_scale: float = 0.0, out=None, workspace=None, stream=None):
+    """One decode step against an INT8 / packed-INT4 KV cache.
+
+    q: bfloat16 [B, H_q, 1, D]; caches [B, H_kv, L, D] (INT8) or
+    [B, H_kv, L, D/2] (INT4). Returns the bfloat16 output [B, H_q, 1, D]."""
+    import torch
+    B, Hq, _, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=q.device)
+    need = qattn_decode_workspace_size(B, Hq, Hkv, L, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = lib().qattn_decode_kvq(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales), kv_dtype,
+                                B, Hq, Hkv, L, D, kv_block, group, float(softmax_scale), _ptr(out),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "qattn_decode_kvq")
+    return out
+
+
+def qattn_device_error(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device error word."""
+    return int(lib().qattn_device_error(_stream(stream)))
+
+
+def qattn_selftest_wait_timeout(timeout_ms: int, stream=None):
+    _check(lib().qattn_selftest_wait_timeout(int(timeout_ms), _stream(stream)), "qattn_selftest_wait_timeout")

@@ -1,0 +1,232 @@
+// qattn_abi.cu -- the extern "C" entry points declared in include/qattn.h:
+// argument validation, per-device state (SM count, error word), dispatch to
+// the kernel launchers.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/qattn.h"
+#include "qattn_device.cuh"
+#include "qattn_internal.h"
+
+namespace qattn {
+
+// Per-device error word written by kernels whose bounded waits run out.
+__device__ int g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  int* err = nullptr;  // device address of g_error_word on this device
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Per-device set-up, done once per device with that device current: SM
+// count and the device address of the error word.
+qattn_status_t device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return QATTN_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return QATTN_ERR_CUDA;
+    if (major != 10) return QATTN_ERR_UNSUPPORTED;  // built for sm_100a only
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return QATTN_ERR_CUDA;
+    s.num_sms = sms;
+    s.err = static_cast<int*>(p);
+    s.ready = true;
+  }
+  *out = &s;
+  return QATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qattn_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? QATTN_OK : QATTN_ERR_CUDA; }
+
+__global__ void wait_selftest_kernel(int* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the bounded wait must run out, record
+  // QATTN_ERR_TIMEOUT and return.
+  mbar_wait(&bar, 0, &abort_flag, err, limit_ns);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(err, static_cast<uint64_t>(timeout_ms) * 1000000ull);
+  return cudaGetLastError();
+}
+
+}  // namespace qattn
+
+using namespace qattn;
+
+extern "C" {
+
+int qattn_abi_version(void) { return QATTN_ABI_VERSION; }
+
+const char* qattn_status_string(qattn_status_t s) {
+  switch (s) {
+    case QATTN_OK: return "ok";
+    case QATTN_ERR_INVALID_ARG: return "invalid argument";
+    case QATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case QATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case QATTN_ERR_CUDA: return "CUDA error";
+    case QATTN_ERR_TIMEOUT: return "kernel barrier wait timed out";
+  }
+  return "unknown status";
+}
+
+qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype, qattn_layout_t layout, int B,
+                                        int H, int N, int D, const float* rot, int block_tokens,
+                                        qattn_dtype_t code_dtype, void* codes, float* scales,
+                                        qattn_stream_t stream) {
+  if (B < 0 || H < 0 || N < 0 || D <= 0 || block_tokens <= 0) return QATTN_ERR_INVALID_ARG;
+  if (x_dtype != QATTN_F16 && x_dtype != QATTN_BF16) return QATTN_ERR_INVALID_ARG;
+  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
+  if (!rotate_block_quant_supported(D, block_tokens)) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * N == 0) return QATTN_OK;
+  if (!x || !codes || !scales) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || (rot && !aligned16(rot))) return QATTN_ERR_ALIGNMENT;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  RotQuantArgs a;
+  a.x = x;
+  a.is_bf16 = x_dtype == QATTN_BF16;
+  a.layout = layout;
+  a.B = B; a.H = H; a.N = N; a.D = D; a.T = block_tokens;
+  a.rot = rot;
+  a.int8 = code_dtype == QATTN_INT8;
+  a.codes = codes;
+  a.scales = scales;
+  return from_cuda(launch_rotate_block_quant(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms));
+}
+
+qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,
+                             const void* v_codes, const float* v_scales, qattn_dtype_t code_dtype,
+                             qattn_layout_t layout, int B, int H, int N_q, int N_kv, int D, int q_block,
+                             int kv_block, int causal, float softmax_scale, void* out, float* lse,
+                             qattn_stream_t stream) {
+  if (B < 0 || H < 0 || N_q < 0 || N_kv < 0 || D <= 0) return QATTN_ERR_INVALID_ARG;
+  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return QATTN_ERR_INVALID_ARG;
+  if (causal && N_q != N_kv) return QATTN_ERR_UNSUPPORTED;
+  if (q_block != 128 || kv_block != 256) return QATTN_ERR_UNSUPPORTED;
+  if (!prefill_supported(D)) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * N_q == 0) return QATTN_OK;
+  if (N_kv == 0) return QATTN_ERR_UNSUPPORTED;  // softmax over no keys is undefined
+  if (!q_codes || !q_scales || !k_codes || !k_scales || !v_codes || !v_scales || !out) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(out))
+    return QATTN_ERR_ALIGNMENT;
+  if (static_cast<int64_t>(B) * H * ((N_q + 127) / 128) >= (1LL << 31)) return QATTN_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / sqrtf(static_cast<float>(D));
+  PrefillArgs a;
+  a.q = q_codes; a.qs = q_scales;
+  a.k = k_codes; a.ks = k_scales;
+  a.v = v_codes; a.vs = v_scales;
+  a.int8 = code_dtype == QATTN_INT8;
+  a.layout = layout;
+  a.B = B; a.H = H; a.Nq = N_q; a.Nkv = N_kv; a.D = D;
+  a.causal = causal;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
+  return from_cuda(launch_prefill(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
+}
+
+size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D) {
+  if (B <= 0 || H_q <= 0 || H_kv <= 0 || L < 0 || D <= 0 || H_q % H_kv) return 0;
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != QATTN_OK) return 0;
+  return decode_workspace_bytes(B, H_q, H_kv, L, D, ds->num_sms);
+}
+
+qattn_status_t qattn_decode_kvq(const void* q, const void* k_cache, const void* v_cache, const void* k_scales,
+                                const void* v_scales, qattn_dtype_t kv_dtype, int B, int H_q, int H_kv, int L,
+                                int D, int kv_block, int group, float softmax_scale, void* out, void* workspace,
+                                size_t workspace_bytes, qattn_stream_t stream) {
+  if (B < 0 || H_q <= 0 || H_kv <= 0 || L < 0 || D <= 0) return QATTN_ERR_INVALID_ARG;
+  if (H_q % H_kv) return QATTN_ERR_INVALID_ARG;
+  if (kv_dtype != QATTN_INT8 && kv_dtype != QATTN_INT4_PACKED) return QATTN_ERR_INVALID_ARG;
+  const int G = H_q / H_kv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return QATTN_ERR_UNSUPPORTED;
+  int group_ratio = 1;
+  if (kv_dtype == QATTN_INT8) {
+    if (kv_block != 256) return QATTN_ERR_UNSUPPORTED;
+  } else {
+    if (group <= 0 || D % group) return QATTN_ERR_INVALID_ARG;
+    group_ratio = D / group;
+  }
+  if (!decode_supported(D, group_ratio)) return QATTN_ERR_UNSUPPORTED;
+  if (B == 0) return QATTN_OK;
+  if (!q || !out || !workspace) return QATTN_ERR_INVALID_ARG;
+  if (L > 0 && (!k_cache || !v_cache || !k_scales || !v_scales)) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || (L > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
+    return QATTN_ERR_ALIGNMENT;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  if (workspace_bytes < decode_workspace_bytes(B, H_q, H_kv, L, D, ds->num_sms)) return QATTN_ERR_WORKSPACE;
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / sqrtf(static_cast<float>(D));
+  DecodeArgs a;
+  a.q = q; a.k = k_cache; a.v = v_cache; a.ks = k_scales; a.vs = v_scales;
+  a.int4 = kv_dtype == QATTN_INT4_PACKED;
+  a.B = B; a.Hq = H_q; a.Hkv = H_kv; a.L = L; a.D = D;
+  a.kv_block = kv_dtype == QATTN_INT8 ? kv_block : 256;
+  a.group = kv_dtype == QATTN_INT4_PACKED ? group : D;
+  a.scale = softmax_scale;
+  a.out = out;
+  a.workspace = workspace;
+  return from_cuda(launch_decode(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
+}
+
+qattn_status_t qattn_device_error(qattn_stream_t stream) {
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ds->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QATTN_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(ds->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return QATTN_ERR_CUDA;
+  }
+  return static_cast<qattn_status_t>(v);
+}
+
+qattn_status_t qattn_selftest_wait_timeout(int timeout_ms, qattn_stream_t stream) {
+  if (timeout_ms < 1 || timeout_ms > 2000) return QATTN_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  return from_cuda(launch_wait_selftest(timeout_ms, reinterpret_cast<cudaStream_t>(stream), ds->err));
+}
+
+}  // extern "C"

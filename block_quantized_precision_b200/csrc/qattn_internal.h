@@ -1,0 +1,65 @@
+// qattn_internal.h -- launcher interfaces between the C ABI (qattn_abi.cu)
+// and the kernel files. Arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qattn {
+
+struct RotQuantArgs {
+  const void* x;      // F16/BF16 bits
+  int is_bf16;
+  int layout;         // 0 = BNSD, 1 = BSND
+  int B, H, N, D, T;  // T = block tokens
+  const float* rot;   // D x D or nullptr
+  int int8;           // 1: INT8 codes, 0: e4m3
+  void* codes;
+  float* scales;
+};
+
+bool rotate_block_quant_supported(int D, int T);
+cudaError_t launch_rotate_block_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms);
+
+struct PrefillArgs {
+  const void* q;
+  const float* qs;
+  const void* k;
+  const float* ks;
+  const void* v;
+  const float* vs;
+  int int8;           // 1: INT8 codes, 0: e4m3
+  int layout;
+  int B, H, Nq, Nkv, D;
+  int causal;
+  float scale_log2;   // softmax_scale * log2(e)
+  void* out;          // bf16
+  float* lse;         // nullable
+};
+
+bool prefill_supported(int D);
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st, int num_sms, int* err);
+
+struct DecodeArgs {
+  const void* q;      // bf16 [B, Hq, 1, D]
+  const void* k;
+  const void* v;
+  const void* ks;
+  const void* vs;
+  int int4;           // 1: packed INT4 cache, 0: INT8 cache
+  int B, Hq, Hkv, L, D;
+  int kv_block, group;
+  float scale;        // softmax scale
+  void* out;          // bf16 [B, Hq, 1, D]
+  void* workspace;
+};
+
+bool decode_supported(int D, int group_size_ratio);
+int decode_splits(int B, int Hkv, int L, int num_sms);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int D, int num_sms);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, int num_sms, int* err);
+
+cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err);
+
+}  // namespace qattn

@@ -1,0 +1,220 @@
+/*
+ * qattn.h -- C ABI of libqattn: block-quantized attention on NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (as stated on the pages this library implements):
+ *   1. Q and K are multiplied by one shared orthogonal matrix R before
+ *      quantization, to spread outlier channels ("MindIE-SD quantization",
+ *      section FA量化 / 技术特点 / 旋转(Rotate)). V is not rotated.
+ *   2. Q, K, V are quantized dynamically per block of tokens, one scale per
+ *      (batch, head, block): Q blocks of 128 tokens, K/V blocks of 256, to
+ *      float8_e4m3fn (same page, 块量化) or to symmetric INT8 with
+ *      scale = max|x| / 127, code = round(x / scale), zero point 0
+ *      ("INT8 量化算子", 对称量化).
+ *   3. Attention runs on the codes: INT8 x INT8 -> INT32 (or e4m3 x e4m3 ->
+ *      FP32) for Q K^T, a running softmax over key tiles, P quantized to the
+ *      same 8-bit type, P V with the per-block V scale, output in bfloat16
+ *      ("MindIE-SD quantization", FP8 Attention; "INT8 量化算子",
+ *      ops-transformer items 1-3; "FlashAttention 的 INT8/INT4 量化",
+ *      三层实现详解).
+ *   4. Decode reads an INT8 or packed INT4 KV cache directly, with no
+ *      dequantize-to-fp16 pass ("INT8 量化算子", item 3 KV Cache 也量化;
+ *      "ops-transformer INT8/INT4 量化推理", 5.1 and 5.2 for INT4 groups and
+ *      packing).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never frees or keeps them. The library allocates no device
+ *     memory per call (scratch for decode is passed in as `workspace`).
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream). The call returns once the launch is enqueued.
+ *   - Arguments are validated before anything is launched; on any error
+ *     nothing is launched and a status other than QATTN_OK is returned.
+ *     A failed launch returns QATTN_ERR_CUDA.
+ *   - Kernels that wait on on-chip barriers give up after about one second,
+ *     record QATTN_ERR_TIMEOUT in a per-device error word and exit cleanly;
+ *     qattn_device_error() reads and clears that word.
+ *   - Layouts: QATTN_BNSD = [B, H, N, D] (head-major), QATTN_BSND =
+ *     [B, N, H, D] (token-major); N is the number of tokens, H the number
+ *     of heads. Both are dense and row-major.
+ *   - Pointers must be 16-byte aligned (QATTN_ERR_ALIGNMENT otherwise).
+ *   - Supported head sizes: D in {64, 128} (D = 128 for decode).
+ */
+#ifndef QATTN_H_
+#define QATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QATTN_ABI_VERSION 1
+
+typedef enum qattn_status {
+  QATTN_OK = 0,
+  QATTN_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shapes */
+  QATTN_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. D = 96) */
+  QATTN_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+  QATTN_ERR_WORKSPACE = 4,   /* decode workspace missing or too small */
+  QATTN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  QATTN_ERR_TIMEOUT = 6      /* a kernel's bounded barrier wait ran out */
+} qattn_status_t;
+
+typedef enum qattn_layout { QATTN_BNSD = 0, QATTN_BSND = 1 } qattn_layout_t;
+
+typedef enum qattn_dtype {
+  QATTN_F16 = 0,
+  QATTN_BF16 = 1,
+  QATTN_INT8 = 2,        /* signed 8-bit codes */
+  QATTN_FP8_E4M3 = 3,    /* float8_e4m3fn codes (OCP E4M3, finite) */
+  QATTN_INT4_PACKED = 4  /* two signed 4-bit codes per byte, element 2i in bits 0..3 */
+} qattn_dtype_t;
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* qattn_stream_t;
+
+/* Returns QATTN_ABI_VERSION of the built library. */
+int qattn_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+const char* qattn_status_string(qattn_status_t status);
+
+/*
+ * Fused rotation + dynamic block quantization (one launch per tensor).
+ *
+ * Defined by: "MindIE-SD quantization", FA量化 / 技术特点 (旋转, 块量化);
+ * "INT8 量化算子", 1. 对称量化.
+ *
+ * For every (b, h) and every block of `block_tokens` consecutive tokens
+ * (the last block may be shorter when N is not a multiple):
+ *   y      = x R                  rotation; R == NULL means y = x. Each
+ *                                 y[j] is the float32 fused multiply-add
+ *                                 chain over k = 0..D-1 in ascending order
+ *                                 starting from +0 (bit-reproducible).
+ *   amax   = max |y| over the block's tokens and all D channels
+ *   scale  = amax / qmax          float32 IEEE division; qmax = 127 (INT8)
+ *                                 or 448 (e4m3)
+ *   code   = RNE(y / scale)       float32 IEEE division, then round half to
+ *                                 even; INT8 saturates to [-127, 127], e4m3
+ *                                 saturates to +-448. scale == 0 gives all
+ *                                 codes 0.
+ *
+ * x:            x_dtype (QATTN_F16 or QATTN_BF16) values, `layout`,
+ *               [B,H,N,D] or [B,N,H,D].
+ * rot:          D x D float32 row-major (rot[k*D + j] = R[k][j]), or NULL.
+ * block_tokens: tokens per block: 128 (Q) or 256 (K/V).
+ * code_dtype:   QATTN_INT8 or QATTN_FP8_E4M3.
+ * codes:        output, 1 byte per element, same layout and shape as x.
+ * scales:       output, float32 [B, H, ceil(N / block_tokens)].
+ */
+qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype,
+                                        qattn_layout_t layout, int B, int H, int N, int D,
+                                        const float* rot, int block_tokens,
+                                        qattn_dtype_t code_dtype, void* codes, float* scales,
+                                        qattn_stream_t stream);
+
+/*
+ * Quantized attention over block-quantized codes (prefill).
+ *
+ * Defined by: "MindIE-SD quantization", FA量化 / FP8 Attention (attention in
+ * the FP8 domain, output returned in the original precision); "INT8 量化算子",
+ * ops-transformer items 1-2 (INT8 x INT8 -> INT32, convert at the output,
+ * scales kept on chip); "FlashAttention 的 INT8/INT4 量化", 三层实现详解
+ * (outer loop over query tiles, inner loop over key/value tiles).
+ *
+ * For query row i of head (b, h), key tiles of 128 keys in ascending order:
+ *   S[i,j] = sum_d qcode[i,d] kcode[j,d]   exact INT32 (INT8 codes) or
+ *                                          FP32-accumulated (e4m3 codes)
+ *   s[i,j] = S[i,j] * q_scales[b,h,i/q_block] * k_scales[b,h,j/kv_block]
+ *            * softmax_scale              (masked: j > i when causal)
+ *   running max m, alpha = exp(m_old - m_new), p = exp(s - m_new)
+ *   P = e4m3(p) for e4m3 codes; round(127 p) / 127 for INT8 codes
+ *   l = l * alpha + sum_j P;  O = O * alpha + sum_j P vcode[j] v_scales[b,h,j/kv_block]
+ *   out = bf16(O / l);  lse = m + ln(l) (natural log)
+ *
+ * q_codes/k_codes/v_codes: code_dtype bytes in `layout`; Q is [B,H,N_q,D]
+ *               (or [B,N_q,H,D]), K and V use N_kv tokens.
+ * q_scales:     float32 [B, H, ceil(N_q / q_block)];
+ * k_scales, v_scales: float32 [B, H, ceil(N_kv / kv_block)].
+ * q_block:      must be 128; kv_block: must be 256 (the method's sizes).
+ * causal:       0 or 1; causal requires N_q == N_kv (top-left aligned).
+ * softmax_scale: <= 0 selects 1/sqrt(D) (computed in float32).
+ * out:          bfloat16, same layout as Q.
+ * lse:          optional (NULL) float32 [B, H, N_q].
+ */
+qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const void* k_codes,
+                             const float* k_scales, const void* v_codes, const float* v_scales,
+                             qattn_dtype_t code_dtype, qattn_layout_t layout, int B, int H,
+                             int N_q, int N_kv, int D, int q_block, int kv_block, int causal,
+                             float softmax_scale, void* out, float* lse, qattn_stream_t stream);
+
+/*
+ * Bytes of device workspace qattn_decode_kvq needs for these sizes on the
+ * current device (0 when no scratch is needed). The value depends on the
+ * device's SM count.
+ */
+size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D);
+
+/*
+ * One decode step against a quantized KV cache, split over the key axis,
+ * with a final softmax merge of the splits.
+ *
+ * Defined by: "INT8 量化算子", ops-transformer item 3 (KV Cache 也量化: K/V
+ * stored as INT8 and attended without converting back to fp16; the query is
+ * INT8 too) and its Int8Attention listing; "ops-transformer INT8/INT4
+ * 量化推理", 5.1 (one fp16 scale per group of G elements) and 5.2 (two INT4
+ * per byte, element 2i in the low nibble).
+ *
+ * Query head h uses KV head h / (H_q / H_kv).
+ *   INT8 cache:  sq = max|q| / 127, qcode = RNE(q / sq) (float32, clamped to
+ *                [-127, 127]); s_t = (qcode . kcode_t) * sq *
+ *                k_scales[b,hk,t/kv_block] * softmax_scale;
+ *                v_t = vcode_t * v_scales[b,hk,t/kv_block].
+ *   INT4 cache:  s_t = sum_g k_scales[b,hk,t,g] * (q . kcode_t over group g)
+ *                * softmax_scale with q in float32;
+ *                v_t[d] = vcode_t[d] * v_scales[b,hk,t,d/group].
+ *   out = bf16(sum_t p_t v_t / sum_t p_t), p_t = exp(s_t - max s) in float32.
+ *
+ * q:        bfloat16 [B, H_q, 1, D].
+ * k_cache, v_cache: QATTN_INT8: int8 [B, H_kv, L, D];
+ *           QATTN_INT4_PACKED: bytes [B, H_kv, L, D/2].
+ * k_scales, v_scales: QATTN_INT8: float32 [B, H_kv, ceil(L/kv_block)];
+ *           QATTN_INT4_PACKED: float16 [B, H_kv, L, D/group].
+ * kv_block: 256 (INT8); group: 128 (INT4, must divide D).
+ * softmax_scale: <= 0 selects 1/sqrt(D) (float32).
+ * out:      bfloat16 [B, H_q, 1, D].
+ * workspace / workspace_bytes: device scratch of at least
+ *           qattn_decode_workspace_size(B, H_q, H_kv, L, D) bytes, 16-byte
+ *           aligned; its contents need no initialisation and are
+ *           overwritten. Calls that share a workspace must not overlap.
+ * L == 0 writes zeros to out.
+ */
+qattn_status_t qattn_decode_kvq(const void* q, const void* k_cache, const void* v_cache,
+                                const void* k_scales, const void* v_scales,
+                                qattn_dtype_t kv_dtype, int B, int H_q, int H_kv, int L, int D,
+                                int kv_block, int group, float softmax_scale, void* out,
+                                void* workspace, size_t workspace_bytes, qattn_stream_t stream);
+
+/*
+ * Waits for `stream`, then reads and clears the per-device error word that
+ * kernels set when a bounded barrier wait runs out. Returns QATTN_OK,
+ * QATTN_ERR_TIMEOUT, or QATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+qattn_status_t qattn_device_error(qattn_stream_t stream);
+
+/*
+ * Self-test of the bounded-wait path: launches one block that waits on an
+ * on-chip barrier that nothing completes, with a limit of `timeout_ms`
+ * milliseconds (1..2000). The kernel records QATTN_ERR_TIMEOUT and returns;
+ * nothing faults or hangs. Follow with qattn_device_error() to observe it.
+ * No counterpart on the pages: it exists to test failure reporting.
+ */
+qattn_status_t qattn_selftest_wait_timeout(int timeout_ms, qattn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QATTN_H_ */

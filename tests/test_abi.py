@@ -1,0 +1,120 @@
+"""The C-ABI library builds, loads and exports every entry point declared in
+include/qattn.h; argument validation answers without launching anything.
+
+CPU only (no kernel is launched by these calls).
+"""
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_quantized_precision_b200 as qa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qattn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qattn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_quantized_precision_b200 import build
+    build.build()
+    return qa.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared()
+    assert set(declared) == set(qa.EXPORTED)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", qa.LIB_PATH]).decode()
+    exported = set(re.findall(r"\bT (qattn_[a-z0-9_]+)", out))
+    assert set(declared) <= exported
+    for name in declared:
+        assert hasattr(L, name)
+
+
+def test_version_and_status_strings(L):
+    assert qa.qattn_abi_version() == 1
+    for code in range(7):
+        assert qa.status_string(code) and qa.status_string(code) != "unknown status"
+    assert qa.status_string(99) == "unknown status"
+
+
+def test_rotate_block_quant_validation(L):
+    f = L.qattn_rotate_block_quant
+    bad = 0x1000
+    # negative size, bad dtypes, bad layout
+    assert f(bad, qa.QATTN_BF16, 0, -1, 1, 1, 128, None, 128, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert f(bad, qa.QATTN_INT8, 0, 1, 1, 1, 128, None, 128, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert f(bad, qa.QATTN_BF16, 0, 1, 1, 1, 128, None, 128, qa.QATTN_BF16, bad, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert f(bad, qa.QATTN_BF16, 7, 1, 1, 1, 128, None, 128, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    # unsupported head size / block size
+    assert f(bad, qa.QATTN_BF16, 0, 1, 1, 1, 96, None, 128, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_UNSUPPORTED
+    assert f(bad, qa.QATTN_BF16, 0, 1, 1, 1, 128, None, 100, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_UNSUPPORTED
+    # empty problem: nothing to do
+    assert f(None, qa.QATTN_BF16, 0, 0, 4, 128, 128, None, 128, qa.QATTN_INT8, None, None, None) == qa.QATTN_OK
+    # null pointers / misalignment
+    assert f(None, qa.QATTN_BF16, 0, 1, 1, 8, 128, None, 128, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert f(bad + 8, qa.QATTN_BF16, 0, 1, 1, 8, 128, None, 128, qa.QATTN_INT8, bad, bad, None) == qa.QATTN_ERR_ALIGNMENT
+
+
+def test_prefill_validation(L):
+    f = L.qattn_prefill
+    p = 0x1000
+    args = dict(B=1, H=1, Nq=256, Nkv=256, D=128, qb=128, kb=256, causal=0)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(p, p, p, p, p, p, kw.get("code", qa.QATTN_INT8), kw.get("layout", 0), a["B"], a["H"], a["Nq"],
+                 a["Nkv"], a["D"], a["qb"], a["kb"], a["causal"], 0.0, kw.get("out", p), None, None)
+    assert call(code=qa.QATTN_BF16) == qa.QATTN_ERR_INVALID_ARG
+    assert call(causal=2) == qa.QATTN_ERR_INVALID_ARG
+    assert call(causal=1, Nkv=512) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(qb=64) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(kb=128) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(D=96) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(Nq=0) == qa.QATTN_OK
+    assert call(Nkv=0) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(out=None) == qa.QATTN_ERR_INVALID_ARG
+    assert call(out=p + 2) == qa.QATTN_ERR_ALIGNMENT
+    assert call(B=-1) == qa.QATTN_ERR_INVALID_ARG
+
+
+def test_decode_validation(L):
+    f = L.qattn_decode_kvq
+    p = 0x1000
+
+    def call(kv=qa.QATTN_INT8, B=1, Hq=32, Hkv=8, Lk=256, D=128, kvb=256, grp=128, ws=p):
+        return f(p, p, p, p, p, kv, B, Hq, Hkv, Lk, D, kvb, grp, 0.0, p, ws, 1 << 30, None)
+    assert call(Hq=30) == qa.QATTN_ERR_INVALID_ARG
+    assert call(kv=qa.QATTN_FP8_E4M3) == qa.QATTN_ERR_INVALID_ARG
+    assert call(Hq=48, Hkv=3) == qa.QATTN_ERR_UNSUPPORTED     # 16 query heads per kv head
+    assert call(kvb=128) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(kv=qa.QATTN_INT4_PACKED, grp=96) == qa.QATTN_ERR_INVALID_ARG
+    assert call(kv=qa.QATTN_INT4_PACKED, grp=32) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(D=64) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(B=0) == qa.QATTN_OK
+    assert call(ws=None) == qa.QATTN_ERR_INVALID_ARG
+    assert call(ws=p + 4) == qa.QATTN_ERR_ALIGNMENT
+
+
+def test_selftest_rejects_out_of_range_limits(L):
+    assert L.qattn_selftest_wait_timeout(0, None) == qa.QATTN_ERR_INVALID_ARG
+    assert L.qattn_selftest_wait_timeout(5000, None) == qa.QATTN_ERR_INVALID_ARG
+
+
+def test_oracle_and_library_share_no_code():
+    """The oracle is plain C compiled by gcc; the library is CUDA. Neither
+    includes or imports the other."""
+    ora = open(os.path.join(ROOT, "oracle", "qattn_oracle.c")).read()
+    assert "qattn.h" not in ora and "csrc" not in ora
+    for f in os.listdir(os.path.join(ROOT, "block_quantized_precision_b200", "csrc")):
+        src = open(os.path.join(ROOT, "block_quantized_precision_b200", "csrc", f)).read()
+        assert "oracle" not in src.lower().replace("oracle-only", "")
+    pkg = open(os.path.join(ROOT, "block_quantized_precision_b200", "__init__.py")).read()
+    assert "import oracle" not in pkg and "from oracle" not in pkg

@@ -1,0 +1,83 @@
+"""GPU parity of the fused rotation + block quantization kernel: codes and
+scales must equal the oracle's bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_precision_b200 as qa
+import synth
+from parity_util import dev, dev_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_all(orc, x_bits, in_dtype, layout, rot, block, code_dtype, blocks=None):
+    x = dev_bits(x_bits, in_dtype)
+    r = dev(rot) if rot is not None else None
+    codes, scales = qa.qattn_rotate_block_quant(x, layout, r, block, code_dtype)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    gc, gs = codes.cpu().numpy(), scales.cpu().numpy()
+    oc, os_ = orc.rotate_block_quant(x_bits, in_dtype, layout, rot, block, code_dtype, blocks=blocks)
+    if blocks is None:
+        assert np.array_equal(gs.view(np.uint32), os_.view(np.uint32))
+        bad = np.nonzero(gc != oc)
+        assert bad[0].size == 0, "codes differ at %d places, first %s" % (bad[0].size, [b[:3] for b in bad])
+    else:
+        N = x_bits.shape[2] if layout == synth.BNSD else x_bits.shape[1]
+        for (b, h, k) in blocks:
+            assert gs[b, h, k].view(np.uint32) == os_[b, h, k].view(np.uint32)
+            n0, n1 = k * block, min(N, (k + 1) * block)
+            if layout == synth.BNSD:
+                assert np.array_equal(gc[b, h, n0:n1], oc[b, h, n0:n1])
+            else:
+                assert np.array_equal(gc[b, n0:n1, h], oc[b, n0:n1, h])
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("layout", [synth.BNSD, synth.BSND])
+@pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
+@pytest.mark.parametrize("rotate", [False, True])
+@pytest.mark.parametrize("block", [128, 256])
+def test_small_shapes_bit_exact(orc, D, layout, code_dtype, rotate, block):
+    B, H, N = 2, 3, 300                     # ragged tail block
+    rng = np.random.default_rng(D + 7 * layout + 13 * code_dtype + rotate + block)
+    shape = (B, H, N, D) if layout == synth.BNSD else (B, N, H, D)
+    x = synth.f32_to_bf16_bits(rng.standard_normal(shape) * np.exp(rng.standard_normal(shape[:-1] + (1,))))
+    rot = synth.haar_orthogonal(17, 4, D) if rotate else None
+    _check_all(orc, x, synth.BF16, layout, rot, block, code_dtype)
+
+
+def test_f16_input_and_edge_blocks(orc):
+    B, H, N, D = 1, 2, 257, 128               # last block holds one token
+    rng = np.random.default_rng(3)
+    x = synth.f64_to_f16_bits(rng.standard_normal((B, H, N, D)))
+    x[0, 1, :128] = 0                         # an all-zero block: scale 0, codes 0
+    rot = synth.haar_orthogonal(3, 4, D)
+    for code in (synth.INT8, synth.FP8_E4M3):
+        _check_all(orc, x, synth.F16, synth.BNSD, rot, 128, code)
+        _check_all(orc, x, synth.F16, synth.BNSD, None, 128, code)
+
+
+def test_outlier_channels_int8_config_small(orc):
+    p = synth.scaled(synth.INT8_CAUSAL, H=4, N=512)
+    d = synth.make_prefill(p)
+    for name, blk, rot in (("q", 128, d["rot"]), ("k", 256, d["rot"]), ("v", 256, None)):
+        _check_all(orc, d[name], p.in_dtype, p.layout, rot, blk, p.code_dtype)
+
+
+@pytest.mark.parametrize("prob", ["tiny_fp8_b1h2n256d64", "int8_causal_b1h32n4096d128", "fp8_bsnd_b1h24n16384d128"])
+def test_full_size_sampled_blocks(orc, prob):
+    """Full-size problems in the launch configuration the benchmark uses;
+    the oracle recomputes a sample of blocks (all of them for the tiny one)."""
+    p = synth.PROBLEMS[prob]
+    d = synth.make_prefill(p)
+    rng = np.random.default_rng(5)
+    for name, blk, rot in (("q", 128, d["rot"]), ("k", 256, d["rot"]), ("v", 256, None)):
+        nblk = -(-p.N // blk)
+        if p.N <= 256:
+            blocks = None
+        else:
+            blocks = [(0, int(h), int(k)) for h, k in zip(rng.integers(0, p.H, 6), rng.integers(0, nblk, 6))]
+            blocks += [(0, p.H - 1, nblk - 1), (0, 0, 0)]
+        _check_all(orc, d[name], p.in_dtype, p.layout, rot, blk, p.code_dtype, blocks=blocks)
