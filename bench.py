@@ -1,0 +1,509 @@
+"""Benchmark of the block-quantized attention hot path on B200.
+
+One step = one pass of the whole prefill path on the INT8 causal problem
+(B=1, H=32, N=4096, D=128, bf16 inputs with outlier channels, shared seeded
+rotation): rotate+quantize Q (blocks of 128), K and V (blocks of 256), then
+quantized attention. value = algorithmic INT8 operations of the attention
+(4*D per unmasked query/key pair) / step time, in TOPS, whole job (all
+ranks). Inputs are resident in HBM; L2 is flushed (256 MB write) before
+every timed step. The same line carries the decode KV bandwidth (INT8 and
+packed-INT4 caches) and the FP8 long-sequence prefill measured in the same
+run, each with its roofline fraction.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the CPU oracle (the reference arm of this repo) on a
+bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np
+
+METRIC = "prefill quantized-attention TFLOPS and decode KV GB/s on 1 B200, % of roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+def prefill_ops(B, H, N, D, causal):
+    pairs = N * (N + 1) // 2 if causal else N * N
+    return 4.0 * D * B * H * pairs
+
+
+def decode_bytes(p):
+    if p.kv_dtype == 2:   # INT8
+        nkb = -(-p.L // p.kv_block)
+        kv = 2 * p.B * p.Hkv * p.L * p.D
+        sc = 2 * p.B * p.Hkv * nkb * 4
+    else:
+        kv = 2 * p.B * p.Hkv * p.L * p.D // 2
+        sc = 2 * p.B * p.Hkv * p.L * (p.D // p.group) * 2
+    qo = 2 * p.B * p.Hq * p.D * 2
+    return kv + sc + qo
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of this GPU while the timed region runs."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self, max_fallback):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 8:
+                    rows.append(f)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": max_fallback, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = max([num(r[1]) for r in rows if num(r[1]) is not None] or [max_fallback])
+        power = [num(r[2]) for r in rows if num(r[2]) is not None]
+        load = [s for s, pw in zip(sm, power) if pw is not None and pw > 200] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    import block_quantized_precision_b200 as qa
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    pk, pk_kind = peaks()
+    hbm_peak = pk["hbm_gbs"]
+    int8_peak = 2.0 * pk["bf16_tflops"]        # INT8/FP8 dense = 2 x bf16 dense (nominal ratio)
+    fp32_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12   # FMA pipe, TFLOP/s
+    launches = [0]
+
+    def cu(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    # ---------------- the step: INT8 causal prefill path ----------------
+    p = synth.INT8_CAUSAL
+    d = synth.make_prefill(p)
+    host = {n: torch.from_numpy(d[n].view(np.int16)).pin_memory() for n in ("q", "k", "v")}
+    x = {n: host[n].to(dev).view(torch.bfloat16) for n in host}
+    rot = cu(d["rot"])
+    nqb, nkb = -(-p.N // 128), -(-p.N // 256)
+    shp = p.shape()
+    bufs = {
+        "qc": torch.empty(shp, dtype=torch.uint8, device=dev), "qs": torch.empty((p.B, p.H, nqb), device=dev),
+        "kc": torch.empty(shp, dtype=torch.uint8, device=dev), "ks": torch.empty((p.B, p.H, nkb), device=dev),
+        "vc": torch.empty(shp, dtype=torch.uint8, device=dev), "vs": torch.empty((p.B, p.H, nkb), device=dev),
+        "out": torch.empty(shp, dtype=torch.bfloat16, device=dev),
+    }
+    out_host = torch.empty(shp, dtype=torch.bfloat16).pin_memory()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
+    names = ["rotq_q", "rotq_k", "quant_v", "prefill"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, p.code_dtype, bufs["qc"], bufs["qs"])
+        mark(1)
+        qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, p.code_dtype, bufs["kc"], bufs["ks"])
+        mark(2)
+        qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, p.code_dtype, bufs["vc"], bufs["vs"])
+        mark(3)
+        qa.qattn_prefill(bufs["qc"], bufs["qs"], bufs["kc"], bufs["ks"], bufs["vc"], bufs["vs"], p.code_dtype,
+                         p.layout, p.causal, out=bufs["out"])
+        mark(4)
+        launches[0] += 4
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    uuid = "GPU-" + str(props.uuid) if getattr(props, "uuid", None) else None
+    launches[0] = 0
+    with ClockSampler(uuid) as clk:
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        barrier()
+    clocks = clk.summary(pk.get("sm_max_mhz", 1965.0))
+    step_launches = launches[0]
+    per = np.array([[evs[i][k].elapsed_time(evs[i][k + 1]) for k in range(4)] for i in range(args.steps)])
+    step_ms = per.sum(axis=1)
+    t = torch.tensor([float(step_ms.mean())], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    value = world * ops / (ms * 1e-3) / 1e12
+    kern_ms = per.mean(axis=0)
+    qk_rows = p.B * p.H * p.N
+    kernels = {
+        "rotq_q": {"ms": kern_ms[0], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (kern_ms[0] * 1e-3) / 1e12,
+                   "peak": fp32_peak, "unit": "TFLOP/s"},
+        "rotq_k": {"ms": kern_ms[1], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (kern_ms[1] * 1e-3) / 1e12,
+                   "peak": fp32_peak, "unit": "TFLOP/s"},
+        "quant_v": {"ms": kern_ms[2], "bound": "hbm", "achieved": qk_rows * p.D * 3 / (kern_ms[2] * 1e-3) / 1e9,
+                    "peak": hbm_peak, "unit": "GB/s"},
+        "prefill": {"ms": kern_ms[3], "bound": "tensor", "achieved": ops / (kern_ms[3] * 1e-3) / 1e12,
+                    "peak": int8_peak, "unit": "TOPS"},
+    }
+    for k in kernels.values():
+        k["frac"] = k["achieved"] / k["peak"]
+        k["ms"] = float(k["ms"])
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    traffic = load_traffic(dom)
+    roof = {"kernel": dom, "bound": kernels[dom]["bound"], "achieved": round(kernels[dom]["achieved"], 2),
+            "peak": kernels[dom]["peak"], "unit": kernels[dom]["unit"], "frac": round(kernels[dom]["frac"], 4),
+            "traffic": traffic, "peak_source": pk_kind + " (burst)"}
+
+    # ---------------- end to end through the C ABI with host buffers ----------------
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for n in ("q", "k", "v"):
+            x[n].view(torch.int16).copy_(host[n], non_blocking=True)
+        step()
+        out_host.copy_(bufs["out"], non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    h2d = sum(host[n].numel() * 2 for n in host)
+    d2h = out_host.numel() * 2
+    te = torch.tensor([float(np.mean(e2e_ms))], device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e = {"value": round(world * ops / (float(te.item()) * 1e-3) / 1e12, 3), "unit": "TOPS",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(float(te.item()), 4)}
+
+    extra = {}
+    if not args.no_extra:
+        extra = extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(p, d, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; shapes and distributions of the stated problem)",
+        "config": {"workload": p.name, "B": p.B, "H": p.H, "N": p.N, "D": p.D, "layout": "BNSD", "causal": True,
+                   "codes": "int8", "rotation": "seeded orthogonal 128x128 on Q and K",
+                   "l2": "flushed before every timed step (256 MB write)", "parallelism": "replicas" if world > 1 else "1 GPU"},
+        "roofline": roof,
+        "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in v.items()} for k, v in kernels.items()},
+        "e2e": e2e,
+        "gpu_launches": int(step_launches),
+        "clocks": clocks,
+        "extra": extra,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def load_traffic(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    capture (profiles/traffic.json), or None when there is none or the
+    kernel's source has changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f).get(kernel)
+        src = open(os.path.join(ROOT, t["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != t["sha256_16"]:
+            return None
+        return t["bytes"]
+    except Exception:
+        return None
+
+
+def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak):
+    import torch
+    res = {}
+    n = max(5, args.steps // 2)
+
+    def timeit(fn, reps, flush=None):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            if flush is not None:
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return float(np.mean(ts))
+
+    # decode, INT8 and packed INT4 caches (inputs far larger than L2)
+    for key, p in (("decode_int8kv", synth.INT8_KV_DECODE), ("decode_int4kv", synth.INT4_KV_DECODE)):
+        dd = synth.make_decode(p)
+        q = torch.from_numpy(dd["q"].view(np.int16)).to(dev).view(torch.bfloat16)
+        k = torch.from_numpy(dd["k"]).to(dev)
+        v = torch.from_numpy(dd["v"]).to(dev)
+        if p.kv_dtype == synth.INT8:
+            ks, vs, kvt = torch.from_numpy(dd["k_scales"]).to(dev), torch.from_numpy(dd["v_scales"]).to(dev), qa.QATTN_INT8
+        else:
+            ks = torch.from_numpy(dd["k_scales"].view(np.int16)).to(dev).view(torch.float16)
+            vs = torch.from_numpy(dd["v_scales"].view(np.int16)).to(dev).view(torch.float16)
+            kvt = qa.QATTN_INT4_PACKED
+        out = torch.empty((p.B, p.Hq, 1, p.D), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, qa.qattn_decode_workspace_size(p.B, p.Hq, p.Hkv, p.L, p.D)), dtype=torch.uint8, device=dev)
+        fn = lambda: qa.qattn_decode_kvq(q, k, v, ks, vs, kvt, kv_block=p.kv_block, group=p.group, out=out, workspace=ws)
+        ms = timeit(fn, n)
+        by = decode_bytes(p)
+        gbs = by / (ms * 1e-3) / 1e9
+        res[key] = {"workload": p.name, "ms": round(ms, 4), "GB/s": round(gbs, 1), "bytes": by,
+                    "roofline": {"bound": "hbm", "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
+        del k, v, dd
+        torch.cuda.empty_cache()
+
+    # FP8 long-sequence prefill path (inputs larger than L2)
+    p = synth.FP8_LONG
+    d = synth.make_prefill(p)
+    x = {nm: torch.from_numpy(d[nm].view(np.int16)).to(dev).view(torch.bfloat16) for nm in ("q", "k", "v")}
+    rot = torch.from_numpy(d["rot"]).to(dev)
+    codes = {nm: qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None,
+                                            128 if nm == "q" else 256, p.code_dtype) for nm in ("q", "k", "v")}
+    out = torch.empty(p.shape(), dtype=torch.bfloat16, device=dev)
+    pf = lambda: qa.qattn_prefill(codes["q"][0], codes["q"][1], codes["k"][0], codes["k"][1], codes["v"][0],
+                                  codes["v"][1], p.code_dtype, p.layout, p.causal, out=out)
+    ms_pf = timeit(pf, n)
+
+    def full():
+        for nm in ("q", "k", "v"):
+            qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
+                                        p.code_dtype, codes[nm][0], codes[nm][1])
+        pf()
+    ms_full = timeit(full, n)
+    ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
+    res["prefill_fp8_long"] = {"workload": p.name, "ms_prefill": round(ms_pf, 4), "ms_path": round(ms_full, 4),
+                               "TFLOPS_prefill": round(ops / (ms_pf * 1e-3) / 1e12, 1),
+                               "TFLOPS_path": round(ops / (ms_full * 1e-3) / 1e12, 1),
+                               "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TFLOP/s",
+                                            "frac": round(ops / (ms_pf * 1e-3) / 1e12 / int8_peak, 4)}}
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(p, d, heads):
+    """The oracle on `heads` of the workload: its own rotate+quantize of Q,
+    K, V and quantized attention for every row of those heads."""
+    import oracle
+    hs = [(0, h) for h in range(heads)]
+    oq = oracle.rotate_block_quant(d["q"], p.in_dtype, p.layout, d["rot"], 128, p.code_dtype, heads=hs)
+    ok_ = oracle.rotate_block_quant(d["k"], p.in_dtype, p.layout, d["rot"], 256, p.code_dtype, heads=hs)
+    ov = oracle.rotate_block_quant(d["v"], p.in_dtype, p.layout, None, 256, p.code_dtype, heads=hs)
+    rows = {(b, h): list(range(p.N)) for (b, h) in hs}
+    oracle.prefill_rows(*oq, *ok_, *ov, p.code_dtype, p.layout, p.causal, rows, row_chunk=128)
+
+
+def cpu_baseline(p, d, target_s):
+    """The oracle on the whole workload when that fits the time budget (it
+    takes a few seconds on 8 cores), else on as many heads as fit."""
+    import oracle
+    oracle.build()
+    cores = oracle.threads()
+    t0 = time.perf_counter()
+    oracle_sample(p, d, 1)
+    one = time.perf_counter() - t0
+    heads = int(max(1, min(p.H, target_s / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    oracle_sample(p, d, heads)
+    dt = time.perf_counter() - t0
+    ops = prefill_ops(1, heads, p.N, p.D, p.causal)
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": "%d of %d heads of %s (all rows: rotate+quantize Q/K/V and quantized attention), %.1f s"
+                      % (heads, p.H, p.name, dt)}
+
+
+def reference_arm(args):
+    """Reference arm: the CPU oracle as it stands, each step a bounded sample
+    (args.ref_heads heads, every row) of the same workload."""
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    p = synth.INT8_CAUSAL
+    d = synth.make_prefill(p)
+    import oracle
+    oracle.build()
+    cores = oracle.threads()
+    heads = args.ref_heads
+    for _ in range(args.warmup):
+        oracle_sample(p, d, heads)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_sample(p, d, heads)
+        ts.append(time.perf_counter() - t0)
+    ms = float(np.mean(ts)) * 1e3
+    ops = prefill_ops(1, heads, p.N, p.D, p.causal)
+    value = ops / (ms * 1e-3) / 1e12
+    sample = "%d of %d heads of %s per step (all rows: rotate+quantize Q/K/V and quantized attention)" % (
+        heads, p.H, p.name)
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": p.name, "B": p.B, "H": p.H, "N": p.N, "D": p.D, "layout": "BNSD", "causal": True},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def profile_case(args):
+    """Runs one workload (warmup + steps launches, no timing, no JSON): the
+    command line that the ncu summaries under profiles/ were captured with."""
+    import torch
+
+    import block_quantized_precision_b200 as qa
+    import synth
+    dev = torch.device("cuda", 0)
+    c = args.case
+    if c.startswith("decode"):
+        p = synth.INT8_KV_DECODE if c == "decode_int8kv" else synth.INT4_KV_DECODE
+        dd = synth.make_decode(p)
+        q = torch.from_numpy(dd["q"].view(np.int16)).to(dev).view(torch.bfloat16)
+        k, v = torch.from_numpy(dd["k"]).to(dev), torch.from_numpy(dd["v"]).to(dev)
+        if p.kv_dtype == synth.INT8:
+            ks, vs, kvt = torch.from_numpy(dd["k_scales"]).to(dev), torch.from_numpy(dd["v_scales"]).to(dev), qa.QATTN_INT8
+        else:
+            ks = torch.from_numpy(dd["k_scales"].view(np.int16)).to(dev).view(torch.float16)
+            vs = torch.from_numpy(dd["v_scales"].view(np.int16)).to(dev).view(torch.float16)
+            kvt = qa.QATTN_INT4_PACKED
+        for _ in range(args.warmup + args.steps):
+            qa.qattn_decode_kvq(q, k, v, ks, vs, kvt, kv_block=p.kv_block, group=p.group)
+    else:
+        p = synth.INT8_CAUSAL if c == "prefill_int8" else synth.FP8_LONG
+        d = synth.make_prefill(p)
+        x = {n: torch.from_numpy(d[n].view(np.int16)).to(dev).view(torch.bfloat16) for n in ("q", "k", "v")}
+        rot = torch.from_numpy(d["rot"]).to(dev)
+        for _ in range(args.warmup + args.steps):
+            qc = qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, p.code_dtype)
+            kc = qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, p.code_dtype)
+            vc = qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, p.code_dtype)
+            qa.qattn_prefill(*qc, *kc, *vc, p.code_dtype, p.layout, p.causal)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    print("case %s: ok" % c)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode / FP8 measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--ref-heads", type=int, default=4, help="heads per reference-arm step")
+    ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "decode_int8kv", "decode_int4kv"],
+                    help="run one workload only (for profiler captures); prints no JSON")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.case:
+        profile_case(args)
+    elif args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

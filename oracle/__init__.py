@@ -166,12 +166,15 @@ def rotate_block_quant(x_bits: np.ndarray, x_dtype: int, layout: int, rot, block
 
 def prefill_rows(qc, qs, kc, ks, vc, vs, code_dtype: int, layout: int, causal: bool,
                  rows_by_head: dict, q_block=128, kv_block=256, kv_tile=128,
-                 softmax_scale=0.0, p_quant=True, Nkv=None, want_f64=False, want_lse=False):
+                 softmax_scale=0.0, p_quant=True, Nkv=None, want_f64=False, want_lse=False,
+                 row_chunk=None):
     """Output rows of quantized attention.
 
     qc/kc/vc: codes (uint8 for INT8/FP8 -- INT8 codes as their byte pattern --
     or float32 for F32), shaped like the layout. rows_by_head: {(b, h): [rows]}.
-    Returns {(b, h): (bf16 bits [n, D], f64 [n, D] or None, lse [n] or None)}.
+    row_chunk: optional number of rows per parallel job (default: one job per
+    head). Returns {(b, h): (bf16 bits [n, D], f64 [n, D] or None, lse [n] or
+    None)}.
     """
     if layout == BNSD:
         B, H, Nq, D = qc.shape
@@ -193,10 +196,17 @@ def prefill_rows(qc, qs, kc, ks, vc, vs, code_dtype: int, layout: int, causal: b
         of = np.empty((len(r), D), dtype=np.float64) if want_f64 else None
         ls = np.empty(len(r), dtype=np.float64) if want_lse else None
         res[(b, h)] = (ob, of, ls)
-        jobs.append(lambda b=b, h=h, r=r, ob=ob, of=of, ls=ls: L.orc_prefill_rows(
-            _p(arrs[0]), _p(arrs[1]), _p(arrs[2]), _p(arrs[3]), _p(arrs[4]), _p(arrs[5]),
-            code_dtype, layout, B, H, Nq, Nk, D, q_block, kv_block, kv_tile, int(causal),
-            float(softmax_scale), int(p_quant), b, h, _p(r), len(r), _p(ob), _p(of), _p(ls)))
+        step = row_chunk or max(1, len(r))
+        for s0 in range(0, len(r), step):
+            s1 = min(len(r), s0 + step)
+            rr = r[s0:s1]
+            obs = ob[s0:s1]
+            ofs = of[s0:s1] if of is not None else None
+            lss = ls[s0:s1] if ls is not None else None
+            jobs.append(lambda b=b, h=h, rr=rr, obs=obs, ofs=ofs, lss=lss: L.orc_prefill_rows(
+                _p(arrs[0]), _p(arrs[1]), _p(arrs[2]), _p(arrs[3]), _p(arrs[4]), _p(arrs[5]),
+                code_dtype, layout, B, H, Nq, Nk, D, q_block, kv_block, kv_tile, int(causal),
+                float(softmax_scale), int(p_quant), b, h, _p(rr), len(rr), _p(obs), _p(ofs), _p(lss)))
     _run_all(jobs)
     return res
 
