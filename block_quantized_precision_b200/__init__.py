@@ -7,7 +7,8 @@ fails, an exception is raised.
 
 Function names follow the C ABI:
     qattn_rotate_block_quant, qattn_prefill, qattn_decode_workspace_size,
-    qattn_decode_kvq, qattn_device_error, qattn_selftest_wait_timeout,
+    qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_device_error,
+    qattn_selftest_wait_timeout,
     qattn_abi_version, qattn_status_string.
 """
 from __future__ import annotations
@@ -32,8 +33,11 @@ QATTN_BNSD, QATTN_BSND = 0, 1
 QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 3, 4
 
 EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
-            "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_device_error",
-            "qattn_selftest_wait_timeout")
+            "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc",
+            "qattn_device_error", "qattn_selftest_wait_timeout")
+
+# Fixed scratch of qattn_decode_kvq_noalloc (bytes).
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 _lib = None
 
@@ -61,6 +65,8 @@ def lib() -> C.CDLL:
         L.qattn_decode_workspace_size.argtypes, L.qattn_decode_workspace_size.restype = [i, i, i, i, i], z
         L.qattn_decode_kvq.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, P, P, z, P]
         L.qattn_decode_kvq.restype = i
+        L.qattn_decode_kvq_noalloc.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, P, P]
+        L.qattn_decode_kvq_noalloc.restype = i
         L.qattn_device_error.argtypes, L.qattn_device_error.restype = [P], i
         L.qattn_selftest_wait_timeout.argtypes, L.qattn_selftest_wait_timeout.restype = [i, P], i
         _lib = L
@@ -160,6 +166,26 @@ def qattn_decode_kvq(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: int, kv_
                                 B, Hq, Hkv, L, D, kv_block, group, float(softmax_scale), _ptr(out),
                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "qattn_decode_kvq")
+    return out
+
+
+def qattn_decode_kvq_noalloc(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: int, kv_block: int = 256,
+                             group: int = 128, softmax_scale: float = 0.0, out=None, stream=None):
+    """qattn_decode_kvq with the split partials in the library's fixed 4 MiB
+    device array instead of a caller workspace: for callers that cannot
+    allocate device memory on their decode path. Calls must not overlap on
+    the GPU (they share the array); make the first call on a device before
+    any stream capture. The output tensor is the caller's: pass `out` to
+    avoid allocating it here."""
+    import torch
+    B, Hq, _, D = q.shape
+    Hkv, L = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=q.device)
+    st = lib().qattn_decode_kvq_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+                                        kv_dtype, B, Hq, Hkv, L, D, kv_block, group, float(softmax_scale),
+                                        _ptr(out), _stream(stream))
+    _check(st, "qattn_decode_kvq_noalloc")
     return out
 
 

@@ -198,6 +198,32 @@ qattn_status_t qattn_decode_kvq(const void* q, const void* k_cache, const void* 
                                 void* workspace, size_t workspace_bytes, qattn_stream_t stream);
 
 /*
+ * qattn_decode_kvq without a workspace argument: the split partials go to a
+ * fixed 4 MiB device array inside the library (4194304 bytes, held on every
+ * GPU that loads the library until the process exits). No counterpart on
+ * the pages; it exists for callers that cannot allocate device memory on
+ * their decode path -- their memory is reserved up front by an allocator
+ * they do not own, or a cudaMalloc/cudaFree there could synchronise the
+ * device and stall other streams. The caller still passes inputs and output.
+ *
+ * Arguments and results are those of qattn_decode_kvq. Sizes whose workspace
+ * (qattn_decode_workspace_size) exceeds 4 MiB are rejected with
+ * QATTN_ERR_WORKSPACE before anything is launched. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.
+ * Nothing is allocated or freed, ever. Every call shares the one array and
+ * it keeps the last call's contents; nothing in it needs to start at zero
+ * (each call writes every partial before reading it). Calls that overlap on
+ * the GPU (different streams, or host threads without ordering) race on the
+ * array: serialise them.
+ */
+qattn_status_t qattn_decode_kvq_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                        const void* k_scales, const void* v_scales,
+                                        qattn_dtype_t kv_dtype, int B, int H_q, int H_kv, int L,
+                                        int D, int kv_block, int group, float softmax_scale,
+                                        void* out, qattn_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the per-device error word that
  * kernels set when a bounded barrier wait runs out. Returns QATTN_OK,
  * QATTN_ERR_TIMEOUT, or QATTN_ERR_CUDA if the synchronisation itself failed.
