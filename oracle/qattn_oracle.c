@@ -421,15 +421,19 @@ int orc_exact_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int 
  * One query token of one (b, h_q) against the KV cache of kv head
  * h_kv = h_q / (H_q / H_kv).
  *
- * INT8 cache ("INT8 量化算子", item 3 of the ops-transformer section: K/V
- * stored as INT8 and read without converting back to fp16; Q is INT8 too):
+ * The query is quantized per (b, h_q) for both cache types:
  *   sq     = max_d |q[d]| / 127 (float32), qcode[d] = RNE(q[d] / sq) (float32
  *            division), clamped to [-127, 127]; sq == 0 gives zero codes
+ * INT8 cache ("INT8 量化算子", item 3 of the ops-transformer section: K/V
+ * stored as INT8 and read without converting back to fp16; Q is INT8 too):
  *   s_t    = (sum_d qcode[d] kcode[t][d]) * sq * sK[t / kv_block] * scale
  *   v_t[d] = vcode[t][d] * sV[t / kv_block]
  * Packed INT4 cache (two codes per byte, element 2i low nibble; one fp16
- * scale per token per group of `group` elements along D):
- *   s_t    = sum_g sK[t][g] * sum_{d in g} q[d] kcode[t][d] * scale  (q as float)
+ * scale per token per group of `group` elements along D): the nibbles are
+ * widened to INT8 and multiplied with the same INT8 query codes ("FlashAttention
+ * 的 INT8/INT4 量化", 第二层: INT4 is converted to INT8 before the matrix
+ * multiply; "INT8 量化算子": the query is INT8 too):
+ *   s_t    = sum_g sK[t][g] * (sum_{d in g} qcode[d] kcode[t][d]) * sq * scale
  *   v_t[d] = vcode[t][d] * sV[t][d / group]
  * Softmax over all L keys (probabilities are not quantized), float64:
  *   out = sum_t p_t v_t / sum_t p_t with p_t = exp(s_t - max s), rounded to
@@ -459,7 +463,7 @@ int orc_decode_one(const uint16_t* q, const void* kc, const void* vc, const void
   double* ls = (double*)malloc(sizeof(double) * splits);
   if (!qf || !O || !ms || !ls) { free(qf); free(O); free(ms); free(ls); return 2; }
   float sq = 0.0f;
-  if (kv_dtype == ORC_INT8) {
+  {
     float amax = 0.0f;
     for (int d = 0; d < D; ++d) {
       float a = fabsf(orc_bf16_to_f32(qrow[d]));
@@ -475,8 +479,6 @@ int orc_decode_one(const uint16_t* q, const void* kc, const void* vc, const void
       }
       qf[d] = (double)c;
     }
-  } else {
-    for (int d = 0; d < D; ++d) qf[d] = (double)orc_bf16_to_f32(qrow[d]);
   }
   int nkb = (L + kv_block - 1) / kv_block;
   int ngroups = D / group;
@@ -500,14 +502,14 @@ int orc_decode_one(const uint16_t* q, const void* kc, const void* vc, const void
         const uint16_t* skr = (const uint16_t*)ksc + (head * L + t) * ngroups;
         s = 0.0;
         for (int g = 0; g < ngroups; ++g) {
-          double part = 0.0;
+          int64_t part = 0;
           for (int d = g * group; d < (g + 1) * group; ++d) {
             int c = (d & 1) ? orc_int4_hi(kr[d / 2]) : orc_int4_lo(kr[d / 2]);
-            part += qf[d] * c;
+            part += (int64_t)qf[d] * c;
           }
-          s += part * (double)orc_f16_to_f32(skr[g]);
+          s += (double)part * (double)orc_f16_to_f32(skr[g]);
         }
-        s *= (double)softmax_scale;
+        s *= (double)sq * (double)softmax_scale;
       }
       double m_new = s > m ? s : m;
       double alpha = exp(m - m_new);

@@ -3,7 +3,9 @@
 INT8 cache read directly with an INT8 query: "INT8 量化算子" page,
 ops-transformer section, item 3 (KV Cache 也量化) and its Int8Attention
 listing. Packed INT4 with one fp16 scale per group of 128 elements:
-"ops-transformer INT8/INT4 量化推理" page, 5.1 and 5.2.
+"ops-transformer INT8/INT4 量化推理" page, 5.1 and 5.2; the nibbles are
+widened to INT8 and meet the same INT8 query codes ("FlashAttention 的
+INT8/INT4 量化", 第二层).
 
 CPU only.
 """
@@ -24,6 +26,14 @@ def _np_softmax_av(scores, vals):
     s = scores - scores.max()
     p = np.exp(s)
     return (p[:, None] * vals).sum(0) / p.sum()
+
+
+def _q_codes(q_bits):
+    """Per-head INT8 query codes and scale with torch float32 arithmetic
+    (absmax / 127, division, round half to even, clamp)."""
+    q = torch.from_numpy(synth.bf16_bits_to_f32(q_bits))
+    sq = q.abs().max() / 127.0
+    return torch.round(q / sq).clamp(-127, 127).numpy().astype(np.int64), float(sq)
 
 
 def _unpack_int4(b):
@@ -66,13 +76,13 @@ def test_int4_decode_matches_closed_form(orc):
                          p.Hkv, heads=heads, want_f64=True)
     g = p.Hq // p.Hkv
     for (b, h) in heads:
-        q = synth.bf16_bits_to_f32(d["q"][b, h, 0]).astype(np.float64)
+        qc, sq = _q_codes(d["q"][b, h, 0])
         kh = h // g
-        kc = _unpack_int4(d["k"][b, kh]).astype(np.float64)
+        kc = _unpack_int4(d["k"][b, kh]).astype(np.int64)
         vc = _unpack_int4(d["v"][b, kh]).astype(np.float64)
         ksc = d["k_scales"][b, kh].view(np.float16).astype(np.float64)      # [L, 1]
         vsc = d["v_scales"][b, kh].view(np.float16).astype(np.float64)
-        s = (kc @ q) * ksc[:, 0] * _scale32(p.D)
+        s = (kc @ qc).astype(np.float64) * ksc[:, 0] * sq * _scale32(p.D)
         ref = _np_softmax_av(s, vc * vsc[:, [0]])
         assert np.abs(of[b, h, 0] - ref).max() <= 1e-12 * np.abs(vc * vsc[:, [0]]).max()
 
@@ -87,13 +97,14 @@ def test_int4_group_scales_apply_per_group(orc):
     ks = synth.f64_to_f16_bits(rng.uniform(0.01, 0.05, (B, Hkv, L, D // G)))
     vs = synth.f64_to_f16_bits(rng.uniform(0.01, 0.05, (B, Hkv, L, D // G)))
     _, of = orc.decode(q, k, v, ks, vs, synth.INT4_PACKED, Hkv, group=G, want_f64=True)
-    kc = _unpack_int4(k[0, 0]).astype(np.float64)
+    kc = _unpack_int4(k[0, 0]).astype(np.int64)
     vc = _unpack_int4(v[0, 0]).astype(np.float64)
-    ksc = np.repeat(ks[0, 0].view(np.float16).astype(np.float64), G, axis=1)
+    ksg = ks[0, 0].view(np.float16).astype(np.float64)                        # [L, groups]
     vsc = np.repeat(vs[0, 0].view(np.float16).astype(np.float64), G, axis=1)
     for h in range(Hq):
-        qf = synth.bf16_bits_to_f32(q[0, h, 0]).astype(np.float64)
-        s = ((kc * ksc) @ qf) * _scale32(D)
+        qc, sq = _q_codes(q[0, h, 0])
+        part = np.stack([kc[:, g * G:(g + 1) * G] @ qc[g * G:(g + 1) * G] for g in range(D // G)], axis=1)
+        s = (part.astype(np.float64) * ksg).sum(axis=1) * sq * _scale32(D)
         ref = _np_softmax_av(s, vc * vsc)
         assert np.abs(of[0, h, 0] - ref).max() <= 1e-12
 
