@@ -32,6 +32,8 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include <climits>
+
 #include "qattn_device.cuh"
 #include "qattn_internal.h"
 
@@ -45,6 +47,7 @@ constexpr int kTileN = 128;   // keys per tile
 constexpr int kStagesKV = 2;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;
+constexpr int kMaxBlk = 512;  // K/V block scales staged in shared memory (keys up to 131072)
 
 struct PrefillParams {
   const float* qs;
@@ -70,6 +73,21 @@ struct Smem {
   static constexpr int kEnd = kV + kStagesKV * kTileBytes;
   static constexpr int kBytes = kEnd + 1024;          // slack for 1024-byte alignment
 };
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// acc + lo + hi of a half2 (bits of `h2`), float32 accumulation.
+__device__ __forceinline__ float add_f32_f16x2(uint32_t h2, float acc) {
+  float r;
+  asm("{\n\t.reg .f16 lo, hi;\n\t.reg .f32 t;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.f16 t, lo, %2;\n\tadd.rn.f32.f16 %0, hi, t;\n\t}"
+      : "=f"(r) : "r"(h2), "f"(acc));
+  return r;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -109,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ __align__(8) uint64_t bar_s_full, bar_p_full, bar_pv_full, bar_free, bar_drain;
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
+  __shared__ float sKsc[kMaxBlk], sVsc[kMaxBlk];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -227,6 +246,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int qrow = q0 + r;
     const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float sq = p.qs[static_cast<int64_t>(bh) * p.nqb + qt];
+    // K/V block scales of this head, staged once (beyond kMaxBlk blocks they
+    // are read from global memory).
+    for (int i = threadIdx.x - 64; i < min(p.nkb, kMaxBlk); i += 128) {
+      sKsc[i] = p.ks[static_cast<int64_t>(bh) * p.nkb + i];
+      sVsc[i] = p.vs[static_cast<int64_t>(bh) * p.nkb + i];
+    }
+    named_bar_sync(1, 128);
     float m_run = -CUDART_INF_F, l_run = 0.0f;
     uint8_t* prow = sP + r * 128;
     const int rsw = r & 7;
@@ -235,28 +261,62 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_s_full, j & 1, &abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
-      const float ksc = sq * p.ks[static_cast<int64_t>(bh) * p.nkb + (j >> 1)] * p.scale_log2;
+      const int blk = j >> 1;
+      const float kscale = blk < kMaxBlk ? sKsc[blk] : p.ks[static_cast<int64_t>(bh) * p.nkb + blk];
+      const float vscale = blk < kMaxBlk ? sVsc[blk] : p.vs[static_cast<int64_t>(bh) * p.nkb + blk];
+      const float ksc = sq * kscale * p.scale_log2;
       const int key0 = j * kTileN;
+      // Only the last tile (ragged N_kv) and the causal diagonal tile have
+      // masked keys; the mask is applied on those tiles only (warp-uniform).
+      const bool partial = (key0 + kTileN > p.Nkv) || (p.causal && key0 + kTileN - 1 > q0);
       int kmax = p.Nkv - key0;                    // keys valid for this row: [0, kmax)
       if (p.causal) kmax = min(kmax, qrow - key0 + 1);
-      // pass 1: row max of the scaled scores
-      float tmax = -CUDART_INF_F;
+
+      // ---- pass 1: row max (integer max of the INT32 scores, or float max) ----
+      float tmax;
+      if constexpr (kInt8) {
+        int im = INT_MIN;
 #pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + c * 32, v);
-        tmem_wait_ld();
+        for (int c = 0; c < kTileN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(trow + c * 32, v);
+          tmem_wait_ld();
+          if (partial) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float sv = kInt8 ? static_cast<float>(static_cast<int>(v[e])) : __uint_as_float(v[e]);
-          if (c * 32 + e < kmax) tmax = fmaxf(tmax, sv * ksc);
+            for (int e = 0; e < 32; ++e) im = max(im, c * 32 + e < kmax ? static_cast<int>(v[e]) : INT_MIN);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) im = max(im, static_cast<int>(v[e]));
+          }
         }
+        tmax = im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
+      } else {
+        float fm = -CUDART_INF_F;
+#pragma unroll 1
+        for (int c = 0; c < kTileN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(trow + c * 32, v);
+          tmem_wait_ld();
+          if (partial) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+              fm = fmax3(fm, c * 32 + e < kmax ? __uint_as_float(v[e]) : -CUDART_INF_F,
+                         c * 32 + e + 1 < kmax ? __uint_as_float(v[e + 1]) : -CUDART_INF_F);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) fm = fmax3(fm, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+          }
+        }
+        tmax = fm * ksc;
       }
       const float m_new = fmaxf(m_run, tmax);
       const float alpha = ex2(m_run - m_new);     // 0 on the first tile
-      // pass 2: probabilities, 8-bit rounding, P to shared memory
-      float rowsum = 0.0f;
-      int rowsum_i = 0;
+      const float2 k2 = make_float2(ksc, ksc);
+      const float2 nm2 = make_float2(-m_new, -m_new);
+
+      // ---- pass 2: probabilities, 8-bit rounding, P to shared memory ----
+      float rs0 = 0.0f, rs1 = 0.0f;
+      int rsum_i = 0;
 #pragma unroll 1
       for (int c = 0; c < kTileN / 32; ++c) {
         uint32_t v[32];
@@ -265,31 +325,45 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint32_t packed[8];
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-          float pr[4];
+          float2 t01, t23;
+          if constexpr (kInt8) {
+            // exact INT32 -> float32: 1.5 * 2^23 + S has S in its low mantissa bits
+            const float2 f01 = fadd2(make_float2(__int_as_float(static_cast<int>(v[4 * w]) + 0x4B400000),
+                                                 __int_as_float(static_cast<int>(v[4 * w + 1]) + 0x4B400000)),
+                                     make_float2(-12582912.0f, -12582912.0f));
+            const float2 f23 = fadd2(make_float2(__int_as_float(static_cast<int>(v[4 * w + 2]) + 0x4B400000),
+                                                 __int_as_float(static_cast<int>(v[4 * w + 3]) + 0x4B400000)),
+                                     make_float2(-12582912.0f, -12582912.0f));
+            t01 = ffma2(f01, k2, nm2);
+            t23 = ffma2(f23, k2, nm2);
+          } else {
+            t01 = ffma2(make_float2(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1])), k2, nm2);
+            t23 = ffma2(make_float2(__uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3])), k2, nm2);
+          }
+          float pr[4] = {ex2(t01.x), ex2(t01.y), ex2(t23.x), ex2(t23.y)};
+          if (partial) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = c * 32 + w * 4 + e;
-            const float sv = kInt8 ? static_cast<float>(static_cast<int>(v[w * 4 + e])) : __uint_as_float(v[w * 4 + e]);
-            pr[e] = col < kmax ? ex2(sv * ksc - m_new) : 0.0f;
+            for (int e = 0; e < 4; ++e) pr[e] = c * 32 + w * 4 + e < kmax ? pr[e] : 0.0f;
           }
           if constexpr (kInt8) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int code = __float2int_rn(pr[e] * 127.0f);
-              rowsum_i += code;
-              word |= static_cast<uint32_t>(code) << (8 * e);
-            }
+            // code = RNE(p * 127): product rounded to float32, then the
+            // 1.5 * 2^23 addend rounds it to an integer (half to even)
+            const float2 q01 = fadd2(fmul2(make_float2(pr[0], pr[1]), make_float2(127.0f, 127.0f)),
+                                     make_float2(12582912.0f, 12582912.0f));
+            const float2 q23 = fadd2(fmul2(make_float2(pr[2], pr[3]), make_float2(127.0f, 127.0f)),
+                                     make_float2(12582912.0f, 12582912.0f));
+            const uint32_t b01 = __byte_perm(__float_as_uint(q01.x), __float_as_uint(q01.y), 0x0040);
+            const uint32_t b23 = __byte_perm(__float_as_uint(q23.x), __float_as_uint(q23.y), 0x0040);
+            const uint32_t word = __byte_perm(b01, b23, 0x5410);
+            rsum_i = __dp4a(static_cast<int>(word), 0x01010101, rsum_i);
             packed[w] = word;
           } else {
             const uint32_t lo = cvt_e4m3x2(pr[0], pr[1]);
             const uint32_t hi = cvt_e4m3x2(pr[2], pr[3]);
             packed[w] = lo | (hi << 16);
-            uint32_t h0 = cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo));
-            uint32_t h1 = cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi));
-            const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-            const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-            rowsum += (f0.x + f0.y) + (f1.x + f1.y);
+            // row sum of the rounded probabilities (exact values via fp16)
+            rs0 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rs0);
+            rs1 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rs1);
           }
         }
         // keys c*32 .. c*32+31 = 16-byte chunks 2c and 2c+1 of this row
@@ -300,18 +374,21 @@ __global__ void __launch_bounds__(kThreads, 2)
               make_uint4(packed[4 * hchunk], packed[4 * hchunk + 1], packed[4 * hchunk + 2], packed[4 * hchunk + 3]);
         }
       }
-      if constexpr (kInt8) rowsum = static_cast<float>(rowsum_i) * (1.0f / 127.0f);
+      const float rowsum = kInt8 ? static_cast<float>(rsum_i) * (1.0f / 127.0f) : rs0 + rs1;
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(&bar_p_full);
       l_run = l_run * alpha + rowsum;
       m_run = m_new;
 
-      // fold PV into O
+      // ---- fold PV into O: O = O * alpha + PV * c_j ----
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_pv_full, j & 1, &abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
-      const float cj = p.vs[static_cast<int64_t>(bh) * p.nkb + (j >> 1)] * (kInt8 ? (1.0f / 127.0f) : 1.0f);
+      const float cj = vscale * (kInt8 ? (1.0f / 127.0f) : 1.0f);
+      const float2 c2 = make_float2(cj, cj);
+      const float2 a2 = make_float2(alpha, alpha);
+      const bool unit_alpha = __all_sync(0xffffffffu, alpha == 1.0f);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t pv[32], o[32];
@@ -319,10 +396,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (j > 0) tmem_ld32(trow + kColO + c * 32, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = kInt8 ? static_cast<float>(static_cast<int>(pv[e])) : __uint_as_float(pv[e]);
-          const float prev = j > 0 ? __uint_as_float(o[e]) * alpha : 0.0f;
-          o[e] = __float_as_uint(fmaf(x, cj, prev));
+        for (int e = 0; e < 32; e += 2) {
+          float2 x;
+          if constexpr (kInt8) {
+            x = fadd2(make_float2(__int_as_float(static_cast<int>(pv[e]) + 0x4B400000),
+                                  __int_as_float(static_cast<int>(pv[e + 1]) + 0x4B400000)),
+                      make_float2(-12582912.0f, -12582912.0f));
+          } else {
+            x = make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
+          }
+          float2 y;
+          if (j == 0) {
+            y = fmul2(x, c2);
+          } else {
+            const float2 prev = make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1]));
+            y = ffma2(x, c2, unit_alpha ? prev : fmul2(prev, a2));
+          }
+          o[e] = __float_as_uint(y.x);
+          o[e + 1] = __float_as_uint(y.y);
         }
         tmem_st32(trow + kColO + c * 32, o);
       }

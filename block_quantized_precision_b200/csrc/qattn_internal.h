@@ -2,11 +2,18 @@
 // and the kernel files. Arguments arrive here already validated.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace qattn {
+
+// Encodes a TMA tensor map over 8-bit data (no interleave, zero fill out of
+// bounds) through the driver entry point; false if that fails. dims[0] is the
+// contiguous dimension; strides (bytes) are given for dims 1..rank-1.
+bool encode_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                   const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle);
 
 struct RotQuantArgs {
   const void* x;      // F16/BF16 bits

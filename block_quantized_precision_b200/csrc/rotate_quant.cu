@@ -29,7 +29,11 @@ namespace qattn {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;                 // quant_kernel
+template <int D>
+struct RotqThreads {
+  static constexpr int value = D == 128 ? 512 : 256;   // 16 warps per SM for D = 128
+};
 
 __device__ __forceinline__ void unpack8(uint4 v, bool is_bf16, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -45,19 +49,52 @@ __device__ __forceinline__ void unpack8(uint4 v, bool is_bf16, float (&f)[8]) {
   }
 }
 
-// Code byte of v = y / scale (scale > 0).
+// Code byte of RNE(y / scale) with y / scale rounded to float32 first, as
+// IEEE division gives it, computed without a division in almost every case.
+//
+// v0 = y * rcp with rcp = RN(1 / scale) is within 1.5 * 2^-23 |v| of the
+// correctly rounded quotient RN(y / scale) (two roundings of 2^-24 relative
+// each, plus the half ulp of the quotient itself). The code only depends on
+// which side of the nearest rounding boundary that quotient lies (a
+// half-integer for INT8, a midpoint between e4m3 values for FP8). When v0 is
+// farther than that bound from every boundary both give the same code; in
+// the rare remaining cases the IEEE quotient is computed (__fdiv_rn).
+//   INT8: |v| <= 127.5, so the bound is below 2.3e-5; v0 is trusted when
+//         its distance to the nearest integer is below 0.5 - 1e-4.
+//   e4m3: in the normal range the boundary sits where float32 mantissa bits
+//         19..0 equal 0x80000, and the bound is 3 units of bit 0; v0 is
+//         trusted when those bits are more than 16 units away from 0x80000.
+//         Below 2^-6 (e4m3 subnormals) the IEEE quotient is used.
+// Saturation needs no care: every value at or beyond +-448 gives +-448.
+// A scale below the smallest normal float32 (`slow`, uniform over the block)
+// breaks these bounds (the reciprocal loses precision or overflows), so such
+// blocks always take the IEEE quotient, clamped for INT8.
+__device__ __noinline__ float ieee_div(float y, float scale) { return __fdiv_rn(y, scale); }
+
 template <bool kInt8>
-__device__ __forceinline__ uint32_t code_of(float y, float scale) {
-  const float v = __fdiv_rn(y, scale);
+__device__ __forceinline__ uint32_t code_of(float y, float scale, float rcp, bool slow) {
+  if (slow) {
+    const float v = ieee_div(y, scale);
+    if constexpr (kInt8) return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(v)))) & 0xFFu;
+    else return cvt_e4m3x2(v, 0.0f) & 0xFFu;
+  }
+  const float v0 = y * rcp;
   if constexpr (kInt8) {
-    int c = __float2int_rn(v);
-    c = max(-127, min(127, c));
-    return static_cast<uint32_t>(c) & 0xFFu;
+    const float r = (v0 + 12582912.0f) - 12582912.0f;   // round half to even (|v0| < 2^22)
+    const float dist = fabsf(v0 - r);                   // exact
+    float v = v0;
+    if (dist > 0.4999f) v = ieee_div(y, scale);         // near a half-integer: decide exactly
+    const float t = v + 12582912.0f;                    // integer in the low mantissa bits
+    return __float_as_uint(t) & 0xFFu;                  // two's complement byte (|v| <= 127.5)
   } else {
+    const uint32_t b = __float_as_uint(v0) & 0x7FFFFFFFu;
+    const int near_mid = abs(static_cast<int>(b & 0xFFFFFu) - 0x80000) <= 16;
+    const float v = (b < 0x3C800000u || near_mid) ? ieee_div(y, scale) : v0;   // 2^-6 = 0x3C800000
     return cvt_e4m3x2(v, 0.0f) & 0xFFu;
   }
 }
 
+template <int kNT>
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -66,7 +103,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   __syncthreads();
   float m = 0.0f;
 #pragma unroll
-  for (int i = 0; i < kThreads / 32; ++i) m = fmaxf(m, red[i]);
+  for (int i = 0; i < kNT / 32; ++i) m = fmaxf(m, red[i]);
   __syncthreads();  // red[] may be reused
   return m;
 }
@@ -82,30 +119,34 @@ __device__ __forceinline__ int64_t row_offset(int layout, int H, int N, int D, i
 // With rotation
 // ---------------------------------------------------------------------------
 
-// Thread tile: kRows rows x 8 columns of y. Column group cg = tid % (D/8),
-// row group rg = tid / (D/8); rows rg*kRPT .. rg*kRPT + kRPT - 1.
+// Thread tile: kRPT rows x 8 columns of y. Column group cg = tid % (D/8)
+// owns columns 4cg..4cg+3 and D/2+4cg..D/2+4cg+3 (two float4 of each R row,
+// consecutive across the warp, so the R reads are free of bank conflicts);
+// row group rg = tid / (D/8) owns rows rg*kRPT .. rg*kRPT + kRPT - 1.
 template <int D, int T, bool kInt8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(RotqThreads<D>::value, 1)
     rotq_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
                 const float* __restrict__ rot, uint8_t* __restrict__ codes,
                 float* __restrict__ scales) {
+  constexpr int kNT = RotqThreads<D>::value;
   constexpr int kCG = D / 8;               // column groups
-  constexpr int kRG = kThreads / kCG;      // row groups
+  constexpr int kRG = kNT / kCG;           // row groups
   constexpr int kRPT = T / kRG;            // rows per thread
   constexpr int kXS = T + 4;               // padded row stride of the transposed x tile
   static_assert(kRPT % 4 == 0 && kRPT >= 4, "row tile");
   extern __shared__ __align__(16) float smem[];
   float* sR = smem;                        // [D][D]
   float* sX = smem + D * D;                // [D][kXS]: sX[k * kXS + r] = x[r][k]
-  __shared__ float red[kThreads / 32];
+  __shared__ float red[kNT / 32];
 
   const int tid = threadIdx.x;
-  for (int i = tid; i < D * D / 4; i += kThreads)
+  for (int i = tid; i < D * D / 4; i += kNT)
     reinterpret_cast<float4*>(sR)[i] = reinterpret_cast<const float4*>(rot)[i];
 
   const int nblk = (N + T - 1) / T;
   const int64_t total = static_cast<int64_t>(B) * H * nblk;
   const int cg = tid % kCG, rg = tid / kCG;
+  const int c0 = 4 * cg, c1 = D / 2 + 4 * cg;   // this thread's two column quads
   const float qmax = kInt8 ? 127.0f : 448.0f;
 
   for (int64_t blk_id = blockIdx.x; blk_id < total; blk_id += gridDim.x) {
@@ -118,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();  // sR ready (first pass); previous block's sX reads done
     // Stage x transposed: thread t handles token row (t % T) and a slice of
     // the 16-byte chunks, so consecutive threads write consecutive words.
-    for (int idx = tid; idx < T * kCG; idx += kThreads) {
+    for (int idx = tid; idx < T * kCG; idx += kNT) {
       const int r = idx % T, c = idx / T;
       float f[8];
       if (r < rows) {
@@ -133,25 +174,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    float acc[kRPT][8];
+    // acc[i][j]: row rg*kRPT + i, column (j < 4 ? c0 + j : c1 + j - 4); each
+    // is the float32 FMA chain over k ascending, two lanes per f32x2 FMA.
+    float2 acc[kRPT][4];
 #pragma unroll
     for (int i = 0; i < kRPT; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+      for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
 #pragma unroll 2
     for (int k = 0; k < D; ++k) {
-      const float4 r0 = *reinterpret_cast<const float4*>(sR + k * D + cg * 8);
-      const float4 r1 = *reinterpret_cast<const float4*>(sR + k * D + cg * 8 + 4);
-      const float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      const float4 r0 = *reinterpret_cast<const float4*>(sR + k * D + c0);
+      const float4 r1 = *reinterpret_cast<const float4*>(sR + k * D + c1);
+      const float2 rv[4] = {make_float2(r0.x, r0.y), make_float2(r0.z, r0.w), make_float2(r1.x, r1.y),
+                            make_float2(r1.z, r1.w)};
 #pragma unroll
       for (int i4 = 0; i4 < kRPT / 4; ++i4) {
         const float4 xv = *reinterpret_cast<const float4*>(sX + k * kXS + rg * kRPT + i4 * 4);
         const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+        for (int ii = 0; ii < 4; ++ii) {
+          const float2 x2 = make_float2(xs[ii], xs[ii]);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i4 * 4 + ii][j] = __fmaf_rn(xs[ii], rv[j], acc[i4 * 4 + ii][j]);
+          for (int j = 0; j < 4; ++j) acc[i4 * 4 + ii][j] = ffma2(x2, rv[j], acc[i4 * 4 + ii][j]);
+        }
       }
     }
 
@@ -159,24 +205,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < kRPT; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(acc[i][j]));  // padded rows are +0
-    const float amax = block_max(m, red);
+      for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(acc[i][j].x), fabsf(acc[i][j].y)));  // padded rows are +0
+    const float amax = block_max<kNT>(m, red);
     const float scale = __fdiv_rn(amax, qmax);
+    const float rcp = __frcp_rn(scale);
+    const bool slow = scale < 1.17549435e-38f;
     if (tid == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
 
 #pragma unroll
     for (int i = 0; i < kRPT; ++i) {
       const int r = rg * kRPT + i;
       if (r >= rows) continue;
-      uint32_t lo = 0, hi = 0;
+      uint32_t w0 = 0, w1 = 0;
       if (scale != 0.0f) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(acc[i][j], scale) << (8 * j);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(acc[i][j + 4], scale) << (8 * j);
+        for (int j = 0; j < 2; ++j) {
+          w0 |= code_of<kInt8>(acc[i][j].x, scale, rcp, slow) << (16 * j);
+          w0 |= code_of<kInt8>(acc[i][j].y, scale, rcp, slow) << (16 * j + 8);
+          w1 |= code_of<kInt8>(acc[i][j + 2].x, scale, rcp, slow) << (16 * j);
+          w1 |= code_of<kInt8>(acc[i][j + 2].y, scale, rcp, slow) << (16 * j + 8);
+        }
       }
-      *reinterpret_cast<uint2*>(codes + row_offset(layout, H, N, D, b, h, n0 + r) + cg * 8) =
-          make_uint2(lo, hi);
+      uint8_t* crow = codes + row_offset(layout, H, N, D, b, h, n0 + r);
+      *reinterpret_cast<uint32_t*>(crow + c0) = w0;
+      *reinterpret_cast<uint32_t*>(crow + c1) = w1;
     }
   }
 }
@@ -203,24 +255,30 @@ __global__ void __launch_bounds__(kThreads)
   const bool bf = is_bf16 != 0;
 
   uint4 v[kVec];
-  float m = 0.0f;
+  // all loads first (16 bytes each, in flight together), then the max
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const int idx = threadIdx.x + i * kThreads;
     const int r = idx / kCG, c = idx % kCG;
-    if (idx < T * kCG && r < rows) {
-      v[i] = __ldg(reinterpret_cast<const uint4*>(x + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8));
-      float f[8];
-      unpack8(v[i], bf, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
-    } else {
-      v[i] = make_uint4(0, 0, 0, 0);
-    }
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (idx < T * kCG && r < rows)
+      v[i] = __ldcs(reinterpret_cast<const uint4*>(x + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8));
   }
-  const float amax = block_max(m, red);
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    float f[8];
+    unpack8(v[i], bf, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+  }
+  const float amax = block_max<kThreads>(m, red);
   const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
+  const float rcp = __frcp_rn(scale);
+  const bool slow = scale < 1.17549435e-38f;
   if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
+  // (the rare exact-division fallback is an out-of-line call, which keeps
+  // this unrolled loop small enough for the instruction cache)
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const int idx = threadIdx.x + i * kThreads;
@@ -231,9 +289,9 @@ __global__ void __launch_bounds__(kThreads)
       uint32_t lo = 0, hi = 0;
       if (scale != 0.0f) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f[j], scale) << (8 * j);
+        for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f[j], scale, rcp, slow) << (8 * j);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f[j + 4], scale) << (8 * j);
+        for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f[j + 4], scale, rcp, slow) << (8 * j);
       }
       *reinterpret_cast<uint2*>(codes + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8) =
           make_uint2(lo, hi);
@@ -249,8 +307,8 @@ cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
   const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
-  k<<<grid, kThreads, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B, a.H,
-                                  a.N, a.rot, static_cast<uint8_t*>(a.codes), a.scales);
+  k<<<grid, RotqThreads<D>::value, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B,
+                                                a.H, a.N, a.rot, static_cast<uint8_t*>(a.codes), a.scales);
   return cudaGetLastError();
 }
 

@@ -167,13 +167,14 @@ size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D);
  * 量化推理", 5.1 (one fp16 scale per group of G elements) and 5.2 (two INT4
  * per byte, element 2i in the low nibble).
  *
- * Query head h uses KV head h / (H_q / H_kv).
- *   INT8 cache:  sq = max|q| / 127, qcode = RNE(q / sq) (float32, clamped to
- *                [-127, 127]); s_t = (qcode . kcode_t) * sq *
- *                k_scales[b,hk,t/kv_block] * softmax_scale;
- *                v_t = vcode_t * v_scales[b,hk,t/kv_block].
- *   INT4 cache:  s_t = sum_g k_scales[b,hk,t,g] * (q . kcode_t over group g)
- *                * softmax_scale with q in float32;
+ * Query head h uses KV head h / (H_q / H_kv). The query is quantized per
+ * head: sq = max|q| / 127, qcode = RNE(q / sq) (float32, clamped to
+ * [-127, 127]).
+ *   INT8 cache:  s_t = (qcode . kcode_t) * sq * k_scales[b,hk,t/kv_block]
+ *                * softmax_scale; v_t = vcode_t * v_scales[b,hk,t/kv_block].
+ *   INT4 cache:  the nibbles are widened to INT8 ("FlashAttention 的
+ *                INT8/INT4 量化", 第二层) and s_t = sum_g k_scales[b,hk,t,g] *
+ *                (qcode . kcode_t over group g) * sq * softmax_scale;
  *                v_t[d] = vcode_t[d] * v_scales[b,hk,t,d/group].
  *   out = bf16(sum_t p_t v_t / sum_t p_t), p_t = exp(s_t - max s) in float32.
  *
@@ -182,7 +183,7 @@ size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D);
  *           QATTN_INT4_PACKED: bytes [B, H_kv, L, D/2].
  * k_scales, v_scales: QATTN_INT8: float32 [B, H_kv, ceil(L/kv_block)];
  *           QATTN_INT4_PACKED: float16 [B, H_kv, L, D/group].
- * kv_block: 256 (INT8); group: 128 (INT4, must divide D).
+ * kv_block: 256 (INT8); group: 128 or 64 (INT4, must divide D).
  * softmax_scale: <= 0 selects 1/sqrt(D) (float32).
  * out:      bfloat16 [B, H_q, 1, D].
  * workspace / workspace_bytes: device scratch of at least

@@ -48,6 +48,35 @@ def test_small_shapes_bit_exact(orc, D, layout, code_dtype, rotate, block):
     _check_all(orc, x, synth.BF16, layout, rot, block, code_dtype)
 
 
+def test_rounding_ties_and_near_ties(orc):
+    """Blocks whose scale is exactly 1 (block max 127 for INT8, 448 for e4m3)
+    hold values on and next to the rounding boundaries of the codes (exact
+    half-integers, exact e4m3 midpoints, and their bf16 neighbours), so the
+    code decisions are exercised where a misrounded quotient would show; a
+    block with a subnormal scale and a signed permutation as rotation (which
+    moves values exactly) are included."""
+    D, T = 128, 128
+    for code, top in ((synth.INT8, 127.0), (synth.FP8_E4M3, 448.0)):
+        if code == synth.INT8:
+            base = np.arange(-126, 127) + 0.5
+        else:
+            import torch as _t
+            grid = np.unique(_t.arange(0, 127, dtype=_t.uint8).view(_t.float8_e4m3fn).float().numpy())
+            base = (grid[:-1].astype(np.float64) + grid[1:]) / 2
+            base = np.concatenate([base, -base])
+        bits = synth.f32_to_bf16_bits(base)
+        nb = np.concatenate([bits, bits + 1, bits - 1]).astype(np.uint16)      # ties and bf16 neighbours
+        vals = np.resize(nb, T * D).reshape(T, D)
+        vals[0, 0] = synth.f32_to_bf16_bits(np.array([top]))[0]
+        tiny = synth.f32_to_bf16_bits(np.random.default_rng(1).standard_normal((T, D)) * 1e-39)
+        x = np.stack([vals, tiny])[None]                                          # [1, 2, T, D]
+        perm = np.random.default_rng(2).permutation(D)
+        P = np.zeros((D, D), dtype=np.float32)
+        P[np.arange(D), perm] = 1.0
+        _check_all(orc, x, synth.BF16, synth.BNSD, None, T, code)
+        _check_all(orc, x, synth.BF16, synth.BNSD, P, T, code)
+
+
 def test_f16_input_and_edge_blocks(orc):
     B, H, N, D = 1, 2, 257, 128               # last block holds one token
     rng = np.random.default_rng(3)
