@@ -8,25 +8,35 @@
 // INT8/INT4 量化推理", 5.1 (group scales) and 5.2 (two codes per byte, even
 // element in the low nibble); the nibbles are widened to INT8 in registers
 // and meet the INT8 query ("FlashAttention 的 INT8/INT4 量化", 第二层).
-// Nothing is ever written back in fp16.
+// Nothing is ever written back in fp16 to global memory.
 //
 // decode_kernel: grid (splits, H_kv, B), 5 warps. Each CTA owns a contiguous
 // range of whole chunks of one (b, h_kv) and all G = H_q / H_kv query heads
 // that share it.
 //   warp 4      producer: K and V chunks (64 tokens INT8 / 128 tokens INT4)
-//               by TMA tensor loads with hardware swizzle into a 4-stage
-//               ring (no multicast).
+//               by TMA tensor loads with hardware swizzle into a ring (no
+//               multicast); it also stages each chunk's scales and the
+//               largest V scale of the chunk.
 //   warps 0-3   consumers, each on its own quarter of every chunk with its
-//               own running softmax (no block barrier per chunk), 16 tokens
-//               per step:
-//                 scores   lane pair per token, each lane half a row: dp4a on
-//                          the INT8 query codes held in registers (INT4
-//                          nibbles widened to bytes first), pair sum by shuffle
-//                 softmax  warp max by redux on order-preserving integer keys,
-//                          exp2, per-lane partial sums
-//                 P.V      lane = 4 channels x all heads; bytes/nibbles turned
-//                          into floats with byte-permute/magic-number tricks
-//                          on the ALU/FMA pipes, packed f32x2 FMAs
+//               own running softmax, 16 tokens per step, on the warp-level
+//               tensor-core instructions:
+//                 scores  S^T[16 tokens x 8 heads] = K Q^T by
+//                         mma.m16n8k32 s8 x s8 -> s32: key rows straight from
+//                         the swizzled tile (INT4 nibbles widened to bytes,
+//                         biased by +8 and corrected with the query code
+//                         sums); the query codes live in 8 registers
+//                 softmax per head over the 16 tokens (shuffles), running
+//                         max / sum in the log2 domain
+//                 P.V     O[heads x 128] += P' V' by mma.m16n8k16 f16 x f16
+//                         -> f32. P' = p * (v scale / running max v scale)
+//                         in [0, 1], split into an fp16 high part and an fp16
+//                         remainder (two MMAs, ~22 significant bits). V' is
+//                         the code plus a constant offset, exact in fp16 and
+//                         built with byte permutes only (odd INT4 channels
+//                         also carry a factor 16); the offsets are removed at
+//                         the end with sum(P'), which two more MMAs against a
+//                         tile of ones provide. V' goes through a per-warp
+//                         fp16 tile and ldmatrix.trans.
 //               then the four warps merge their states and write (O, m, l)
 //               of the range to the workspace (log2 domain).
 // merge_kernel: grid B*H_q, D threads: out = sum_s w_s O_s / sum_s w_s l_s,
@@ -48,17 +58,21 @@ namespace {
 constexpr int kD = 128;               // head size handled by this kernel
 constexpr int kConsumers = 4;         // consumer warps
 constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int kStages = 4;
 constexpr int kStep = 16;             // tokens per consumer step
 constexpr int kWsStride = kD + 4;     // floats per (b, h_q, split) partial: O[D], m, l, pad
+constexpr int kVhStride = kD + 8;     // halves per row of the per-warp V' tile (conflict-free ldmatrix)
+constexpr uint32_t kOnesF16x2 = 0x3C003C00u;
+constexpr int kCtasPerSm = 2;         // resident CTAs per SM (registers)
 
 template <bool kInt4>
 struct Cfg {
   static constexpr int kRowBytes = kInt4 ? kD / 2 : kD;
   static constexpr int kChunk = kInt4 ? 128 : 64;             // tokens per stage
+  static constexpr int kStages = kInt4 ? 3 : 4;
   static constexpr int kTileBytes = kChunk * kRowBytes;       // one tensor, one stage (8 KB)
   static constexpr int kPerWarp = kChunk / kConsumers;        // tokens per warp per chunk
-  static constexpr int kSmemBytes = 2 * kStages * kTileBytes + 1024;
+  static constexpr int kVhBytes = kConsumers * kStep * kVhStride * 2;
+  static constexpr int kSmemBytes = 2 * kStages * kTileBytes + kVhBytes + 1024;
 };
 
 struct DecodeParams {
@@ -81,58 +95,78 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Four signed bytes of w -> floats: byte b becomes the mantissa of
-// 2^23 + (b + 128), then 2^23 + 128 is subtracted (exact).
-__device__ __forceinline__ void s8x4_to_f32(uint32_t w, float2& lo, float2& hi) {
-  const uint32_t u = w ^ 0x80808080u;
-  const float2 off = make_float2(-8388736.0f, -8388736.0f);
-  lo = fadd2(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)),
-                         __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541))), off);
-  hi = fadd2(make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)),
-                         __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543))), off);
+// D[16x8] (+)= A[16x32] B[32x8]; signed 8-bit inputs, 32-bit accumulation.
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Four signed nibbles (bits 0..15 of w, element i in bits 4i..4i+3) ->
-// floats: 2^23 + (c + 8) built by one LOP3 each, then 2^23 + 8 subtracted.
-__device__ __forceinline__ void s4x4_to_f32(uint32_t w, float2& lo, float2& hi) {
-  const float2 off = make_float2(-8388616.0f, -8388616.0f);
-  lo = fadd2(make_float2(__uint_as_float((w & 0xFu) ^ 0x4B000008u), __uint_as_float(((w >> 4) & 0xFu) ^ 0x4B000008u)),
-             off);
-  hi = fadd2(make_float2(__uint_as_float(((w >> 8) & 0xFu) ^ 0x4B000008u),
-                         __uint_as_float(((w >> 12) & 0xFu) ^ 0x4B000008u)),
-             off);
+// D[16x8] += A[16x16] B[16x8], fp16 inputs, fp32 accumulation. Rows 8..15 of
+// A are zero here (at most 8 query heads), so only the first two accumulator
+// registers carry data; the other two are scratch.
+__device__ __forceinline__ void mma_f16(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  float z0 = 0.0f, z1 = 0.0f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c0), "+f"(c1), "+f"(z0), "+f"(z1)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Two fp16 parts of (x, y): high = RN_f16(x, y), low = RN_f16((x, y) - high).
+__device__ __forceinline__ void split_f16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x, y);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x - f.x, y - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 template <int G, bool kInt4, int kGroups>
-__global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
+  static_assert(G >= 1 && G <= 8, "query heads per kv head");
   using C = Cfg<kInt4>;
-  constexpr int kRowBytes = C::kRowBytes;
+  constexpr int kStages = C::kStages;
   constexpr int kTile = C::kTileBytes;
+  constexpr int kNAcc = (kInt4 && kGroups == 2) ? 2 : 1;      // score accumulators (one per INT4 group)
+  // V' = code + kOff (INT8, INT4 even channels) or 16 * (code + 8) + 1024
+  // (INT4 odd channels, kept in stored columns 4i+2, 4i+3).
+  constexpr float kOffA = kInt4 ? 1032.0f : 1152.0f;
+  constexpr float kOffB = 1152.0f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;                          // [stages][chunk rows], swizzled
   uint8_t* sV = smem + kStages * kTile;
+  __half* sVh = reinterpret_cast<__half*>(smem + 2 * kStages * kTile);   // [warp][16][kVhStride]
   float* sRed = reinterpret_cast<float*>(smem);   // after the loop: [warps][G][D]
 
   __shared__ __align__(16) uint32_t sQw[G][kD / 4];    // query codes, 4 per word (natural order)
-  __shared__ int sQsum[G][2];                          // INT4: sum of query codes per half row
+  __shared__ int sQsum[G][2];                          // sum of query codes per 64-channel half
   __shared__ float sQf[G];                             // sq * softmax scale * log2(e)
-  __shared__ __align__(16) float2 sP[kConsumers][kStep][G];  // (p, p) * v scale, per warp
-  __shared__ float sSV[kConsumers][kStep][2];          // INT4 with two groups: v scales
-  // Scales of each staged chunk, written by the producer warp: INT8 one K and
-  // one V block scale per chunk; INT4 one fp16 per token and group.
-  __shared__ float sKsc[kStages], sVsc[kStages];
+  __shared__ __align__(16) float sPw[kConsumers][kGroups][8][kStep];   // P'[head][token], per warp
+  __shared__ float sAlpha[kConsumers][8];
+  __shared__ float sKsc[kStages], sVsc[kStages], sVmax[kStages];
   __shared__ uint16_t sKs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
   __shared__ uint16_t sVs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
-  __shared__ float sWm[kConsumers][G], sWl[kConsumers][G];
+  __shared__ float sWm[kConsumers][8], sWl[kConsumers][8];
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
-  const int g = p.Hq / p.Hkv;
+  const int g_all = p.Hq / p.Hkv;
   const int64_t head = static_cast<int64_t>(b) * p.Hkv + hk;
   const int t_begin = split * p.chunks_per_split * C::kChunk;
   const int t_end = min(p.L, t_begin + p.chunks_per_split * C::kChunk);
@@ -147,10 +181,10 @@ __global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
     abort_flag = 0;
     mbar_fence_init();
   }
-  // Query codes of the G heads (consumer warps; warp w: heads w, w+4, ...).
+  // Query codes of the G heads (consumer warps; warp w: heads w, w+4).
   if (warp < kConsumers) {
     for (int hh = warp; hh < G; hh += kConsumers) {
-      const uint2 raw = *reinterpret_cast<const uint2*>(p.q + (static_cast<int64_t>(b) * p.Hq + hk * g + hh) * kD + lane * 4);
+      const uint2 raw = *reinterpret_cast<const uint2*>(p.q + (static_cast<int64_t>(b) * p.Hq + hk * g_all + hh) * kD + lane * 4);
       const float f[4] = {bf16f(raw.x & 0xFFFF), bf16f(raw.x >> 16), bf16f(raw.y & 0xFFFF), bf16f(raw.y >> 16)};
       float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
 #pragma unroll
@@ -166,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
         w |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * e);
       }
       sQw[hh][lane] = w;
-      // lanes 0..15 hold channels 0..63 (first half row), 16..31 the second
+      // lanes 0..15 hold channels 0..63, lanes 16..31 channels 64..127
       const int half_sum0 = __reduce_add_sync(0xffffffffu, lane < 16 ? csum : 0);
       const int half_sum1 = __reduce_add_sync(0xffffffffu, lane >= 16 ? csum : 0);
       if (lane == 0) {
@@ -224,13 +258,20 @@ __global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
         if (lane == 0) {
           sKsc[s] = ksc;
           sVsc[s] = vsc;
+          sVmax[s] = fabsf(vsc);
         }
       } else {
+        // largest V scale of the chunk (non-negative fp16 values order as
+        // their bit patterns; the sign bit is cleared)
+        uint32_t vm = 0;
 #pragma unroll
         for (int j = 0; j < kScalePerLane; ++j) {
           sKs16[s][lane + 32 * j] = ksv[j];
           sVs16[s][lane + 32 * j] = vsv[j];
+          vm = max(vm, static_cast<uint32_t>(vsv[j] & 0x7FFFu));
         }
+        vm = __reduce_max_sync(0xffffffffu, vm);
+        if (lane == 0) sVmax[s] = __half2float(__ushort_as_half(static_cast<unsigned short>(vm)));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
@@ -245,49 +286,63 @@ __global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
   }
 
   // ---------------------------------------------------------------- consumers
-  const int tp = lane >> 1;          // token of this lane within a step
-  const int half = lane & 1;         // which half row this lane scores
-  // Query words for this lane's half row, in the order the key words are read.
-  int qreg[G][16];
-  int qsum_half[G];
+  const int gq = lane >> 2;          // mma group: token row (scores) / head row (P.V)
+  const int cq = lane & 3;           // mma thread in group
+  // Query fragments (B of the score MMA): for 32-channel block kb this lane
+  // supplies head gq, channels kb*32 + 8*cq + {0..3} (b0) and {4..7} (b1);
+  // INT4: the even channels of those 8 (b0) and the odd ones (b1). Any
+  // channel order works as long as the key fragments use the same one.
+  uint32_t qb0[4], qb1[4];
+  {
+    const uint8_t* qbytes = reinterpret_cast<const uint8_t*>(&sQw[gq < G ? gq : 0][0]);
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    qsum_half[hh] = sQsum[hh][half];
-    if constexpr (!kInt4) {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) qreg[hh][j] = static_cast<int>(sQw[hh][half * 16 + j]);
-    } else {
-      // 8 key words (64 nibbles) per half row; word j holds channels
-      // half*64 + 8j + {0..7}: even channels (low nibbles) and odd channels
-      // (high nibbles) are widened into separate byte vectors.
-      const uint8_t* qb = reinterpret_cast<const uint8_t*>(&sQw[hh][0]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int d0 = half * 64 + 8 * j;
-        qreg[hh][2 * j] = static_cast<int>(qb[d0] | (qb[d0 + 2] << 8) | (qb[d0 + 4] << 16) | (static_cast<uint32_t>(qb[d0 + 6]) << 24));
-        qreg[hh][2 * j + 1] = static_cast<int>(qb[d0 + 1] | (qb[d0 + 3] << 8) | (qb[d0 + 5] << 16) | (static_cast<uint32_t>(qb[d0 + 7]) << 24));
+    for (int kb = 0; kb < 4; ++kb) {
+      const int d0 = kb * 32 + 8 * cq;
+      uint32_t x0, x1;
+      if constexpr (!kInt4) {
+        x0 = *reinterpret_cast<const uint32_t*>(qbytes + d0);
+        x1 = *reinterpret_cast<const uint32_t*>(qbytes + d0 + 4);
+      } else {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(qbytes + d0);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(qbytes + d0 + 4);
+        x0 = __byte_perm(w0, w1, 0x6420);
+        x1 = __byte_perm(w0, w1, 0x7531);
       }
+      qb0[kb] = gq < G ? x0 : 0u;
+      qb1[kb] = gq < G ? x1 : 0u;
     }
   }
-  float qf[G];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) qf[hh] = sQf[hh];
-  const int my_group = kGroups == 2 ? (lane >> 4) : 0;   // group of this lane's 4 P.V channels
-  // Byte offset of this lane's 4 P.V channels inside a swizzled V row: the
-  // unswizzled offset is 4*lane (INT8) or 2*lane (INT4); the swizzle XORs
-  // the 16-byte chunk index with row % 8 (INT8) or (row / 2) % 4 (INT4).
-  // Steps start at multiples of 16 rows, so the XOR term is a compile-time
-  // function of the row within the step.
-  const int lane_off = kInt4 ? 2 * lane : 4 * lane;
-
-  float m_run[G], l_run[G];
-  float2 acc[G][2];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    m_run[hh] = -CUDART_INF_F;
-    l_run[hh] = 0.0f;
-    acc[hh][0] = acc[hh][1] = make_float2(0.0f, 0.0f);
+  // Heads of this lane's score columns: 2*cq and 2*cq + 1.
+  const int h0 = 2 * cq, h1 = 2 * cq + 1;
+  const bool h0ok = h0 < G, h1ok = h1 < G;
+  const float qf0 = h0ok ? sQf[h0] : 0.0f, qf1 = h1ok ? sQf[h1] : 0.0f;
+  int qs0[2] = {0, 0}, qs1[2] = {0, 0};          // INT4: 8 * query code sums per group
+  if constexpr (kInt4) {
+    const int s00 = h0ok ? sQsum[h0][0] : 0, s01 = h0ok ? sQsum[h0][1] : 0;
+    const int s10 = h1ok ? sQsum[h1][0] : 0, s11 = h1ok ? sQsum[h1][1] : 0;
+    if constexpr (kGroups == 2) {
+      qs0[0] = 8 * s00; qs0[1] = 8 * s01; qs1[0] = 8 * s10; qs1[1] = 8 * s11;
+    } else {
+      qs0[0] = 8 * (s00 + s01); qs1[0] = 8 * (s10 + s11);
+    }
   }
+  __half* myVh = sVh + warp * kStep * kVhStride;
+  float (*myP)[8][kStep] = sPw[warp];
+  const uint32_t vh_base = smem_u32(myVh);
+  // ldmatrix row address of this lane: matrix lane/8 = (token half, n-tile
+  // of the pair), row lane%8
+  const uint32_t ldsm_off =
+      static_cast<uint32_t>(((((lane >> 3) & 1) * 8 + (lane & 7)) * kVhStride + ((lane >> 4) * 8)) * 2);
+
+  float m_run0 = -CUDART_INF_F, m_run1 = -CUDART_INF_F;   // heads h0, h1
+  float l_run0 = 0.0f, l_run1 = 0.0f;                      // over this lane's tokens
+  float vref = 0.0f;                                       // running max V scale
+  float acc[16][2];                                        // head gq, stored columns 8nt + 2cq, +1
+  float sacc[kGroups][2];                                  // sum of P' per group (head gq)
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = 0.0f;
+#pragma unroll
+  for (int gg = 0; gg < kGroups; ++gg) sacc[gg][0] = sacc[gg][1] = 0.0f;
 
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % kStages;
@@ -296,144 +351,234 @@ __global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
     const uint8_t* cK = sK + s * kTile;
     const uint8_t* cV = sV + s * kTile;
     const int chunk_t0 = t_begin + c * C::kChunk;
+    // running V-scale reference: P' = p * vscale / vref stays in [0, 1]
+    const float vref_new = fmaxf(vref, sVmax[s]);
+    const float vratio = vref_new > 0.0f ? vref / vref_new : 1.0f;
+    const float inv_vref = vref_new > 0.0f ? 1.0f / vref_new : 0.0f;
+    vref = vref_new;
+    if (vratio != 1.0f) {                     // the same on every lane
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        acc[nt][0] *= vratio;
+        acc[nt][1] *= vratio;
+      }
+#pragma unroll
+      for (int gg = 0; gg < kGroups; ++gg) {
+        sacc[gg][0] *= vratio;
+        sacc[gg][1] *= vratio;
+      }
+    }
 #pragma unroll 1
     for (int sub = 0; sub < C::kPerWarp / kStep; ++sub) {
-      const int r0 = warp * C::kPerWarp + sub * kStep;      // first row (token) of this step in the chunk
-      const int tok = chunk_t0 + r0 + tp;                   // this lane's token
-      const bool valid = tok < t_end;
-      const int row = r0 + tp;
-      // ---------------- scores ----------------
-      float sc[G];
+      const int r0 = warp * C::kPerWarp + sub * kStep;      // first row of this step in the chunk
+      const int ra = r0 + gq, rb = r0 + gq + 8;             // this lane's score rows (tokens)
+      const bool va = chunk_t0 + ra < t_end, vb = chunk_t0 + rb < t_end;
+      // ---------------- scores: S^T = K Q^T ----------------
+      int sc[kNAcc][4];
+#pragma unroll
+      for (int a = 0; a < kNAcc; ++a) sc[a][0] = sc[a][1] = sc[a][2] = sc[a][3] = 0;
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) {
+        if constexpr (!kInt4) {
+          // 8 bytes of rows ra / rb at channel kb*32 + 8*cq: 16-byte chunk
+          // 2kb + cq/2, stored at chunk ^ (row % 8)
+          const int ch = 2 * kb + (cq >> 1);
+          const int off = ((ch ^ gq) << 4) + (cq & 1) * 8;
+          const uint2 xa = *reinterpret_cast<const uint2*>(cK + ra * 128 + off);
+          const uint2 xb = *reinterpret_cast<const uint2*>(cK + rb * 128 + off);
+          mma_s8(sc[0], xa.x, xb.x, xa.y, xb.y, qb0[kb], qb1[kb]);
+        } else {
+          // 4 bytes (8 nibbles) of rows ra / rb at channel kb*32 + 8*cq:
+          // 16-byte chunk kb, stored at kb ^ ((row / 2) % 4)
+          const int off = ((kb ^ ((gq >> 1) & 3)) << 4) + 4 * cq;
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cK + ra * 64 + off);
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cK + rb * 64 + off);
+          // nibble c -> byte c + 8 (even channels, odd channels)
+          const uint32_t ea = (wa & 0x0F0F0F0Fu) ^ 0x08080808u, oa = ((wa >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+          const uint32_t eb = (wb & 0x0F0F0F0Fu) ^ 0x08080808u, ob = ((wb >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+          mma_s8(sc[kNAcc == 2 ? (kb >> 1) : 0], ea, eb, oa, ob, qb0[kb], qb1[kb]);
+        }
+      }
+      // accumulator layout: [0] = (ra, h0), [1] = (ra, h1), [2] = (rb, h0), [3] = (rb, h1)
+      float s_a0, s_a1, s_b0, s_b1;
       if constexpr (!kInt4) {
-        int dot[G];
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) dot[hh] = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int ch = half * 4 + i;                       // 16-byte chunk of the 128-byte row
-          const uint4 kv = *reinterpret_cast<const uint4*>(cK + row * 128 + ((ch ^ (row & 7)) << 4));
-#pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            dot[hh] = __dp4a(static_cast<int>(kv.x), qreg[hh][4 * i + 0], dot[hh]);
-            dot[hh] = __dp4a(static_cast<int>(kv.y), qreg[hh][4 * i + 1], dot[hh]);
-            dot[hh] = __dp4a(static_cast<int>(kv.z), qreg[hh][4 * i + 2], dot[hh]);
-            dot[hh] = __dp4a(static_cast<int>(kv.w), qreg[hh][4 * i + 3], dot[hh]);
-          }
-        }
-        const float sk = sKsc[s];
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const int full_dot = dot[hh] + __shfl_xor_sync(0xffffffffu, dot[hh], 1);
-          sc[hh] = valid ? static_cast<float>(full_dot) * (qf[hh] * sk) : -CUDART_INF_F;
-        }
+        const float kq0 = qf0 * sKsc[s], kq1 = qf1 * sKsc[s];
+        s_a0 = static_cast<float>(sc[0][0]) * kq0;
+        s_a1 = static_cast<float>(sc[0][1]) * kq1;
+        s_b0 = static_cast<float>(sc[0][2]) * kq0;
+        s_b1 = static_cast<float>(sc[0][3]) * kq1;
       } else {
-        int dot[G];
+        float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) dot[hh] = 0;
+        for (int gg = 0; gg < kNAcc; ++gg) {
+          const float ka = __half2float(__ushort_as_half(sKs16[s][ra * kGroups + gg]));
+          const float kb2 = __half2float(__ushort_as_half(sKs16[s][rb * kGroups + gg]));
+          t0 += static_cast<float>(sc[gg][0] - qs0[gg]) * ka;
+          t1 += static_cast<float>(sc[gg][1] - qs1[gg]) * ka;
+          t2 += static_cast<float>(sc[gg][2] - qs0[gg]) * kb2;
+          t3 += static_cast<float>(sc[gg][3] - qs1[gg]) * kb2;
+        }
+        s_a0 = t0 * qf0; s_a1 = t1 * qf1; s_b0 = t2 * qf0; s_b1 = t3 * qf1;
+      }
+      if (!va) { s_a0 = -CUDART_INF_F; s_a1 = -CUDART_INF_F; }
+      if (!vb) { s_b0 = -CUDART_INF_F; s_b1 = -CUDART_INF_F; }
+      // ---------------- running softmax per head over the 16 tokens ----------------
+      float mx0 = fmaxf(s_a0, s_b0), mx1 = fmaxf(s_a1, s_b1);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int ch = half * 2 + i;                       // 16-byte chunk of the 64-byte row
-          const uint4 kv = *reinterpret_cast<const uint4*>(cK + row * 64 + ((ch ^ ((row >> 1) & 3)) << 4));
-          const uint32_t w4[4] = {kv.x, kv.y, kv.z, kv.w};
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (mx0 == -CUDART_INF_F) continue;     // no valid token in this step (the same on every lane)
+      const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
+      const float al0 = ex2(m_run0 - mn0), al1 = ex2(m_run1 - mn1);
+      m_run0 = mn0;
+      m_run1 = mn1;
+      const float pa0 = ex2(s_a0 - mn0), pa1 = ex2(s_a1 - mn1);
+      const float pb0 = ex2(s_b0 - mn0), pb1 = ex2(s_b1 - mn1);
+      l_run0 = l_run0 * al0 + (pa0 + pb0);
+      l_run1 = l_run1 * al1 + (pa1 + pb1);
+      // P' = p * vscale / vref -> per-warp buffer [group][head][token]
+      if constexpr (!kInt4) {
+        const float f = sVsc[s] * inv_vref;
+        if (h0ok) { myP[0][h0][gq] = pa0 * f; myP[0][h0][gq + 8] = pb0 * f; }
+        if (h1ok) { myP[0][h1][gq] = pa1 * f; myP[0][h1][gq + 8] = pb1 * f; }
+      } else {
 #pragma unroll
-          for (int wi = 0; wi < 4; ++wi) {
-            const int ev = static_cast<int>((w4[wi] & 0x0F0F0F0Fu) ^ 0x08080808u);        // code + 8, even channels
-            const int od = static_cast<int>(((w4[wi] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u); // code + 8, odd channels
-            const int j = i * 4 + wi;
+        for (int gg = 0; gg < kGroups; ++gg) {
+          const float fa = __half2float(__ushort_as_half(sVs16[s][ra * kGroups + gg])) * inv_vref;
+          const float fb = __half2float(__ushort_as_half(sVs16[s][rb * kGroups + gg])) * inv_vref;
+          if (h0ok) { myP[gg][h0][gq] = pa0 * fa; myP[gg][h0][gq + 8] = pb0 * fb; }
+          if (h1ok) { myP[gg][h1][gq] = pa1 * fa; myP[gg][h1][gq + 8] = pb1 * fb; }
+        }
+      }
+      if (gq == 0) {
+        sAlpha[warp][h0] = al0;
+        sAlpha[warp][h1] = al1;
+      }
+      // ---------------- V' rows of this step -> fp16 tile ----------------
+      {
+        const int t = lane >> 1, hf = lane & 1;               // token row, half of its channels
+        const int vr = r0 + t;
+        __half* dst = myVh + t * kVhStride + hf * 64;
+        if constexpr (!kInt4) {
+          // byte b -> fp16 with bits 0x64 | (b ^ 0x80) = 1152 + b (exact)
 #pragma unroll
-            for (int hh = 0; hh < G; ++hh) {
-              dot[hh] = __dp4a(ev, qreg[hh][2 * j], dot[hh]);
-              dot[hh] = __dp4a(od, qreg[hh][2 * j + 1], dot[hh]);
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = *reinterpret_cast<const uint4*>(cV + vr * 128 + (((hf * 4 + i) ^ (vr & 7)) << 4));
+            const uint32_t ws[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u, w.z ^ 0x80808080u, w.w ^ 0x80808080u};
+            uint32_t hv[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              hv[2 * k] = __byte_perm(ws[k], 0x64646464u, 0x5140);
+              hv[2 * k + 1] = __byte_perm(ws[k], 0x64646464u, 0x7362);
+            }
+            *reinterpret_cast<uint4*>(dst + i * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(dst + i * 16 + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+          }
+        } else {
+          // byte pair (b0, b1) = channels (8k, 8k+1), (8k+2, 8k+3) ->
+          //   even channels: 0x64 | 0x08 ^ low nibble      = 1032 + code
+          //   odd channels:  0x64 | (0x80 ^ high nibble<<4) = 1152 + 16 code
+          // stored per 4 channels in the order 0, 2, 1, 3
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint4 w = *reinterpret_cast<const uint4*>(cV + vr * 64 + (((hf * 2 + i) ^ ((vr >> 1) & 3)) << 4));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t lo = __byte_perm(ws[k], 0u, 0x4140);     // b0, 0, b1, 0
+              const uint32_t hi = __byte_perm(ws[k], 0u, 0x4342);     // b2, 0, b3, 0
+              const uint4 out = make_uint4((lo & 0x000F000Fu) ^ 0x64086408u, (lo & 0x00F000F0u) ^ 0x64806480u,
+                                           (hi & 0x000F000Fu) ^ 0x64086408u, (hi & 0x00F000F0u) ^ 0x64806480u);
+              *reinterpret_cast<uint4*>(dst + i * 32 + k * 8) = out;
             }
           }
         }
-        const float skg = __half2float(__ushort_as_half(sKs16[s][row * kGroups + (kGroups == 2 ? half : 0)]));
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const float part = static_cast<float>(dot[hh] - 8 * qsum_half[hh]) * skg;
-          const float tot = part + __shfl_xor_sync(0xffffffffu, part, 1);
-          sc[hh] = valid ? tot * qf[hh] : -CUDART_INF_F;
-        }
-      }
-      // ---------------- running softmax ----------------
-      float alpha[G];
-      bool any = false;
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float step_max = key_float(__reduce_max_sync(0xffffffffu, float_key(sc[hh])));
-        const float m_new = fmaxf(m_run[hh], step_max);
-        any = step_max != -CUDART_INF_F;
-        alpha[hh] = any ? ex2(m_run[hh] - m_new) : 1.0f;
-        const float pr = valid ? ex2(sc[hh] - m_new) : 0.0f;
-        l_run[hh] = l_run[hh] * alpha[hh] + (half == 0 ? pr : 0.0f);
-        if (any) m_run[hh] = m_new;
-        float pw = pr;
-        if constexpr (!kInt4) {
-          pw *= sVsc[s];
-        } else if constexpr (kGroups == 1) {
-          pw *= __half2float(__ushort_as_half(sVs16[s][row]));
-        }
-        if (half == 0) sP[warp][tp][hh] = make_float2(pw, pw);
-      }
-      if constexpr (kInt4 && kGroups == 2) {
-        sSV[warp][tp][half] = __half2float(__ushort_as_half(sVs16[s][row * 2 + half]));
       }
       __syncwarp();
-      if (!any) continue;            // no valid token in this step (warp-uniform)
-      // ---------------- P.V ----------------
+      // ---------------- rescale O and sum(P') by alpha, P' as fp16 high / low ----------------
+      {
+        const float fac = gq < G ? sAlpha[warp][gq] : 1.0f;
+        if (!__all_sync(0xffffffffu, fac == 1.0f)) {
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float2 a2 = make_float2(alpha[hh], alpha[hh]);
-        acc[hh][0] = fmul2(acc[hh][0], a2);
-        acc[hh][1] = fmul2(acc[hh][1], a2);
-      }
-      const uint8_t* vbase = cV + r0 * kRowBytes;
-#pragma unroll 4
-      for (int t = 0; t < kStep; ++t) {
-        float2 v01, v23;
-        if constexpr (!kInt4) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(vbase + t * 128 + (lane_off ^ ((t & 7) << 4)));
-          s8x4_to_f32(w, v01, v23);
-        } else {
-          const uint32_t w = *reinterpret_cast<const uint16_t*>(vbase + t * 64 + (lane_off ^ (((t >> 1) & 3) << 4)));
-          s4x4_to_f32(w, v01, v23);
-          if constexpr (kGroups == 2) {
-            const float sv = sSV[warp][t][my_group];
-            v01 = fmul2(v01, make_float2(sv, sv));
-            v23 = fmul2(v23, make_float2(sv, sv));
+          for (int nt = 0; nt < 16; ++nt) {
+            acc[nt][0] *= fac;
+            acc[nt][1] *= fac;
+          }
+#pragma unroll
+          for (int gg = 0; gg < kGroups; ++gg) {
+            sacc[gg][0] *= fac;
+            sacc[gg][1] *= fac;
           }
         }
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const float2 p2 = sP[warp][t][hh];
-          acc[hh][0] = ffma2(p2, v01, acc[hh][0]);
-          acc[hh][1] = ffma2(p2, v23, acc[hh][1]);
-        }
       }
-      __syncwarp();                  // sP / sSV reused by the next step
+      uint32_t pa_hi[kGroups], pa_lo[kGroups], pb_hi[kGroups], pb_lo[kGroups];
+#pragma unroll
+      for (int gg = 0; gg < kGroups; ++gg) {
+        float2 x01 = make_float2(0.0f, 0.0f), x89 = make_float2(0.0f, 0.0f);
+        if (gq < G) {
+          x01 = *reinterpret_cast<const float2*>(&myP[gg][gq][2 * cq]);
+          x89 = *reinterpret_cast<const float2*>(&myP[gg][gq][2 * cq + 8]);
+        }
+        split_f16x2(x01.x, x01.y, pa_hi[gg], pa_lo[gg]);
+        split_f16x2(x89.x, x89.y, pb_hi[gg], pb_lo[gg]);
+      }
+      // ---------------- O += P' V', sum(P') against a tile of ones ----------------
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {                        // pairs of 8-channel tiles
+        uint32_t b0a, b1a, b0b, b1b;
+        ldsm_x4_trans(vh_base + ldsm_off + np * 32, b0a, b1a, b0b, b1b);
+        const int gg = (kGroups == 2 && np >= 4) ? 1 : 0;
+        mma_f16(acc[2 * np][0], acc[2 * np][1], pa_hi[gg], pb_hi[gg], b0a, b1a);
+        mma_f16(acc[2 * np][0], acc[2 * np][1], pa_lo[gg], pb_lo[gg], b0a, b1a);
+        mma_f16(acc[2 * np + 1][0], acc[2 * np + 1][1], pa_hi[gg], pb_hi[gg], b0b, b1b);
+        mma_f16(acc[2 * np + 1][0], acc[2 * np + 1][1], pa_lo[gg], pb_lo[gg], b0b, b1b);
+      }
+#pragma unroll
+      for (int gg = 0; gg < kGroups; ++gg) {
+        mma_f16(sacc[gg][0], sacc[gg][1], pa_hi[gg], pb_hi[gg], kOnesF16x2, kOnesF16x2);
+        mma_f16(sacc[gg][0], sacc[gg][1], pa_lo[gg], pb_lo[gg], kOnesF16x2, kOnesF16x2);
+      }
+      __syncwarp();                  // buffers reused by the next step
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 
   // ---------------- merge the four consumer warps ----------------
+  // l: sum over the 8 token rows (lanes with the same cq)
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    float l = l_run[hh];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    l_run[hh] = l;
+  for (int o = 4; o < 32; o <<= 1) {
+    l_run0 += __shfl_xor_sync(0xffffffffu, l_run0, o);
+    l_run1 += __shfl_xor_sync(0xffffffffu, l_run1, o);
   }
   // every issued copy was consumed (or waited for on a timeout): the ring can
   // be reused for the reduction once all consumer warps are past their loops
   named_bar_sync(1, 32 * kConsumers);
+  if (gq == 0) {
+    if (h0ok) { sWm[warp][h0] = m_run0; sWl[warp][h0] = l_run0; }
+    if (h1ok) { sWm[warp][h1] = m_run1; sWl[warp][h1] = l_run1; }
+  }
+  if (gq < G) {
+    // O = (acc - offset * sum(P')) * vref; INT4 odd channels also / 16
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    *reinterpret_cast<float4*>(&sRed[(warp * G + hh) * kD + lane * 4]) =
-        make_float4(acc[hh][0].x, acc[hh][0].y, acc[hh][1].x, acc[hh][1].y);
-    if (lane == 0) {
-      sWm[warp][hh] = m_run[hh];
-      sWl[warp][hh] = l_run[hh];
+    for (int nt = 0; nt < 16; ++nt) {
+      const int gg = (kGroups == 2 && nt >= 8) ? 1 : 0;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = nt * 8 + 2 * cq + e;                 // stored column
+        float o;
+        int ch = col;
+        if constexpr (kInt4) {
+          const bool odd = (col & 2) != 0;                   // stored 0,2,1,3 -> channels 0,2 | 1,3
+          o = (acc[nt][e] - (odd ? kOffB : kOffA) * sacc[gg][0]) * (odd ? vref * 0.0625f : vref);
+          ch = (col & ~3) | ((col & 1) << 1) | ((col >> 1) & 1);
+        } else {
+          o = (acc[nt][e] - kOffA * sacc[gg][0]) * vref;
+        }
+        sRed[(warp * G + gq) * kD + ch] = o;
+      }
     }
   }
   named_bar_sync(1, 32 * kConsumers);
@@ -452,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, kInt4 ? 2 : 3)
         l = fmaf(sc, sWl[w][hh], l);
       }
     }
-    float* wsp = p.ws + ((static_cast<int64_t>(b) * p.Hq + hk * g + hh) * p.splits + split) * kWsStride;
+    float* wsp = p.ws + ((static_cast<int64_t>(b) * p.Hq + hk * g_all + hh) * p.splits + split) * kWsStride;
     wsp[d] = o;
     if (d == 0) {
       wsp[kD] = M;
@@ -527,14 +672,13 @@ bool decode_supported(int D, int group_ratio) { return D == kD && (group_ratio =
 // Split count: each split is a whole number of chunks (at least 4, to keep
 // the ring busy); among the counts that give at least two waves of resident
 // CTAs, take the smallest whose last wave is at least 90% full (else the
-// fullest). Resident CTAs per SM: 3 (INT8) / 2 (INT4), set by registers and
-// shared memory.
+// fullest). kCtasPerSm CTAs per SM are resident.
 static int splits_for(int B, int Hkv, int L, int num_sms, bool int4) {
   const int ck = chunk_tokens(int4);
   const int chunks = (L + ck - 1) / ck;
   if (chunks == 0) return 1;
   const int64_t pairs = static_cast<int64_t>(B) * Hkv;
-  const int64_t slots = static_cast<int64_t>(num_sms) * (int4 ? 2 : 3);
+  const int64_t slots = static_cast<int64_t>(num_sms) * kCtasPerSm;
   const int max_splits = max(1, min(64, chunks / 4));
   int best = 1;
   double best_fill = -1.0;

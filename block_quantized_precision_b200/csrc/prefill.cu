@@ -8,25 +8,29 @@
 // tiles, inner loop over key/value tiles with a running softmax; the page's
 // normalisation is replaced by the standard running-max form).
 //
-// One CTA = one tile of 128 query rows of one (b, h); two CTAs share an SM
-// (each allocates 256 TMEM columns and ~97 KB of shared memory).
-//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into a
-//               two-stage ring (128B / 64B swizzle, no multicast).
-//   warp 1      TMEM allocation; lane 0 issues the MMAs:
-//                 S  = Q K^T        M=128, N=128, K=D      -> TMEM cols [0,128)
-//                 PV = P V          M=128, N=D,   K=128    -> TMEM cols [0,D)
-//               kind::i8 (s32 accumulate) or kind::f8f6f4 (e4m3, f32).
-//               P is read from shared memory (K-major), V is used MN-major
-//               straight from its token-major tile.
-//   warps 2-5   one thread per query row: reads S from TMEM, applies the
-//               block scales and the mask, running max / sum in the log2
-//               domain, rounds P to 8 bits (e4m3, or round(127 p) for INT8)
-//               and writes it to shared memory in the swizzled K-major
-//               layout; then folds PV into the float32 output kept in TMEM
-//               cols [128, 128+D): O = O * alpha + PV * c_j; finally writes
-//               O / l as bfloat16 (and the LSE).
-// Per key tile: QK^T -> softmax -> PV -> fold, handed over with mbarriers
-// (all waits bounded).
+// One CTA = two consecutive tiles of 128 query rows (A, B) of one (b, h);
+// one CTA per SM (all 512 TMEM columns, ~161 KB of shared memory at D = 128),
+// 12 warps.
+//   warp 0      TMA producer: both Q tiles once, then K/V tiles of 128 keys
+//               into a three-stage ring (128B / 64B swizzle, no multicast).
+//   warps 1, 2  MMA issuers of tile A and tile B (warp 1 also allocates
+//               TMEM); one lane each, so neither tile waits for the other:
+//                 S_x  = Q_x K_j^T   M=128, N=128, K=D   -> TMEM [256x, 256x+128)
+//                 PV_x = P_x V_j     M=128, N=D,   K=128 -> TMEM [256x+128, +D)
+//               kind::i8 (s32 accumulate) or kind::f8f6f4 (e4m3, f32). P is
+//               read from shared memory (K-major); V is used MN-major straight
+//               from its token-major tile.
+//   warp 3      idle (it completes warpgroup 0 for the register split).
+//   warps 4-7   tile A, warps 8-11 tile B: one query row per thread. Per key
+//               tile j: (1) row max of S_j, (2) probabilities in the log2
+//               domain, rounded to 8 bits (e4m3, or RNE(127 p) for INT8),
+//               written to shared memory in the swizzled K-major layout --
+//               from here the tensor core may compute S_{j+1}; (3) PV_{j-1}
+//               folded into the float32 output held in registers -- from
+//               here it may compute PV_j. Finally O / l as bfloat16 (and the
+//               LSE).
+// With two tiles per CTA the tensor core works on one tile's products while
+// the other tile's rows are in their softmax. Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -41,13 +45,22 @@ namespace qattn {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kTileM = 128;   // query rows per CTA
-constexpr int kTileN = 128;   // keys per tile
-constexpr int kStagesKV = 2;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 128;
-constexpr int kMaxBlk = 512;  // K/V block scales staged in shared memory (keys up to 131072)
+constexpr int kThreads = 384;   // 12 warps = 3 warpgroups
+// Register split (setmaxnreg): the launch gives every thread the kernel's register count (168);
+// warpgroup 0 (TMA, two MMA issuers, one idle warp) drops to kRegsLow so that the two
+// row warpgroups can rise to kRegsHigh (each row thread keeps its 128-float
+// output row in registers). 128 * kRegsLow + 256 * kRegsHigh must not exceed
+// 384 * (registers per thread at launch); the host checks this before every
+// launch.
+constexpr int kRegsLow = 40;
+constexpr int kRegsHigh = 232;
+constexpr int kRegsNeeded = (128 * kRegsLow + 256 * kRegsHigh + kThreads - 1) / kThreads;
+constexpr int kTileM = 128;     // query rows per tile
+constexpr int kTileN = 128;     // keys per tile
+constexpr int kStagesKV = 3;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxBlk = 512;    // K/V block scales staged in shared memory (keys up to 131072)
+constexpr float kLog2_127 = 6.988684686772166f;
 
 struct PrefillParams {
   const float* qs;
@@ -56,7 +69,7 @@ struct PrefillParams {
   __nv_bfloat16* out;
   float* lse;
   int B, H, Nq, Nkv;
-  int nqt, nqb, nkb;
+  int nqt, npairs, nqb, nkb;
   int causal;
   int layout;
   float scale_log2;
@@ -66,9 +79,9 @@ struct PrefillParams {
 template <int D>
 struct Smem {
   static constexpr int kTileBytes = kTileM * D;       // one 128-row code tile
-  static constexpr int kQ = 0;
-  static constexpr int kP = kQ + kTileBytes;
-  static constexpr int kK = kP + kTileM * kTileN;     // P tile: 128 rows x 128 keys
+  static constexpr int kQ = 0;                        // two Q tiles
+  static constexpr int kP = kQ + 2 * kTileBytes;      // two P tiles: 128 rows x 128 keys
+  static constexpr int kK = kP + 2 * kTileM * kTileN;
   static constexpr int kV = kK + kStagesKV * kTileBytes;
   static constexpr int kEnd = kV + kStagesKV * kTileBytes;
   static constexpr int kBytes = kEnd + 1024;          // slack for 1024-byte alignment
@@ -95,14 +108,268 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Exact INT32 -> float32 of two accumulator words (|S| < 2^22): the bits of
+// 1.5 * 2^23 + S are formed by an integer add, then 1.5 * 2^23 is removed.
+__device__ __forceinline__ float2 s32x2_to_f32x2(uint32_t a, uint32_t b) {
+  return fadd2(make_float2(__int_as_float(static_cast<int>(a) + 0x4B400000),
+                           __int_as_float(static_cast<int>(b) + 0x4B400000)),
+               make_float2(-12582912.0f, -12582912.0f));
+}
+
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Element offset of token n of head (b, h), channel 0.
 __device__ __forceinline__ int64_t row_offset(int layout, int H, int N, int D, int b, int h, int n) {
   return layout == 0 ? ((static_cast<int64_t>(b) * H + h) * N + n) * D
                      : ((static_cast<int64_t>(b) * N + n) * H + h) * D;
 }
 
+struct TileBars {
+  uint64_t s_full;    // S_j in TMEM               (MMA commit)
+  uint64_t p_full;    // P_j in shared memory      (128 row threads)
+  uint64_t pv_full;   // PV_j in TMEM              (MMA commit)
+  uint64_t pv_free;   // PV_j read by the rows     (128 row threads)
+};
+
+// O = alpha * O + g * PV for this thread's row: PV read from TMEM 32 columns
+// at a time. `scale_o` is false when alpha == 1 for every lane of the warp.
 template <int D, bool kInt8>
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ __forceinline__ void fold_pv(float (&O)[D], uint32_t tPV, float alpha, float g, bool scale_o) {
+  const float2 a2 = make_float2(alpha, alpha);
+  const float2 g2 = make_float2(g, g);
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t pv[32];
+    tmem_ld32(tPV + c * 32, pv);
+    tmem_wait_ld();
+    reg_fence(pv);
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const float2 x = kInt8 ? s32x2_to_f32x2(pv[e], pv[e + 1])
+                             : make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
+      float2 o = make_float2(O[c * 32 + e], O[c * 32 + e + 1]);
+      if (scale_o) o = fmul2(o, a2);
+      o = ffma2(x, g2, o);
+      O[c * 32 + e] = o.x;
+      O[c * 32 + e + 1] = o.y;
+    }
+  }
+}
+
+// The rows of one query tile (4 warps, one row per thread).
+template <int D, bool kInt8>
+__device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars, uint32_t tS, uint32_t tPV,
+                                          uint8_t* sP, const float* sKsc, const float* sVsc, int qt, int ntiles,
+                                          int bh, int b, int h, int quarter, int lane, volatile int* abort_flag) {
+  const int r = quarter * 32 + lane;            // row within the tile (= TMEM lane)
+  const int q0 = qt * kTileM;
+  const int qrow = q0 + r;
+  tS += static_cast<uint32_t>(quarter * 32) << 16;
+  tPV += static_cast<uint32_t>(quarter * 32) << 16;
+  const float sq = p.qs[static_cast<int64_t>(bh) * p.nqb + qt];
+  uint8_t* prow = sP + r * 128;
+  const int rsw = r & 7;
+
+  float O[D];
+#pragma unroll
+  for (int d = 0; d < D; ++d) O[d] = 0.0f;
+  float m_run = -CUDART_INF_F, l_run = 0.0f;
+  float g_prev = 0.0f;                          // V dequantization factor of the previous tile
+  bool ok = true;
+  for (int j = 0; j < ntiles; ++j) {
+    ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full, j & 1, abort_flag, p.err));
+    if (!ok) break;
+    tc_fence_after();
+    const int blk = j >> 1;
+    const float kscale = blk < kMaxBlk ? sKsc[blk] : p.ks[static_cast<int64_t>(bh) * p.nkb + blk];
+    const float vscale = blk < kMaxBlk ? sVsc[blk] : p.vs[static_cast<int64_t>(bh) * p.nkb + blk];
+    const float ksc = sq * kscale * p.scale_log2;
+    const int key0 = j * kTileN;
+    // Only the last tile (ragged N_kv) and the causal diagonal tiles have
+    // masked keys; the mask is applied on those tiles only (warp-uniform).
+    const bool partial = (key0 + kTileN > p.Nkv) || (p.causal && key0 + kTileN - 1 > q0);
+    int kmax = p.Nkv - key0;                    // keys valid for this row: [0, kmax)
+    if (p.causal) kmax = min(kmax, qrow - key0 + 1);
+
+    // ---- (1) row max: integer max of the INT32 scores, or float max ----
+    float tmax;
+    if constexpr (kInt8) {
+      int i0 = INT_MIN, i1 = INT_MIN, i2 = INT_MIN, i3 = INT_MIN;
+#pragma unroll 1
+      for (int c = 0; c < kTileN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        if (partial) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e >= kmax) v[e] = 0x80000000u;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          i0 = max(i0, static_cast<int>(v[e]));
+          i1 = max(i1, static_cast<int>(v[e + 1]));
+          i2 = max(i2, static_cast<int>(v[e + 2]));
+          i3 = max(i3, static_cast<int>(v[e + 3]));
+        }
+      }
+      const int im = max(max(i0, i1), max(i2, i3));
+      tmax = im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
+    } else {
+      float f0 = -CUDART_INF_F, f1 = -CUDART_INF_F, f2 = -CUDART_INF_F, f3 = -CUDART_INF_F;
+#pragma unroll 1
+      for (int c = 0; c < kTileN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        if (partial) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e >= kmax) v[e] = 0xFF800000u;        // -inf
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          f0 = fmax3(f0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+          f1 = fmax3(f1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          f2 = fmax3(f2, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+          f3 = fmax3(f3, __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+        }
+      }
+      const float fm = fmaxf(fmaxf(f0, f1), fmaxf(f2, f3));
+      tmax = fm == -CUDART_INF_F ? -CUDART_INF_F : fm * ksc;
+    }
+    const float m_new = fmaxf(m_run, tmax);
+    const float m_use = m_new == -CUDART_INF_F ? 0.0f : m_new;
+    const float alpha = ex2(m_run - m_use);     // 0 on the first tile
+
+    // P_{j-1} must have been consumed (PV_{j-1} complete) before P_j is written.
+    if (j > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_full, (j - 1) & 1, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+    }
+
+    // ---- (2) probabilities, 8-bit rounding, P to shared memory ----
+    // INT8: code = RNE(127 p) taken as RNE(2^(t + log2 127)); FP8: e4m3(p).
+    const float2 k2 = make_float2(ksc, ksc);
+    const float toff = (kInt8 ? kLog2_127 : 0.0f) - m_use;
+    const float2 t2 = make_float2(toff, toff);
+    float rowsum;
+    {
+      int ri0 = 0, ri1 = 0;
+      float rf0 = 0.0f, rf1 = 0.0f, rf2 = 0.0f, rf3 = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < kTileN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_wait_ld();
+        reg_fence(v);
+        uint32_t packed[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          float2 t01, t23;
+          if constexpr (kInt8) {
+            t01 = ffma2(s32x2_to_f32x2(v[4 * w], v[4 * w + 1]), k2, t2);
+            t23 = ffma2(s32x2_to_f32x2(v[4 * w + 2], v[4 * w + 3]), k2, t2);
+          } else {
+            t01 = ffma2(make_float2(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1])), k2, t2);
+            t23 = ffma2(make_float2(__uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3])), k2, t2);
+          }
+          float pr[4] = {ex2(t01.x), ex2(t01.y), ex2(t23.x), ex2(t23.y)};
+          if (partial) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[e] = c * 32 + w * 4 + e < kmax ? pr[e] : 0.0f;
+          }
+          if constexpr (kInt8) {
+            // adding 1.5 * 2^23 rounds to an integer (half to even) and leaves
+            // it in the low mantissa byte
+            const float2 q01 = fadd2(make_float2(pr[0], pr[1]), make_float2(12582912.0f, 12582912.0f));
+            const float2 q23 = fadd2(make_float2(pr[2], pr[3]), make_float2(12582912.0f, 12582912.0f));
+            const uint32_t b01 = __byte_perm(__float_as_uint(q01.x), __float_as_uint(q01.y), 0x0040);
+            const uint32_t b23 = __byte_perm(__float_as_uint(q23.x), __float_as_uint(q23.y), 0x0040);
+            const uint32_t word = __byte_perm(b01, b23, 0x5410);
+            if (w & 1) ri1 = __dp4a(static_cast<int>(word), 0x01010101, ri1);
+            else ri0 = __dp4a(static_cast<int>(word), 0x01010101, ri0);
+            packed[w] = word;
+          } else {
+            const uint32_t lo = cvt_e4m3x2(pr[0], pr[1]);
+            const uint32_t hi = cvt_e4m3x2(pr[2], pr[3]);
+            packed[w] = lo | (hi << 16);
+            // row sum of the rounded probabilities (exact values via fp16)
+            if (w & 1) {
+              rf2 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rf2);
+              rf3 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rf3);
+            } else {
+              rf0 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rf0);
+              rf1 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rf1);
+            }
+          }
+        }
+        // keys c*32 .. c*32+31 = 16-byte chunks 2c and 2c+1 of this row
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          const int chunk = 2 * c + hc;
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ rsw) << 4)) =
+              make_uint4(packed[4 * hc], packed[4 * hc + 1], packed[4 * hc + 2], packed[4 * hc + 3]);
+        }
+      }
+      rowsum = kInt8 ? static_cast<float>(ri0 + ri1) * (1.0f / 127.0f) : (rf0 + rf1) + (rf2 + rf3);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive(&bars.p_full);
+    l_run = l_run * alpha + rowsum;
+    m_run = m_new;
+
+    // ---- (3) fold PV_{j-1}: O <- alpha_j (O + g_{j-1} PV_{j-1}) ----
+    // (O is kept relative to the newest running max.)
+    if (j > 0) {
+      const bool scale_o = !__all_sync(0xffffffffu, alpha == 1.0f);
+      fold_pv<D, kInt8>(O, tPV, alpha, alpha * g_prev, scale_o);
+      tc_fence_before();
+      mbar_arrive(&bars.pv_free);
+    }
+    g_prev = vscale * (kInt8 ? (1.0f / 127.0f) : 1.0f);
+  }
+  if (!ok || ntiles == 0) return;
+  // last product: O += g_{n-1} PV_{n-1}
+  ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_full, (ntiles - 1) & 1, abort_flag, p.err));
+  if (!ok) return;
+  tc_fence_after();
+  fold_pv<D, kInt8>(O, tPV, 1.0f, g_prev, false);
+
+  // epilogue: out = O / l (bf16), lse
+  if (qrow < p.Nq) {
+    const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+    __nv_bfloat16* orow = p.out + row_offset(p.layout, p.H, p.Nq, D, b, h, qrow);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 t = __floats2bfloat162_rn(O[c * 8 + 2 * e] * inv_l, O[c * 8 + 2 * e + 1] * inv_l);
+        w4[e] = *reinterpret_cast<const uint32_t*>(&t);
+      }
+      *reinterpret_cast<uint4*>(orow + c * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    if (p.lse) p.lse[static_cast<int64_t>(bh) * p.Nq + qrow] = m_run * 0.6931471805599453f + logf(l_run);
+  }
+}
+
+// Grid: one CTA per pair of consecutive query tiles (2i, 2i+1) of one (b, h),
+// the pairs with the most key tiles first (causal).
+template <int D, bool kInt8>
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using L = Smem<D>;
@@ -116,15 +383,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + L::kQ;
-  uint8_t* sP = smem + L::kP;
-  uint8_t* sK = smem + L::kK;
-  uint8_t* sV = smem + L::kV;
+  uint8_t* sQ = smem + L::kQ;                          // [2][128 x D]
+  uint8_t* sP = smem + L::kP;                          // [2][128 x 128]
+  uint8_t* sK = smem + L::kK;                          // [stages][128 x D]
+  uint8_t* sV = smem + L::kV;                          // [stages][128 x D]
 
   __shared__ __align__(8) uint64_t bar_q_full;
   __shared__ __align__(8) uint64_t bar_kv_full[kStagesKV];
   __shared__ __align__(8) uint64_t bar_kv_empty[kStagesKV];
-  __shared__ __align__(8) uint64_t bar_s_full, bar_p_full, bar_pv_full, bar_free, bar_drain;
+  __shared__ __align__(8) TileBars bars[2];
+  __shared__ __align__(8) uint64_t bar_drain[2];
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ float sKsc[kMaxBlk], sVsc[kMaxBlk];
@@ -132,24 +400,31 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  const int qt = p.nqt - 1 - static_cast<int>(blockIdx.x) / BH;   // longest (causal) tiles first
+  const int pair = p.npairs - 1 - static_cast<int>(blockIdx.x) / BH;
   const int bh = static_cast<int>(blockIdx.x) % BH;
   const int b = bh / p.H, h = bh % p.H;
-  const int q0 = qt * kTileM;
+  const int qt2[2] = {2 * pair, 2 * pair + 1 < p.nqt ? 2 * pair + 1 : -1};
   const int nkt_all = (p.Nkv + kTileN - 1) / kTileN;
-  const int ntiles = p.causal ? min(nkt_all, (q0 + kTileM - 1) / kTileN + 1) : nkt_all;
+  int nt2[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+    nt2[x] = qt2[x] < 0 ? 0 : (p.causal ? min(nkt_all, (qt2[x] * kTileM + kTileM - 1) / kTileN + 1) : nkt_all);
+  const int nt_max = max(nt2[0], nt2[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(&bar_q_full, 1);
     for (int s = 0; s < kStagesKV; ++s) {
       mbar_init(&bar_kv_full[s], 1);
-      mbar_init(&bar_kv_empty[s], 1);
+      mbar_init(&bar_kv_empty[s], 2);
     }
-    mbar_init(&bar_s_full, 1);
-    mbar_init(&bar_p_full, 128);
-    mbar_init(&bar_pv_full, 1);
-    mbar_init(&bar_free, 128);
-    mbar_init(&bar_drain, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars[x].s_full, 1);
+      mbar_init(&bars[x].p_full, 128);
+      mbar_init(&bars[x].pv_full, 1);
+      mbar_init(&bars[x].pv_free, 128);
+    }
+    mbar_init(&bar_drain[0], 1);
+    mbar_init(&bar_drain[1], 1);
     abort_flag = 0;
     mbar_fence_init();
   }
@@ -162,19 +437,19 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem = tmem_base_slot;
 
-  // Waits below are made warp-uniform (__all_sync): a whole warp leaves its
-  // loop together, so every .sync.aligned instruction stays convergent.
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    regs_dec<kRegsLow>();
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar_q_full, L::kTileBytes);
-      tma_load_4d(sQ, &tmQ, &bar_q_full, 0, q0, h, b);
+      mbar_arrive_expect_tx(&bar_q_full, (qt2[1] >= 0 ? 2 : 1) * L::kTileBytes);
+      for (int x = 0; x < 2; ++x)
+        if (qt2[x] >= 0) tma_load_4d(sQ + x * L::kTileBytes, &tmQ, &bar_q_full, 0, qt2[x] * kTileM, h, b);
     }
     int j = 0;
-    for (; j < ntiles; ++j) {
+    for (; j < nt_max; ++j) {
       const int st = j % kStagesKV;
       if (j >= kStagesKV) {
         const bool ok = mbar_wait(&bar_kv_empty[st], ((j / kStagesKV) - 1) & 1, &abort_flag, p.err);
@@ -194,30 +469,60 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_wait(&bar_kv_full[i % kStagesKV], (i / kStagesKV) & 1, nullptr, nullptr, 100000000ull);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t aQ = smem_u32(sQ), aP = smem_u32(sP);
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues tile A's products, warp 2 tile B's (one elected lane
+    // each), so neither tile waits for the other. Per key tile j:
+    //   S(j+1)  once P(j) has been written (S free) and K/V(j+1) has landed,
+    //   PV(j)   once PV(j-1) has been read,
+    // then a commit releases K/V stage j (two arrivals: one per tile; a tile
+    // with fewer key tiles arrives at once for the stages it does not read).
+    regs_dec<kRegsLow>();
+    const int x = warp - 1;
+    const int nt = nt2[x];
+    const uint32_t aQ = smem_u32(sQ) + x * L::kTileBytes, aP = smem_u32(sP) + x * kTileM * kTileN;
     const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_q_full, 0, &abort_flag, p.err));
-    for (int j = 0; ok && j < ntiles; ++j) {
-      const int st = j % kStagesKV;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err));
-      if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar_free, (j - 1) & 1, &abort_flag, p.err));
-      if (!ok) break;
-      tc_fence_after();
+    const uint32_t tS = tmem + x * 256, tPV = tmem + x * 256 + 128;
+    TileBars& tb = bars[x];
+    auto issue_s = [&](int j) {
       if (lane == 0) {
-        const uint32_t kbase = aK + st * L::kTileBytes;
+        const uint32_t kbase = aK + (j % kStagesKV) * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const uint64_t da = smem_desc(aQ + kk * 32, 16, kSBO, kSwz);
           const uint64_t db = smem_desc(kbase + kk * 32, 16, kSBO, kSwz);
-          mma_ss<kInt8>(tmem, da, db, kIdescQK, kk > 0 ? 1u : 0u);
+          mma_ss<kInt8>(tS, da, db, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bar_s_full);
+        mma_commit(&tb.s_full);
       }
       __syncwarp();
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_p_full, j & 1, &abort_flag, p.err));
+    };
+    bool ok = nt == 0 || __all_sync(0xffffffffu, mbar_wait(&bar_q_full, 0, &abort_flag, p.err));
+    for (int j = 0; ok && j < nt_max; ++j) {
+      const int st = j % kStagesKV;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err));
       if (!ok) break;
+      if (j >= nt) {
+        if (lane == 0) mbar_arrive(&bar_kv_empty[st]);
+        __syncwarp();
+        continue;
+      }
+      tc_fence_after();
+      if (j == 0) issue_s(0);
+      // S(j) consumed: P(j) is in shared memory
+      ok = __all_sync(0xffffffffu, mbar_wait(&tb.p_full, j & 1, &abort_flag, p.err));
+      if (!ok) break;
+      if (j + 1 < nt) {
+        const int j1 = j + 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[j1 % kStagesKV], (j1 / kStagesKV) & 1, &abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(j1);
+      }
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&tb.pv_free, (j - 1) & 1, &abort_flag, p.err));
+        if (!ok) break;
+      }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t vbase = aV + st * L::kTileBytes;
@@ -226,226 +531,37 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint64_t da = smem_desc(aP + kk * 32, 16, 1024, 2u);
           // MN-major V: 32 keys per MMA = 4 groups of 8 key rows, SBO apart.
           const uint64_t db = smem_desc(vbase + kk * 32 * kRowB, kTileN * kRowB, kSBO, kSwz);
-          mma_ss<kInt8>(tmem, da, db, kIdescPV, kk > 0 ? 1u : 0u);
+          mma_ss<kInt8>(tPV, da, db, kIdescPV, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bar_pv_full);
+        mma_commit(&tb.pv_full);
         mma_commit(&bar_kv_empty[st]);
       }
       __syncwarp();
     }
     if (abort_flag && lane == 0) {
-      // Wait (bounded) until every MMA issued so far has completed.
-      mma_commit(&bar_drain);
-      mbar_wait(&bar_drain, 0, nullptr, nullptr, 100000000ull);
+      // Wait (bounded) until every MMA this thread issued has completed.
+      mma_commit(&bar_drain[x]);
+      mbar_wait(&bar_drain[x], 0, nullptr, nullptr, 100000000ull);
     }
     __syncwarp();
+  } else if (warp == 3) {
+    regs_dec<kRegsLow>();
   } else {
     // ------------------------------------------------------------ softmax rows
-    const int quarter = warp & 3;                 // TMEM lane quarter of this warp
-    const int r = quarter * 32 + lane;            // query row within the tile
-    const int qrow = q0 + r;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const float sq = p.qs[static_cast<int64_t>(bh) * p.nqb + qt];
-    // K/V block scales of this head, staged once (beyond kMaxBlk blocks they
-    // are read from global memory).
-    for (int i = threadIdx.x - 64; i < min(p.nkb, kMaxBlk); i += 128) {
-      sKsc[i] = p.ks[static_cast<int64_t>(bh) * p.nkb + i];
-      sVsc[i] = p.vs[static_cast<int64_t>(bh) * p.nkb + i];
+    regs_inc<kRegsHigh>();
+    const int x = (warp - 4) >> 2;                // which query tile
+    // K/V block scales of this head, staged once by tile A's warps (beyond
+    // kMaxBlk blocks they are read from global memory).
+    if (x == 0) {
+      for (int i = threadIdx.x - 128; i < min(p.nkb, kMaxBlk); i += 128) {
+        sKsc[i] = p.ks[static_cast<int64_t>(bh) * p.nkb + i];
+        sVsc[i] = p.vs[static_cast<int64_t>(bh) * p.nkb + i];
+      }
     }
-    named_bar_sync(1, 128);
-    float m_run = -CUDART_INF_F, l_run = 0.0f;
-    uint8_t* prow = sP + r * 128;
-    const int rsw = r & 7;
-    bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_s_full, j & 1, &abort_flag, p.err));
-      if (!ok) break;
-      tc_fence_after();
-      const int blk = j >> 1;
-      const float kscale = blk < kMaxBlk ? sKsc[blk] : p.ks[static_cast<int64_t>(bh) * p.nkb + blk];
-      const float vscale = blk < kMaxBlk ? sVsc[blk] : p.vs[static_cast<int64_t>(bh) * p.nkb + blk];
-      const float ksc = sq * kscale * p.scale_log2;
-      const int key0 = j * kTileN;
-      // Only the last tile (ragged N_kv) and the causal diagonal tile have
-      // masked keys; the mask is applied on those tiles only (warp-uniform).
-      const bool partial = (key0 + kTileN > p.Nkv) || (p.causal && key0 + kTileN - 1 > q0);
-      int kmax = p.Nkv - key0;                    // keys valid for this row: [0, kmax)
-      if (p.causal) kmax = min(kmax, qrow - key0 + 1);
-
-      // ---- pass 1: row max (integer max of the INT32 scores, or float max) ----
-      float tmax;
-      if constexpr (kInt8) {
-        int im = INT_MIN;
-#pragma unroll 1
-        for (int c = 0; c < kTileN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(trow + c * 32, v);
-          tmem_wait_ld();
-          if (partial) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) im = max(im, c * 32 + e < kmax ? static_cast<int>(v[e]) : INT_MIN);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) im = max(im, static_cast<int>(v[e]));
-          }
-        }
-        tmax = im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
-      } else {
-        float fm = -CUDART_INF_F;
-#pragma unroll 1
-        for (int c = 0; c < kTileN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(trow + c * 32, v);
-          tmem_wait_ld();
-          if (partial) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2)
-              fm = fmax3(fm, c * 32 + e < kmax ? __uint_as_float(v[e]) : -CUDART_INF_F,
-                         c * 32 + e + 1 < kmax ? __uint_as_float(v[e + 1]) : -CUDART_INF_F);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) fm = fmax3(fm, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-          }
-        }
-        tmax = fm * ksc;
-      }
-      const float m_new = fmaxf(m_run, tmax);
-      const float alpha = ex2(m_run - m_new);     // 0 on the first tile
-      const float2 k2 = make_float2(ksc, ksc);
-      const float2 nm2 = make_float2(-m_new, -m_new);
-
-      // ---- pass 2: probabilities, 8-bit rounding, P to shared memory ----
-      float rs0 = 0.0f, rs1 = 0.0f;
-      int rsum_i = 0;
-#pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + c * 32, v);
-        tmem_wait_ld();
-        uint32_t packed[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          float2 t01, t23;
-          if constexpr (kInt8) {
-            // exact INT32 -> float32: 1.5 * 2^23 + S has S in its low mantissa bits
-            const float2 f01 = fadd2(make_float2(__int_as_float(static_cast<int>(v[4 * w]) + 0x4B400000),
-                                                 __int_as_float(static_cast<int>(v[4 * w + 1]) + 0x4B400000)),
-                                     make_float2(-12582912.0f, -12582912.0f));
-            const float2 f23 = fadd2(make_float2(__int_as_float(static_cast<int>(v[4 * w + 2]) + 0x4B400000),
-                                                 __int_as_float(static_cast<int>(v[4 * w + 3]) + 0x4B400000)),
-                                     make_float2(-12582912.0f, -12582912.0f));
-            t01 = ffma2(f01, k2, nm2);
-            t23 = ffma2(f23, k2, nm2);
-          } else {
-            t01 = ffma2(make_float2(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1])), k2, nm2);
-            t23 = ffma2(make_float2(__uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3])), k2, nm2);
-          }
-          float pr[4] = {ex2(t01.x), ex2(t01.y), ex2(t23.x), ex2(t23.y)};
-          if (partial) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) pr[e] = c * 32 + w * 4 + e < kmax ? pr[e] : 0.0f;
-          }
-          if constexpr (kInt8) {
-            // code = RNE(p * 127): product rounded to float32, then the
-            // 1.5 * 2^23 addend rounds it to an integer (half to even)
-            const float2 q01 = fadd2(fmul2(make_float2(pr[0], pr[1]), make_float2(127.0f, 127.0f)),
-                                     make_float2(12582912.0f, 12582912.0f));
-            const float2 q23 = fadd2(fmul2(make_float2(pr[2], pr[3]), make_float2(127.0f, 127.0f)),
-                                     make_float2(12582912.0f, 12582912.0f));
-            const uint32_t b01 = __byte_perm(__float_as_uint(q01.x), __float_as_uint(q01.y), 0x0040);
-            const uint32_t b23 = __byte_perm(__float_as_uint(q23.x), __float_as_uint(q23.y), 0x0040);
-            const uint32_t word = __byte_perm(b01, b23, 0x5410);
-            rsum_i = __dp4a(static_cast<int>(word), 0x01010101, rsum_i);
-            packed[w] = word;
-          } else {
-            const uint32_t lo = cvt_e4m3x2(pr[0], pr[1]);
-            const uint32_t hi = cvt_e4m3x2(pr[2], pr[3]);
-            packed[w] = lo | (hi << 16);
-            // row sum of the rounded probabilities (exact values via fp16)
-            rs0 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rs0);
-            rs1 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rs1);
-          }
-        }
-        // keys c*32 .. c*32+31 = 16-byte chunks 2c and 2c+1 of this row
-#pragma unroll
-        for (int hchunk = 0; hchunk < 2; ++hchunk) {
-          const int chunk = 2 * c + hchunk;
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ rsw) << 4)) =
-              make_uint4(packed[4 * hchunk], packed[4 * hchunk + 1], packed[4 * hchunk + 2], packed[4 * hchunk + 3]);
-        }
-      }
-      const float rowsum = kInt8 ? static_cast<float>(rsum_i) * (1.0f / 127.0f) : rs0 + rs1;
-      tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(&bar_p_full);
-      l_run = l_run * alpha + rowsum;
-      m_run = m_new;
-
-      // ---- fold PV into O: O = O * alpha + PV * c_j ----
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar_pv_full, j & 1, &abort_flag, p.err));
-      if (!ok) break;
-      tc_fence_after();
-      const float cj = vscale * (kInt8 ? (1.0f / 127.0f) : 1.0f);
-      const float2 c2 = make_float2(cj, cj);
-      const float2 a2 = make_float2(alpha, alpha);
-      const bool unit_alpha = __all_sync(0xffffffffu, alpha == 1.0f);
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t pv[32], o[32];
-        tmem_ld32(trow + c * 32, pv);
-        if (j > 0) tmem_ld32(trow + kColO + c * 32, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float2 x;
-          if constexpr (kInt8) {
-            x = fadd2(make_float2(__int_as_float(static_cast<int>(pv[e]) + 0x4B400000),
-                                  __int_as_float(static_cast<int>(pv[e + 1]) + 0x4B400000)),
-                      make_float2(-12582912.0f, -12582912.0f));
-          } else {
-            x = make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
-          }
-          float2 y;
-          if (j == 0) {
-            y = fmul2(x, c2);
-          } else {
-            const float2 prev = make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1]));
-            y = ffma2(x, c2, unit_alpha ? prev : fmul2(prev, a2));
-          }
-          o[e] = __float_as_uint(y.x);
-          o[e + 1] = __float_as_uint(y.y);
-        }
-        tmem_st32(trow + kColO + c * 32, o);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_free);
-    }
-    // epilogue: out = O / l (bf16), lse. TMEM reads are done by the whole
-    // warp; only the stores depend on the row.
-    if (ok && ntiles > 0) {
-      const bool store = qrow < p.Nq;
-      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      __nv_bfloat16* orow = p.out + row_offset(p.layout, p.H, p.Nq, D, b, h, store ? qrow : 0);
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(trow + kColO + c * 32, o);
-        tmem_wait_ld();
-        uint32_t wds[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-          wds[e] = *reinterpret_cast<const uint32_t*>(&t2);
-        }
-        if (store) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = make_uint4(wds[4 * q4], wds[4 * q4 + 1], wds[4 * q4 + 2], wds[4 * q4 + 3]);
-        }
-      }
-      if (store && p.lse) p.lse[static_cast<int64_t>(bh) * p.Nq + qrow] = m_run * 0.6931471805599453f + logf(l_run);
-    }
+    named_bar_sync(1, 256);
+    if (qt2[x] >= 0)
+      tile_rows<D, kInt8>(p, bars[x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN, sKsc, sVsc,
+                          qt2[x], nt2[x], bh, b, h, warp & 3, lane, &abort_flag);
   }
 
   tc_fence_before();
@@ -460,45 +576,24 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Host side
 // ---------------------------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 // 4-D map {D, N, H, B} over 8-bit codes; box {D, 128, 1, 1}: one tile of 128
 // token rows of one head lands as 128 rows of D bytes (swizzled).
 bool make_map(CUtensorMap* m, const void* base, int layout, int B, int H, int N, int D) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(H),
-                        static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[3];
+  const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N), static_cast<uint64_t>(H),
+                            static_cast<uint64_t>(B)};
+  uint64_t strides[3];
   if (layout == 0) {
-    strides[0] = static_cast<cuuint64_t>(D);
-    strides[1] = static_cast<cuuint64_t>(N) * D;
-    strides[2] = static_cast<cuuint64_t>(H) * N * D;
+    strides[0] = static_cast<uint64_t>(D);
+    strides[1] = static_cast<uint64_t>(N) * D;
+    strides[2] = static_cast<uint64_t>(H) * N * D;
   } else {
-    strides[0] = static_cast<cuuint64_t>(H) * D;
-    strides[1] = static_cast<cuuint64_t>(D);
-    strides[2] = static_cast<cuuint64_t>(N) * H * D;
+    strides[0] = static_cast<uint64_t>(H) * D;
+    strides[1] = static_cast<uint64_t>(D);
+    strides[2] = static_cast<uint64_t>(N) * H * D;
   }
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(kTileM), 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const uint32_t box[4] = {static_cast<uint32_t>(D), static_cast<uint32_t>(kTileM), 1, 1};
+  return encode_map_u8(m, 4, base, dims, strides, box,
+                       D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 template <int D, bool kInt8>
@@ -513,6 +608,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   p.lse = a.lse;
   p.B = a.B; p.H = a.H; p.Nq = a.Nq; p.Nkv = a.Nkv;
   p.nqt = (a.Nq + kTileM - 1) / kTileM;
+  p.npairs = (p.nqt + 1) / 2;
   p.nqb = (a.Nq + 127) / 128;
   p.nkb = (a.Nkv + 255) / 256;
   p.causal = a.causal;
@@ -522,7 +618,13 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   auto k = prefill_kernel<D, kInt8>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::kBytes);
   if (e != cudaSuccess) return e;
-  const int64_t grid = static_cast<int64_t>(p.nqt) * a.B * a.H;
+  // The register split inside the kernel needs at least kRegsNeeded
+  // registers per thread at launch; never launch with fewer.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, k);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < kRegsNeeded) return cudaErrorInvalidConfiguration;
+  const int64_t grid = static_cast<int64_t>(p.npairs) * a.B * a.H;
   k<<<static_cast<unsigned>(grid), kThreads, Smem<D>::kBytes, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }
