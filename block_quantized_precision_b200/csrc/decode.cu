@@ -61,6 +61,7 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStep = 16;             // tokens per consumer step
 constexpr int kWsStride = kD + 4;     // floats per (b, h_q, split) partial: O[D], m, l, pad
 constexpr int kVhStride = kD + 8;     // halves per row of the per-warp V' tile (conflict-free ldmatrix)
+constexpr int kPStride = 20;          // floats per head row of the per-warp P' buffer
 constexpr uint32_t kOnesF16x2 = 0x3C003C00u;
 constexpr int kCtasPerSm = 2;         // resident CTAs per SM (registers)
 
@@ -155,7 +156,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __shared__ __align__(16) uint32_t sQw[G][kD / 4];    // query codes, 4 per word (natural order)
   __shared__ int sQsum[G][2];                          // sum of query codes per 64-channel half
   __shared__ float sQf[G];                             // sq * softmax scale * log2(e)
-  __shared__ __align__(16) float sPw[kConsumers][kGroups][8][kStep];   // P'[head][token], per warp
+  // P'[head][token] per warp; rows of kPStride floats keep the stores of a
+  // warp on distinct banks
+  __shared__ __align__(16) float sPw[kConsumers][kGroups][8][kPStride];
   __shared__ float sAlpha[kConsumers][8];
   __shared__ float sKsc[kStages], sVsc[kStages], sVmax[kStages];
   __shared__ uint16_t sKs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
@@ -327,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
   __half* myVh = sVh + warp * kStep * kVhStride;
-  float (*myP)[8][kStep] = sPw[warp];
+  float (*myP)[8][kPStride] = sPw[warp];
   const uint32_t vh_base = smem_u32(myVh);
   // ldmatrix row address of this lane: matrix lane/8 = (token half, n-tile
   // of the pair), row lane%8
@@ -458,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       // ---------------- V' rows of this step -> fp16 tile ----------------
       {
-        const int t = lane >> 1, hf = lane & 1;               // token row, half of its channels
+        const int t = lane & 15, hf = lane >> 4;              // token row, half of its channels
         const int vr = r0 + t;
         __half* dst = myVh + t * kVhStride + hf * 64;
         if constexpr (!kInt4) {

@@ -139,29 +139,147 @@ struct TileBars {
   uint64_t pv_free;   // PV_j read by the rows     (128 row threads)
 };
 
-// O = alpha * O + g * PV for this thread's row: PV read from TMEM 32 columns
-// at a time. `scale_o` is false when alpha == 1 for every lane of the warp.
-template <int D, bool kInt8>
-__device__ __forceinline__ void fold_pv(float (&O)[D], uint32_t tPV, float alpha, float g, bool scale_o) {
-  const float2 a2 = make_float2(alpha, alpha);
-  const float2 g2 = make_float2(g, g);
+// Calls body(c, v) for the 16-column chunks c = 0..N-1 of this thread's TMEM
+// lane starting at taddr; chunk c + 1 is loaded while chunk c is processed.
+template <int N, typename F>
+__device__ __forceinline__ void tmem_chunks(uint32_t taddr, F&& body) {
+  uint32_t a[16], b[16];
+  tmem_ld16(taddr, a);
+  tmem_wait_ld();
+  reg_fence(a);
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t pv[32];
-    tmem_ld32(tPV + c * 32, pv);
-    tmem_wait_ld();
-    reg_fence(pv);
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const float2 x = kInt8 ? s32x2_to_f32x2(pv[e], pv[e + 1])
-                             : make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
-      float2 o = make_float2(O[c * 32 + e], O[c * 32 + e + 1]);
-      if (scale_o) o = fmul2(o, a2);
-      o = ffma2(x, g2, o);
-      O[c * 32 + e] = o.x;
-      O[c * 32 + e + 1] = o.y;
+  for (int c = 0; c < N; ++c) {
+    uint32_t(&cur)[16] = (c & 1) ? b : a;
+    uint32_t(&nxt)[16] = (c & 1) ? a : b;
+    if (c + 1 < N) tmem_ld16(taddr + (c + 1) * 16, nxt);
+    body(c, cur);
+    if (c + 1 < N) {
+      tmem_wait_ld();
+      reg_fence(nxt);
     }
   }
+}
+
+// O = alpha * O + g * PV for this thread's row (kScaleO false: alpha == 1
+// for every lane of the warp).
+template <int D, bool kInt8, bool kScaleO>
+__device__ __forceinline__ void fold_pv(float (&O)[D], uint32_t tPV, float alpha, float g) {
+  const float2 a2 = make_float2(alpha, alpha);
+  const float2 g2 = make_float2(g, g);
+  tmem_chunks<D / 16>(tPV, [&](int c, uint32_t(&pv)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const float2 x = kInt8 ? s32x2_to_f32x2(pv[e], pv[e + 1])
+                             : make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
+      float2 o = make_float2(O[c * 16 + e], O[c * 16 + e + 1]);
+      if constexpr (kScaleO) o = fmul2(o, a2);
+      o = ffma2(x, g2, o);
+      O[c * 16 + e] = o.x;
+      O[c * 16 + e + 1] = o.y;
+    }
+  });
+}
+
+// Row max of one 128-key tile of S, scaled: INT8 the integer max of the
+// INT32 scores, FP8 the float max; keys >= kmax are masked when kPartial.
+// Returns -inf if every key is masked.
+template <bool kInt8, bool kPartial>
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc) {
+  if constexpr (kInt8) {
+    int i0 = INT_MIN, i1 = INT_MIN, i2 = INT_MIN, i3 = INT_MIN;
+    tmem_chunks<kTileN / 16>(tS, [&](int c, uint32_t(&v)[16]) {
+      if constexpr (kPartial) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (c * 16 + e >= kmax) v[e] = 0x80000000u;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        i0 = max(i0, static_cast<int>(v[e]));
+        i1 = max(i1, static_cast<int>(v[e + 1]));
+        i2 = max(i2, static_cast<int>(v[e + 2]));
+        i3 = max(i3, static_cast<int>(v[e + 3]));
+      }
+    });
+    const int im = max(max(i0, i1), max(i2, i3));
+    return im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
+  } else {
+    float f0 = -CUDART_INF_F, f1 = -CUDART_INF_F, f2 = -CUDART_INF_F, f3 = -CUDART_INF_F;
+    tmem_chunks<kTileN / 16>(tS, [&](int c, uint32_t(&v)[16]) {
+      if constexpr (kPartial) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (c * 16 + e >= kmax) v[e] = 0xFF800000u;        // -inf
+      }
+#pragma unroll
+      for (int e = 0; e < 16; e += 8) {
+        f0 = fmax3(f0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        f1 = fmax3(f1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        f2 = fmax3(f2, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+        f3 = fmax3(f3, __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+      }
+    });
+    const float fm = fmaxf(fmaxf(f0, f1), fmaxf(f2, f3));
+    return fm == -CUDART_INF_F ? -CUDART_INF_F : fm * ksc;
+  }
+}
+
+// Probabilities of one 128-key tile, rounded to 8 bits and written to this
+// row of P in shared memory (128-byte swizzled K-major rows); returns the row
+// sum of the rounded values. t = S * ksc + toff; INT8: code = RNE(2^t) with
+// toff = log2(127) - m (so 2^t = 127 p); FP8: e4m3(2^t) with toff = -m.
+template <bool kInt8, bool kPartial>
+__device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw, float ksc, float toff, int kmax) {
+  const float2 k2 = make_float2(ksc, ksc);
+  const float2 t2 = make_float2(toff, toff);
+  int ri0 = 0, ri1 = 0;
+  float rf0 = 0.0f, rf1 = 0.0f, rf2 = 0.0f, rf3 = 0.0f;
+  tmem_chunks<kTileN / 16>(tS, [&](int c, uint32_t(&v)[16]) {
+    uint32_t packed[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      float2 t01, t23;
+      if constexpr (kInt8) {
+        t01 = ffma2(s32x2_to_f32x2(v[4 * w], v[4 * w + 1]), k2, t2);
+        t23 = ffma2(s32x2_to_f32x2(v[4 * w + 2], v[4 * w + 3]), k2, t2);
+      } else {
+        t01 = ffma2(make_float2(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1])), k2, t2);
+        t23 = ffma2(make_float2(__uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3])), k2, t2);
+      }
+      float pr[4] = {ex2(t01.x), ex2(t01.y), ex2(t23.x), ex2(t23.y)};
+      if constexpr (kPartial) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = c * 16 + w * 4 + e < kmax ? pr[e] : 0.0f;
+      }
+      if constexpr (kInt8) {
+        // adding 1.5 * 2^23 rounds to an integer (half to even) and leaves it
+        // in the low mantissa byte
+        const float2 q01 = fadd2(make_float2(pr[0], pr[1]), make_float2(12582912.0f, 12582912.0f));
+        const float2 q23 = fadd2(make_float2(pr[2], pr[3]), make_float2(12582912.0f, 12582912.0f));
+        const uint32_t b01 = __byte_perm(__float_as_uint(q01.x), __float_as_uint(q01.y), 0x0040);
+        const uint32_t b23 = __byte_perm(__float_as_uint(q23.x), __float_as_uint(q23.y), 0x0040);
+        const uint32_t word = __byte_perm(b01, b23, 0x5410);
+        if (w & 1) ri1 = __dp4a(static_cast<int>(word), 0x01010101, ri1);
+        else ri0 = __dp4a(static_cast<int>(word), 0x01010101, ri0);
+        packed[w] = word;
+      } else {
+        const uint32_t lo = cvt_e4m3x2(pr[0], pr[1]);
+        const uint32_t hi = cvt_e4m3x2(pr[2], pr[3]);
+        packed[w] = lo | (hi << 16);
+        // row sum of the rounded probabilities (exact values via fp16)
+        if (w & 1) {
+          rf2 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rf2);
+          rf3 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rf3);
+        } else {
+          rf0 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rf0);
+          rf1 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rf1);
+        }
+      }
+    }
+    // keys 16c .. 16c+15 = 16-byte chunk c of this row
+    *reinterpret_cast<uint4*>(prow + ((c ^ rsw) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  });
+  return kInt8 ? static_cast<float>(ri0 + ri1) * (1.0f / 127.0f) : (rf0 + rf1) + (rf2 + rf3);
 }
 
 // The rows of one query tile (4 warps, one row per thread).
@@ -199,55 +317,8 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     int kmax = p.Nkv - key0;                    // keys valid for this row: [0, kmax)
     if (p.causal) kmax = min(kmax, qrow - key0 + 1);
 
-    // ---- (1) row max: integer max of the INT32 scores, or float max ----
-    float tmax;
-    if constexpr (kInt8) {
-      int i0 = INT_MIN, i1 = INT_MIN, i2 = INT_MIN, i3 = INT_MIN;
-#pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        if (partial) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e >= kmax) v[e] = 0x80000000u;
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          i0 = max(i0, static_cast<int>(v[e]));
-          i1 = max(i1, static_cast<int>(v[e + 1]));
-          i2 = max(i2, static_cast<int>(v[e + 2]));
-          i3 = max(i3, static_cast<int>(v[e + 3]));
-        }
-      }
-      const int im = max(max(i0, i1), max(i2, i3));
-      tmax = im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
-    } else {
-      float f0 = -CUDART_INF_F, f1 = -CUDART_INF_F, f2 = -CUDART_INF_F, f3 = -CUDART_INF_F;
-#pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        if (partial) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e >= kmax) v[e] = 0xFF800000u;        // -inf
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          f0 = fmax3(f0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-          f1 = fmax3(f1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-          f2 = fmax3(f2, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
-          f3 = fmax3(f3, __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
-        }
-      }
-      const float fm = fmaxf(fmaxf(f0, f1), fmaxf(f2, f3));
-      tmax = fm == -CUDART_INF_F ? -CUDART_INF_F : fm * ksc;
-    }
+    // ---- (1) row max ----
+    const float tmax = partial ? tile_row_max<kInt8, true>(tS, kmax, ksc) : tile_row_max<kInt8, false>(tS, kmax, ksc);
     const float m_new = fmaxf(m_run, tmax);
     const float m_use = m_new == -CUDART_INF_F ? 0.0f : m_new;
     const float alpha = ex2(m_run - m_use);     // 0 on the first tile
@@ -260,71 +331,9 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     }
 
     // ---- (2) probabilities, 8-bit rounding, P to shared memory ----
-    // INT8: code = RNE(127 p) taken as RNE(2^(t + log2 127)); FP8: e4m3(p).
-    const float2 k2 = make_float2(ksc, ksc);
     const float toff = (kInt8 ? kLog2_127 : 0.0f) - m_use;
-    const float2 t2 = make_float2(toff, toff);
-    float rowsum;
-    {
-      int ri0 = 0, ri1 = 0;
-      float rf0 = 0.0f, rf1 = 0.0f, rf2 = 0.0f, rf3 = 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < kTileN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_wait_ld();
-        reg_fence(v);
-        uint32_t packed[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          float2 t01, t23;
-          if constexpr (kInt8) {
-            t01 = ffma2(s32x2_to_f32x2(v[4 * w], v[4 * w + 1]), k2, t2);
-            t23 = ffma2(s32x2_to_f32x2(v[4 * w + 2], v[4 * w + 3]), k2, t2);
-          } else {
-            t01 = ffma2(make_float2(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1])), k2, t2);
-            t23 = ffma2(make_float2(__uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3])), k2, t2);
-          }
-          float pr[4] = {ex2(t01.x), ex2(t01.y), ex2(t23.x), ex2(t23.y)};
-          if (partial) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) pr[e] = c * 32 + w * 4 + e < kmax ? pr[e] : 0.0f;
-          }
-          if constexpr (kInt8) {
-            // adding 1.5 * 2^23 rounds to an integer (half to even) and leaves
-            // it in the low mantissa byte
-            const float2 q01 = fadd2(make_float2(pr[0], pr[1]), make_float2(12582912.0f, 12582912.0f));
-            const float2 q23 = fadd2(make_float2(pr[2], pr[3]), make_float2(12582912.0f, 12582912.0f));
-            const uint32_t b01 = __byte_perm(__float_as_uint(q01.x), __float_as_uint(q01.y), 0x0040);
-            const uint32_t b23 = __byte_perm(__float_as_uint(q23.x), __float_as_uint(q23.y), 0x0040);
-            const uint32_t word = __byte_perm(b01, b23, 0x5410);
-            if (w & 1) ri1 = __dp4a(static_cast<int>(word), 0x01010101, ri1);
-            else ri0 = __dp4a(static_cast<int>(word), 0x01010101, ri0);
-            packed[w] = word;
-          } else {
-            const uint32_t lo = cvt_e4m3x2(pr[0], pr[1]);
-            const uint32_t hi = cvt_e4m3x2(pr[2], pr[3]);
-            packed[w] = lo | (hi << 16);
-            // row sum of the rounded probabilities (exact values via fp16)
-            if (w & 1) {
-              rf2 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rf2);
-              rf3 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rf3);
-            } else {
-              rf0 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(lo)), rf0);
-              rf1 = add_f32_f16x2(cvt_e4m3x2_to_f16x2(static_cast<uint16_t>(hi)), rf1);
-            }
-          }
-        }
-        // keys c*32 .. c*32+31 = 16-byte chunks 2c and 2c+1 of this row
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          const int chunk = 2 * c + hc;
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ rsw) << 4)) =
-              make_uint4(packed[4 * hc], packed[4 * hc + 1], packed[4 * hc + 2], packed[4 * hc + 3]);
-        }
-      }
-      rowsum = kInt8 ? static_cast<float>(ri0 + ri1) * (1.0f / 127.0f) : (rf0 + rf1) + (rf2 + rf3);
-    }
+    const float rowsum = partial ? tile_probs<kInt8, true>(tS, prow, rsw, ksc, toff, kmax)
+                                 : tile_probs<kInt8, false>(tS, prow, rsw, ksc, toff, kmax);
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(&bars.p_full);
@@ -334,8 +343,8 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     // ---- (3) fold PV_{j-1}: O <- alpha_j (O + g_{j-1} PV_{j-1}) ----
     // (O is kept relative to the newest running max.)
     if (j > 0) {
-      const bool scale_o = !__all_sync(0xffffffffu, alpha == 1.0f);
-      fold_pv<D, kInt8>(O, tPV, alpha, alpha * g_prev, scale_o);
+      if (__all_sync(0xffffffffu, alpha == 1.0f)) fold_pv<D, kInt8, false>(O, tPV, alpha, alpha * g_prev);
+      else fold_pv<D, kInt8, true>(O, tPV, alpha, alpha * g_prev);
       tc_fence_before();
       mbar_arrive(&bars.pv_free);
     }
@@ -346,7 +355,7 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
   ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_full, (ntiles - 1) & 1, abort_flag, p.err));
   if (!ok) return;
   tc_fence_after();
-  fold_pv<D, kInt8>(O, tPV, 1.0f, g_prev, false);
+  fold_pv<D, kInt8, false>(O, tPV, 1.0f, g_prev);
 
   // epilogue: out = O / l (bf16), lse
   if (qrow < p.Nq) {
