@@ -27,8 +27,10 @@
 //                         sums); the query codes live in 8 registers
 //                 softmax per head over the 16 tokens (shuffles), running
 //                         max / sum in the log2 domain
-//                 P.V     O[heads x 128] += P' V' by mma.m16n8k16 f16 x f16
-//                         -> f32. P' = p * (v scale / running max v scale)
+//                 P.V     O^T[128 x heads] += V'^T P'^T by mma.m16n8k16
+//                         f16 x f16 -> f32 (channels fill the 16-row side,
+//                         heads the 8-column side). P' = p * (v scale /
+//                         running max v scale)
 //                         in [0, 1], split into an fp16 high part and an fp16
 //                         remainder (two MMAs, ~22 significant bits). V' is
 //                         the code plus a constant offset, exact in fp16 and
@@ -106,16 +108,15 @@ __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, ui
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// D[16x8] += A[16x16] B[16x8], fp16 inputs, fp32 accumulation. Rows 8..15 of
-// A are zero here (at most 8 query heads), so only the first two accumulator
-// registers carry data; the other two are scratch.
-__device__ __forceinline__ void mma_f16(float& c0, float& c1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  float z0 = 0.0f, z1 = 0.0f;
+// D[16x8] += A[16x16] B[16x8], fp16 inputs, fp32 accumulation (all four
+// accumulator registers used).
+__device__ __forceinline__ void mma_f16x4(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
-      : "+f"(c0), "+f"(c1), "+f"(z0), "+f"(z1)
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -159,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // P'[head][token] per warp; rows of kPStride floats keep the stores of a
   // warp on distinct banks
   __shared__ __align__(16) float sPw[kConsumers][kGroups][8][kPStride];
-  __shared__ float sAlpha[kConsumers][8];
   __shared__ float sKsc[kStages], sVsc[kStages], sVmax[kStages];
   __shared__ uint16_t sKs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
   __shared__ uint16_t sVs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
@@ -332,20 +332,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __half* myVh = sVh + warp * kStep * kVhStride;
   float (*myP)[8][kPStride] = sPw[warp];
   const uint32_t vh_base = smem_u32(myVh);
-  // ldmatrix row address of this lane: matrix lane/8 = (token half, n-tile
-  // of the pair), row lane%8
+  // P.V is computed transposed, O^T[channels x heads] += V'^T P'^T: A = V'^T
+  // (16 channels x 16 tokens) by ldmatrix.trans from the [token][channel]
+  // tile, B = P'^T (16 tokens x 8 heads). ldmatrix row address of this lane:
+  // matrix lane/8 = (token half = lane/16, channel half = (lane/8)%2), row
+  // lane%8.
   const uint32_t ldsm_off =
-      static_cast<uint32_t>(((((lane >> 3) & 1) * 8 + (lane & 7)) * kVhStride + ((lane >> 4) * 8)) * 2);
+      static_cast<uint32_t>((((lane >> 4) * 8 + (lane & 7)) * kVhStride + (((lane >> 3) & 1) * 8)) * 2);
 
   float m_run0 = -CUDART_INF_F, m_run1 = -CUDART_INF_F;   // heads h0, h1
   float l_run0 = 0.0f, l_run1 = 0.0f;                      // over this lane's tokens
   float vref = 0.0f;                                       // running max V scale
-  float acc[16][2];                                        // head gq, stored columns 8nt + 2cq, +1
-  float sacc[kGroups][2];                                  // sum of P' per group (head gq)
+  // acc[mt]: stored channels 16mt + gq ([0] head h0, [1] head h1) and
+  // 16mt + gq + 8 ([2] h0, [3] h1); sacc[gg]: sum of P' of group gg for
+  // heads h0 ([0]) and h1 ([1]).
+  float acc[8][4];
+  float sacc[kGroups][4];
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = 0.0f;
+  for (int mt = 0; mt < 8; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
 #pragma unroll
-  for (int gg = 0; gg < kGroups; ++gg) sacc[gg][0] = sacc[gg][1] = 0.0f;
+  for (int gg = 0; gg < kGroups; ++gg) sacc[gg][0] = sacc[gg][1] = sacc[gg][2] = sacc[gg][3] = 0.0f;
 
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % kStages;
@@ -361,15 +367,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     vref = vref_new;
     if (vratio != 1.0f) {                     // the same on every lane
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        acc[nt][0] *= vratio;
-        acc[nt][1] *= vratio;
-      }
+      for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-      for (int gg = 0; gg < kGroups; ++gg) {
-        sacc[gg][0] *= vratio;
-        sacc[gg][1] *= vratio;
-      }
+        for (int e = 0; e < 4; ++e) acc[mt][e] *= vratio;
+#pragma unroll
+      for (int gg = 0; gg < kGroups; ++gg)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[gg][e] *= vratio;
     }
 #pragma unroll 1
     for (int sub = 0; sub < C::kPerWarp / kStep; ++sub) {
@@ -455,10 +459,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if (h1ok) { myP[gg][h1][gq] = pa1 * fa; myP[gg][h1][gq + 8] = pb1 * fb; }
         }
       }
-      if (gq == 0) {
-        sAlpha[warp][h0] = al0;
-        sAlpha[warp][h1] = al1;
-      }
       // ---------------- V' rows of this step -> fp16 tile ----------------
       {
         const int t = lane & 15, hf = lane >> 4;              // token row, half of its channels
@@ -500,23 +500,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
       }
       __syncwarp();
-      // ---------------- rescale O and sum(P') by alpha, P' as fp16 high / low ----------------
-      {
-        const float fac = gq < G ? sAlpha[warp][gq] : 1.0f;
-        if (!__all_sync(0xffffffffu, fac == 1.0f)) {
+      // ---------------- rescale O^T and sum(P') by alpha (heads h0, h1 of this lane) ----------------
+      if (!__all_sync(0xffffffffu, al0 == 1.0f && al1 == 1.0f)) {
 #pragma unroll
-          for (int nt = 0; nt < 16; ++nt) {
-            acc[nt][0] *= fac;
-            acc[nt][1] *= fac;
-          }
+        for (int mt = 0; mt < 8; ++mt) {
+          acc[mt][0] *= al0; acc[mt][1] *= al1; acc[mt][2] *= al0; acc[mt][3] *= al1;
+        }
 #pragma unroll
-          for (int gg = 0; gg < kGroups; ++gg) {
-            sacc[gg][0] *= fac;
-            sacc[gg][1] *= fac;
-          }
+        for (int gg = 0; gg < kGroups; ++gg) {
+          sacc[gg][0] *= al0; sacc[gg][1] *= al1; sacc[gg][2] *= al0; sacc[gg][3] *= al1;
         }
       }
-      uint32_t pa_hi[kGroups], pa_lo[kGroups], pb_hi[kGroups], pb_lo[kGroups];
+      // P'^T fragments (B): head gq, tokens 2cq, 2cq+1 (b0) and 2cq+8, 2cq+9
+      // (b1), as fp16 high and low parts
+      uint32_t p0_hi[kGroups], p0_lo[kGroups], p1_hi[kGroups], p1_lo[kGroups];
 #pragma unroll
       for (int gg = 0; gg < kGroups; ++gg) {
         float2 x01 = make_float2(0.0f, 0.0f), x89 = make_float2(0.0f, 0.0f);
@@ -524,24 +521,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           x01 = *reinterpret_cast<const float2*>(&myP[gg][gq][2 * cq]);
           x89 = *reinterpret_cast<const float2*>(&myP[gg][gq][2 * cq + 8]);
         }
-        split_f16x2(x01.x, x01.y, pa_hi[gg], pa_lo[gg]);
-        split_f16x2(x89.x, x89.y, pb_hi[gg], pb_lo[gg]);
+        split_f16x2(x01.x, x01.y, p0_hi[gg], p0_lo[gg]);
+        split_f16x2(x89.x, x89.y, p1_hi[gg], p1_lo[gg]);
       }
-      // ---------------- O += P' V', sum(P') against a tile of ones ----------------
+      // ---------------- O^T += V'^T P'^T, sum(P') against a tile of ones ----------------
 #pragma unroll
-      for (int np = 0; np < 8; ++np) {                        // pairs of 8-channel tiles
-        uint32_t b0a, b1a, b0b, b1b;
-        ldsm_x4_trans(vh_base + ldsm_off + np * 32, b0a, b1a, b0b, b1b);
-        const int gg = (kGroups == 2 && np >= 4) ? 1 : 0;
-        mma_f16(acc[2 * np][0], acc[2 * np][1], pa_hi[gg], pb_hi[gg], b0a, b1a);
-        mma_f16(acc[2 * np][0], acc[2 * np][1], pa_lo[gg], pb_lo[gg], b0a, b1a);
-        mma_f16(acc[2 * np + 1][0], acc[2 * np + 1][1], pa_hi[gg], pb_hi[gg], b0b, b1b);
-        mma_f16(acc[2 * np + 1][0], acc[2 * np + 1][1], pa_lo[gg], pb_lo[gg], b0b, b1b);
+      for (int mt = 0; mt < 8; ++mt) {                        // 16-channel tiles
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(vh_base + ldsm_off + mt * 32, a0, a1, a2, a3);
+        const int gg = (kGroups == 2 && mt >= 4) ? 1 : 0;
+        mma_f16x4(acc[mt], a0, a1, a2, a3, p0_hi[gg], p1_hi[gg]);
+        mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[gg], p1_lo[gg]);
       }
 #pragma unroll
       for (int gg = 0; gg < kGroups; ++gg) {
-        mma_f16(sacc[gg][0], sacc[gg][1], pa_hi[gg], pb_hi[gg], kOnesF16x2, kOnesF16x2);
-        mma_f16(sacc[gg][0], sacc[gg][1], pa_lo[gg], pb_lo[gg], kOnesF16x2, kOnesF16x2);
+        mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_hi[gg], p1_hi[gg]);
+        mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_lo[gg], p1_lo[gg]);
       }
       __syncwarp();                  // buffers reused by the next step
     }
@@ -563,25 +558,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (h0ok) { sWm[warp][h0] = m_run0; sWl[warp][h0] = l_run0; }
     if (h1ok) { sWm[warp][h1] = m_run1; sWl[warp][h1] = l_run1; }
   }
-  if (gq < G) {
-    // O = (acc - offset * sum(P')) * vref; INT4 odd channels also / 16
+  // O = (acc - offset * sum(P')) * vref; INT4 odd channels also / 16
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int gg = (kGroups == 2 && nt >= 8) ? 1 : 0;
+  for (int mt = 0; mt < 8; ++mt) {
+    const int gg = (kGroups == 2 && mt >= 4) ? 1 : 0;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = nt * 8 + 2 * cq + e;                 // stored column
-        float o;
-        int ch = col;
-        if constexpr (kInt4) {
-          const bool odd = (col & 2) != 0;                   // stored 0,2,1,3 -> channels 0,2 | 1,3
-          o = (acc[nt][e] - (odd ? kOffB : kOffA) * sacc[gg][0]) * (odd ? vref * 0.0625f : vref);
-          ch = (col & ~3) | ((col & 1) << 1) | ((col >> 1) & 1);
-        } else {
-          o = (acc[nt][e] - kOffA * sacc[gg][0]) * vref;
-        }
-        sRed[(warp * G + gq) * kD + ch] = o;
+    for (int e = 0; e < 4; ++e) {
+      const int hh = 2 * cq + (e & 1);
+      if (hh >= G) continue;
+      const int col = mt * 16 + gq + (e >> 1) * 8;           // stored column
+      const float sp = sacc[gg][e & 1];
+      float o;
+      int ch = col;
+      if constexpr (kInt4) {
+        const bool odd = (col & 2) != 0;                     // stored 0,2,1,3 -> channels 0,2 | 1,3
+        o = (acc[mt][e] - (odd ? kOffB : kOffA) * sp) * (odd ? vref * 0.0625f : vref);
+        ch = (col & ~3) | ((col & 1) << 1) | ((col >> 1) & 1);
+      } else {
+        o = (acc[mt][e] - kOffA * sp) * vref;
       }
+      sRed[(warp * G + hh) * kD + ch] = o;
     }
   }
   named_bar_sync(1, 32 * kConsumers);
