@@ -62,7 +62,6 @@ constexpr int kConsumers = 4;         // consumer warps
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStep = 16;             // tokens per consumer step
 constexpr int kWsStride = kD + 4;     // floats per (b, h_q, split) partial: O[D], m, l, pad
-constexpr int kVhStride = kD + 8;     // halves per row of the per-warp V' tile (conflict-free ldmatrix)
 constexpr int kPStride = 20;          // floats per head row of the per-warp P' buffer
 constexpr uint32_t kOnesF16x2 = 0x3C003C00u;
 constexpr int kCtasPerSm = 2;         // resident CTAs per SM (registers)
@@ -74,8 +73,7 @@ struct Cfg {
   static constexpr int kStages = kInt4 ? 3 : 4;
   static constexpr int kTileBytes = kChunk * kRowBytes;       // one tensor, one stage (8 KB)
   static constexpr int kPerWarp = kChunk / kConsumers;        // tokens per warp per chunk
-  static constexpr int kVhBytes = kConsumers * kStep * kVhStride * 2;
-  static constexpr int kSmemBytes = 2 * kStages * kTileBytes + kVhBytes + 1024;
+  static constexpr int kSmemBytes = 2 * kStages * kTileBytes + 1024;
 };
 
 struct DecodeParams {
@@ -151,7 +149,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;                          // [stages][chunk rows], swizzled
   uint8_t* sV = smem + kStages * kTile;
-  __half* sVh = reinterpret_cast<__half*>(smem + 2 * kStages * kTile);   // [warp][16][kVhStride]
   float* sRed = reinterpret_cast<float*>(smem);   // after the loop: [warps][G][D]
 
   __shared__ __align__(16) uint32_t sQw[G][kD / 4];    // query codes, 4 per word (natural order)
@@ -329,17 +326,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       qs0[0] = 8 * (s00 + s01); qs1[0] = 8 * (s10 + s11);
     }
   }
-  __half* myVh = sVh + warp * kStep * kVhStride;
   float (*myP)[8][kPStride] = sPw[warp];
-  const uint32_t vh_base = smem_u32(myVh);
-  // P.V is computed transposed, O^T[channels x heads] += V'^T P'^T: A = V'^T
-  // (16 channels x 16 tokens) by ldmatrix.trans from the [token][channel]
-  // tile, B = P'^T (16 tokens x 8 heads). ldmatrix row address of this lane:
-  // matrix lane/8 = (token half = lane/16, channel half = (lane/8)%2), row
-  // lane%8.
-  const uint32_t ldsm_off =
-      static_cast<uint32_t>((((lane >> 4) * 8 + (lane & 7)) * kVhStride + (((lane >> 3) & 1) * 8)) * 2);
-
+  // P.V is computed transposed, O^T[channels x heads] += V'^T P'^T, with
+  // A = V'^T taken straight from the swizzled V tile: ldmatrix.trans on
+  // 2-byte elements gives each lane, for tokens (2cq, 2cq+1) of a 16-token
+  // step, the bytes of one 2-byte element (2 INT8 channels / 4 INT4
+  // channels) of both tokens; byte permutes turn them into fp16 pairs
+  // (V' = code + offset, exact). Rows of each 16-channel MMA tile are
+  // therefore a permutation of the channels, undone at the output.
+  // ldmatrix row of this lane: matrix lane/8 = (token half = (lane/8)%2,
+  // 16-byte chunk offset = lane/16), row lane%8 = token.
+  const int ldsm_tok = ((lane >> 3) & 1) * 8 + (lane & 7);
+  const int ldsm_chunk = lane >> 4;
   float m_run0 = -CUDART_INF_F, m_run1 = -CUDART_INF_F;   // heads h0, h1
   float l_run0 = 0.0f, l_run1 = 0.0f;                      // over this lane's tokens
   float vref = 0.0f;                                       // running max V scale
@@ -459,46 +457,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if (h1ok) { myP[gg][h1][gq] = pa1 * fa; myP[gg][h1][gq + 8] = pb1 * fb; }
         }
       }
-      // ---------------- V' rows of this step -> fp16 tile ----------------
-      {
-        const int t = lane & 15, hf = lane >> 4;              // token row, half of its channels
-        const int vr = r0 + t;
-        __half* dst = myVh + t * kVhStride + hf * 64;
-        if constexpr (!kInt4) {
-          // byte b -> fp16 with bits 0x64 | (b ^ 0x80) = 1152 + b (exact)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 w = *reinterpret_cast<const uint4*>(cV + vr * 128 + (((hf * 4 + i) ^ (vr & 7)) << 4));
-            const uint32_t ws[4] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u, w.z ^ 0x80808080u, w.w ^ 0x80808080u};
-            uint32_t hv[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              hv[2 * k] = __byte_perm(ws[k], 0x64646464u, 0x5140);
-              hv[2 * k + 1] = __byte_perm(ws[k], 0x64646464u, 0x7362);
-            }
-            *reinterpret_cast<uint4*>(dst + i * 16) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<uint4*>(dst + i * 16 + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-          }
-        } else {
-          // byte pair (b0, b1) = channels (8k, 8k+1), (8k+2, 8k+3) ->
-          //   even channels: 0x64 | 0x08 ^ low nibble      = 1032 + code
-          //   odd channels:  0x64 | (0x80 ^ high nibble<<4) = 1152 + 16 code
-          // stored per 4 channels in the order 0, 2, 1, 3
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const uint4 w = *reinterpret_cast<const uint4*>(cV + vr * 64 + (((hf * 2 + i) ^ ((vr >> 1) & 3)) << 4));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t lo = __byte_perm(ws[k], 0u, 0x4140);     // b0, 0, b1, 0
-              const uint32_t hi = __byte_perm(ws[k], 0u, 0x4342);     // b2, 0, b3, 0
-              const uint4 out = make_uint4((lo & 0x000F000Fu) ^ 0x64086408u, (lo & 0x00F000F0u) ^ 0x64806480u,
-                                           (hi & 0x000F000Fu) ^ 0x64086408u, (hi & 0x00F000F0u) ^ 0x64806480u);
-              *reinterpret_cast<uint4*>(dst + i * 32 + k * 8) = out;
-            }
-          }
-        }
-      }
       __syncwarp();
       // ---------------- rescale O^T and sum(P') by alpha (heads h0, h1 of this lane) ----------------
       if (!__all_sync(0xffffffffu, al0 == 1.0f && al1 == 1.0f)) {
@@ -525,13 +483,47 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         split_f16x2(x89.x, x89.y, p1_hi[gg], p1_lo[gg]);
       }
       // ---------------- O^T += V'^T P'^T, sum(P') against a tile of ones ----------------
+      {
+        const int vt = r0 + ldsm_tok;                        // this lane's ldmatrix row (token)
+        const uint32_t vrow = smem_u32(cV + vt * C::kRowBytes);
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {                        // 16-channel tiles
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_trans(vh_base + ldsm_off + mt * 32, a0, a1, a2, a3);
-        const int gg = (kGroups == 2 && mt >= 4) ? 1 : 0;
-        mma_f16x4(acc[mt], a0, a1, a2, a3, p0_hi[gg], p1_hi[gg]);
-        mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[gg], p1_lo[gg]);
+        for (int cp = 0; cp < (kInt4 ? 2 : 4); ++cp) {        // pairs of 16-byte chunks
+          const int chunk = 2 * cp + ldsm_chunk;
+          const int pos = kInt4 ? (chunk ^ ((vt >> 1) & 3)) : (chunk ^ (vt & 7));
+          uint32_t r[4];                                     // (tokens 0-7 | 8-15) x (chunk 2cp | 2cp+1)
+          ldsm_x4_trans(vrow + (pos << 4), r[0], r[1], r[2], r[3]);
+          if constexpr (!kInt4) {
+            // chunk 2cp + h -> m-tile 2cp + h: row g = channel 2g, row g+8 =
+            // channel 2g+1 of the chunk; byte b -> fp16 bits 0x64 | (b ^ 0x80)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t xl = r[2 * h] ^ 0x80808080u, xh = r[2 * h + 1] ^ 0x80808080u;
+              const uint32_t a0 = __byte_perm(xl, 0x64646464u, 0x4240), a1 = __byte_perm(xl, 0x64646464u, 0x4341);
+              const uint32_t a2 = __byte_perm(xh, 0x64646464u, 0x4240), a3 = __byte_perm(xh, 0x64646464u, 0x4341);
+              const int mt = 2 * cp + h;
+              mma_f16x4(acc[mt], a0, a1, a2, a3, p0_hi[0], p1_hi[0]);
+              mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[0], p1_lo[0]);
+            }
+          } else {
+            // chunk 2cp + h (32 channels) -> m-tiles 4cp + 2h + u: row g =
+            // channel 4g + 2u (low nibble, 1032 + code), row g+8 = channel
+            // 4g + 2u + 1 (high nibble, 1152 + 16 code)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const uint32_t yl = __byte_perm(r[2 * h], 0u, u ? 0x4341 : 0x4240);
+                const uint32_t yh = __byte_perm(r[2 * h + 1], 0u, u ? 0x4341 : 0x4240);
+                const uint32_t a0 = (yl & 0x000F000Fu) ^ 0x64086408u, a1 = (yl & 0x00F000F0u) ^ 0x64806480u;
+                const uint32_t a2 = (yh & 0x000F000Fu) ^ 0x64086408u, a3 = (yh & 0x00F000F0u) ^ 0x64806480u;
+                const int mt = 4 * cp + 2 * h + u;
+                const int gg = (kGroups == 2 && mt >= 4) ? 1 : 0;
+                mma_f16x4(acc[mt], a0, a1, a2, a3, p0_hi[gg], p1_hi[gg]);
+                mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[gg], p1_lo[gg]);
+              }
+            }
+          }
+        }
       }
 #pragma unroll
       for (int gg = 0; gg < kGroups; ++gg) {
@@ -558,7 +550,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (h0ok) { sWm[warp][h0] = m_run0; sWl[warp][h0] = l_run0; }
     if (h1ok) { sWm[warp][h1] = m_run1; sWl[warp][h1] = l_run1; }
   }
-  // O = (acc - offset * sum(P')) * vref; INT4 odd channels also / 16
+  // O = (acc - offset * sum(P')) * vref; INT4 odd channels also / 16.
+  // Row g of m-tile mt holds channel 16mt + 2g (INT8) or 32(mt/4)... see the
+  // P.V comment: INT8 rows g / g+8 = channels 16mt + 2g / +1; INT4 rows
+  // g / g+8 = channels 32(mt/2) + 4g + 2(mt%2) / +1.
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
     const int gg = (kGroups == 2 && mt >= 4) ? 1 : 0;
@@ -566,15 +561,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int e = 0; e < 4; ++e) {
       const int hh = 2 * cq + (e & 1);
       if (hh >= G) continue;
-      const int col = mt * 16 + gq + (e >> 1) * 8;           // stored column
+      const bool odd = (e >> 1) != 0;                        // row g+8
       const float sp = sacc[gg][e & 1];
       float o;
-      int ch = col;
+      int ch;
       if constexpr (kInt4) {
-        const bool odd = (col & 2) != 0;                     // stored 0,2,1,3 -> channels 0,2 | 1,3
+        ch = 32 * (mt >> 1) + 4 * gq + 2 * (mt & 1) + (odd ? 1 : 0);
         o = (acc[mt][e] - (odd ? kOffB : kOffA) * sp) * (odd ? vref * 0.0625f : vref);
-        ch = (col & ~3) | ((col & 1) << 1) | ((col >> 1) & 1);
       } else {
+        ch = 16 * mt + 2 * gq + (odd ? 1 : 0);
         o = (acc[mt][e] - kOffA * sp) * vref;
       }
       sRed[(warp * G + hh) * kD + ch] = o;
