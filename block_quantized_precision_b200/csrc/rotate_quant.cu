@@ -237,14 +237,64 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
 // Without rotation
 // ---------------------------------------------------------------------------
 
-// One CTA per block; each thread owns kV = T*D/8/256 (rounded up) 16-byte
-// input vectors, kept in registers between the max and the code pass.
+// Codes of 8 values by the fast path of code_of alone (v0 = y * rcp), packed
+// little-endian into lo (values 0..3) and hi (4..7). Returns false when any
+// value is too close to a rounding boundary (or, for e4m3, in the subnormal
+// range) for v0 to be trusted; the caller then takes the exact path.
+template <bool kInt8>
+__device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
+  bool ok = true;
+  uint32_t t[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float v0 = f[e] * rcp;
+    if constexpr (kInt8) {
+      const float m = v0 + 12582912.0f;                  // RNE integer in the low mantissa bits
+      ok = ok && fabsf(v0 - (m - 12582912.0f)) <= 0.4999f;
+      t[e] = __float_as_uint(m);
+    } else {
+      const uint32_t bb = __float_as_uint(v0) & 0x7FFFFFFFu;
+      ok = ok && bb >= 0x3C800000u && abs(static_cast<int>(bb & 0xFFFFFu) - 0x80000) > 16;
+      t[e] = __float_as_uint(v0);
+    }
+  }
+  if constexpr (kInt8) {
+    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+  } else {
+    lo = cvt_e4m3x2(__uint_as_float(t[0]), __uint_as_float(t[1])) |
+         (cvt_e4m3x2(__uint_as_float(t[2]), __uint_as_float(t[3])) << 16);
+    hi = cvt_e4m3x2(__uint_as_float(t[4]), __uint_as_float(t[5])) |
+         (cvt_e4m3x2(__uint_as_float(t[6]), __uint_as_float(t[7])) << 16);
+  }
+  return ok;
+}
+
+// Codes of 8 values with the IEEE quotient for every value.
+template <bool kInt8>
+__device__ __noinline__ uint2 codes8_exact(uint4 raw, bool is_bf16, float scale) {
+  float f[8];
+  unpack8(raw, is_bf16, f);
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f[j], scale, 0.0f, true) << (8 * j);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f[j + 4], scale, 0.0f, true) << (8 * j);
+  return make_uint2(lo, hi);
+}
+
+// One CTA per block; each thread owns kVec = T*D/8/256 (rounded up) 16-byte
+// input vectors, kept in registers between the max and the code pass. Codes
+// are formed by the division-free fast path; the few vectors holding a value
+// it cannot decide are reloaded and coded with IEEE divisions afterwards,
+// which keeps the unrolled main loop small and branch-free.
 template <int D, int T, bool kInt8>
 __global__ void __launch_bounds__(kThreads)
     quant_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
                  uint8_t* __restrict__ codes, float* __restrict__ scales) {
   constexpr int kCG = D / 8;
   constexpr int kVec = (T * kCG + kThreads - 1) / kThreads;
+  static_assert(kVec <= 32, "fix-up mask");
   __shared__ float red[kThreads / 32];
   const int nblk = (N + T - 1) / T;
   const int blk = blockIdx.x % nblk;
@@ -275,10 +325,9 @@ __global__ void __launch_bounds__(kThreads)
   const float amax = block_max<kThreads>(m, red);
   const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
   const float rcp = __frcp_rn(scale);
-  const bool slow = scale < 1.17549435e-38f;
+  const bool slow = scale < 1.17549435e-38f;          // zero or subnormal scale: exact path
   if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
-  // (the rare exact-division fallback is an out-of-line call, which keeps
-  // this unrolled loop small enough for the instruction cache)
+  uint32_t fix = 0;
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
     const int idx = threadIdx.x + i * kThreads;
@@ -286,16 +335,24 @@ __global__ void __launch_bounds__(kThreads)
     if (idx < T * kCG && r < rows) {
       float f[8];
       unpack8(v[i], bf, f);
-      uint32_t lo = 0, hi = 0;
-      if (scale != 0.0f) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f[j], scale, rcp, slow) << (8 * j);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f[j + 4], scale, rcp, slow) << (8 * j);
+      uint32_t lo, hi;
+      const bool ok = codes8_fast<kInt8>(f, rcp, lo, hi);
+      if (ok && !slow) {
+        *reinterpret_cast<uint2*>(codes + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8) = make_uint2(lo, hi);
+      } else {
+        fix |= 1u << i;
       }
-      *reinterpret_cast<uint2*>(codes + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8) =
-          make_uint2(lo, hi);
     }
+  }
+  while (fix != 0) {
+    const int i = __ffs(fix) - 1;
+    fix &= fix - 1;
+    const int idx = threadIdx.x + i * kThreads;
+    const int r = idx / kCG, c = idx % kCG;
+    const int64_t off = row_offset(layout, H, N, D, b, h, n0 + r) + c * 8;
+    uint2 w = make_uint2(0, 0);
+    if (scale != 0.0f) w = codes8_exact<kInt8>(*reinterpret_cast<const uint4*>(x + off), bf, scale);
+    *reinterpret_cast<uint2*>(codes + off) = w;
   }
 }
 
