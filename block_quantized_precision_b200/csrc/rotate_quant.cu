@@ -149,6 +149,31 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
   const int c0 = 4 * cg, c1 = D / 2 + 4 * cg;   // this thread's two column quads
   const float qmax = kInt8 ? 127.0f : 448.0f;
 
+  // Raw 16-byte input vectors of the next block, loaded into registers while
+  // the current block is being computed (thread t: token row idx % T and
+  // 8-channel chunk idx / T for idx = t, t + kNT, ...).
+  constexpr int kLd = (T * kCG + kNT - 1) / kNT;
+  uint4 xr[kLd];
+  auto load_block = [&](int64_t id) {
+    const int blk_ = static_cast<int>(id % nblk);
+    const int bh_ = static_cast<int>(id / nblk);
+    const int b_ = bh_ / H, h_ = bh_ % H;
+    const int n0_ = blk_ * T;
+    const int rows_ = min(T, N - n0_);
+#pragma unroll
+    for (int i = 0; i < kLd; ++i) {
+      const int idx = tid + i * kNT;
+      const int r = idx % T, c = idx / T;
+      xr[i] = make_uint4(0, 0, 0, 0);
+      if (idx < T * kCG && r < rows_)
+        xr[i] = __ldcs(reinterpret_cast<const uint4*>(x + row_offset(layout, H, N, D, b_, h_, n0_ + r) + c * 8));
+    }
+  };
+  // Only where the registers allow it (the larger row tiles of 256-token
+  // blocks already use them all): otherwise the block is loaded on the spot.
+  constexpr bool kPrefetch = kLd <= 4;
+  if (kPrefetch && blockIdx.x < total) load_block(blockIdx.x);
+
   for (int64_t blk_id = blockIdx.x; blk_id < total; blk_id += gridDim.x) {
     const int blk = static_cast<int>(blk_id % nblk);
     const int bh = static_cast<int>(blk_id / nblk);
@@ -156,23 +181,22 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
     const int n0 = blk * T;
     const int rows = min(T, N - n0);
 
+    if (!kPrefetch) load_block(blk_id);
     __syncthreads();  // sR ready (first pass); previous block's sX reads done
-    // Stage x transposed: thread t handles token row (t % T) and a slice of
-    // the 16-byte chunks, so consecutive threads write consecutive words.
-    for (int idx = tid; idx < T * kCG; idx += kNT) {
-      const int r = idx % T, c = idx / T;
-      float f[8];
-      if (r < rows) {
-        const uint4 v = *reinterpret_cast<const uint4*>(x + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8);
-        unpack8(v, is_bf16 != 0, f);
-      } else {
+    // Stage x transposed: consecutive threads write consecutive words.
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+    for (int i = 0; i < kLd; ++i) {
+      const int idx = tid + i * kNT;
+      if (idx < T * kCG) {
+        const int r = idx % T, c = idx / T;
+        float f[8];
+        unpack8(xr[i], is_bf16 != 0, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sX[(c * 8 + e) * kXS + r] = f[e];
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sX[(c * 8 + e) * kXS + r] = f[e];
     }
     __syncthreads();
+    if (kPrefetch && blk_id + gridDim.x < total) load_block(blk_id + gridDim.x);
 
     // acc[i][j]: row rg*kRPT + i, column (j < 4 ? c0 + j : c1 + j - 4); each
     // is the float32 FMA chain over k ascending, two lanes per f32x2 FMA.
