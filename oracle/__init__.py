@@ -62,6 +62,9 @@ def lib():
                                        i, i, P, i, P, P, P]
         L.orc_exact_rows.argtypes = [P, P, P, i, i, i, i, i, i, i, i, d, i, i, P, i, P]
         L.orc_decode_one.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, i, i, i, P, P]
+        L.orc_f32_to_f16.argtypes, L.orc_f32_to_f16.restype = [f], C.c_uint16
+        L.orc_kv_append_int8.argtypes = [P, i, i, i, i, i, i, i, P, P, i, i]
+        L.orc_kv_append_int4.argtypes = [P, i, i, i, i, i, i, i, P, P, i, i]
         _lib = L
     return _lib
 
@@ -260,3 +263,37 @@ def decode(q_bits, k, v, k_scales, v_scales, kv_dtype: int, Hkv: int, heads=None
             D, kv_block, group, float(softmax_scale), splits, b, h, _p(ob), _p(fb)))
     _run_all(jobs)
     return out, of
+
+
+# ---------------------------------------------------------------------------
+# KV-cache quantize-on-append
+# ---------------------------------------------------------------------------
+
+def f32_to_f16_bits(x: float) -> int:
+    return int(lib().orc_f32_to_f16(float(x)))
+
+
+def kv_append(x_bits: np.ndarray, cache: np.ndarray, scales: np.ndarray, L: int, kv_dtype: int,
+              kv_block: int = 256, group: int = 128):
+    """Appends x (bf16 bits [B, H_kv, n, D]) at token L of a quantized cache.
+
+    INT8: cache int8 [B, H_kv, L_max, D], scales float32 [B, H_kv, nblk].
+    INT4_PACKED: cache uint8 [B, H_kv, L_max, D/2], scales fp16 bits (uint16)
+    [B, H_kv, L_max, D/group]. Returns updated copies (cache, scales)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    B, Hkv, n, D = x_bits.shape
+    Lmax = cache.shape[2]
+    cache = np.ascontiguousarray(cache).copy()
+    scales = np.ascontiguousarray(scales).copy()
+    L_ = lib()
+    if kv_dtype == INT8:
+        assert cache.dtype == np.int8 and scales.dtype == np.float32
+        fn = lambda b, h: L_.orc_kv_append_int8(_p(x_bits), B, Hkv, n, D, L, Lmax, kv_block, _p(cache),
+                                                 _p(scales), b, h)
+    else:
+        assert cache.dtype == np.uint8 and scales.dtype == np.uint16
+        fn = lambda b, h: L_.orc_kv_append_int4(_p(x_bits), B, Hkv, n, D, L, Lmax, group, _p(cache),
+                                                 _p(scales), b, h)
+    jobs = [(lambda b=b, h=h: fn(b, h)) for b in range(B) for h in range(Hkv)]
+    _run_all(jobs)
+    return cache, scales

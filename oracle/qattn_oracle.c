@@ -556,4 +556,136 @@ int orc_decode_one(const uint16_t* q, const void* kc, const void* vc, const void
   return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* KV-cache quantize-on-append                                              */
+/* ------------------------------------------------------------------------ */
+
+/* float32 -> fp16 bits, round to nearest even (overflow -> inf; subnormal
+ * results rounded at their own spacing of 2^-24). Worked from the binary16
+ * format: 1 sign, 5 exponent (bias 15), 10 mantissa bits. */
+uint16_t orc_f32_to_f16(float x) {
+  uint16_t sign = signbit(x) ? 0x8000 : 0;
+  double a = fabs((double)x);
+  if (isnan(x)) return sign | 0x7E00;
+  if (a >= 65520.0) return sign | 0x7C00;     /* rounds beyond the largest finite 65504 */
+  int e;
+  frexp(a, &e);                               /* a = f * 2^e, f in [0.5, 1) */
+  int ulp_e = (e - 1) - 10;                   /* spacing 2^(e-1-10) for normals */
+  if (ulp_e < -24) ulp_e = -24;               /* subnormal spacing */
+  double q = a / ldexp(1.0, ulp_e);           /* exact: a power-of-two scaling */
+  double r = nearbyint(q);                    /* default rounding mode: half to even */
+  double v = r * ldexp(1.0, ulp_e);
+  if (v == 0.0) return sign;
+  int ev;
+  frexp(v, &ev);
+  if (ev - 1 < -14) return sign | (uint16_t)(v / ldexp(1.0, -24));      /* subnormal */
+  uint16_t bits = (uint16_t)(((ev - 1 + 15) << 10) | ((uint32_t)(ldexp(v, -(ev - 1)) * 1024.0) - 1024));
+  return sign | bits;
+}
+
+/*
+ * INT8 cache, one float32 scale per block of kv_block tokens per (b, h_kv):
+ * "INT8 量化算子", ops-transformer item 3 (KV Cache 也量化: in the decode phase
+ * the new K/V rows are written into the cache as INT8 codes). How a block's
+ * scale evolves while tokens are appended to it is not on the pages; the
+ * reading taken here keeps it at absmax / 127 of every token written to the
+ * block so far. For each block touched by the n new tokens at [L, L + n):
+ *   a     = max |x| over the block's new tokens and all D channels
+ *   s_new = max(s_old, a / 127)        (float32 division; s_old = 0 when the
+ *                                       block holds no token before L)
+ *   if s_new > s_old and the block holds tokens before L, each of their codes
+ *   is requantized:  c' = clamp(RNE(f32(c * s_old) / s_new), -127, 127)
+ *   new tokens:      c  = clamp(RNE(x / s_new), -127, 127)   (float32 division)
+ *   s_new == 0 gives zero codes.
+ * x: bf16 [B, H_kv, n, D]; cache: int8 [B, H_kv, L_max, D]; scales: float32
+ * [B, H_kv, ceil(L_max / kv_block)]. Updates (b, h) in place.
+ */
+int orc_kv_append_int8(const uint16_t* x, int B, int Hkv, int n, int D, int L, int Lmax, int kv_block,
+                       int8_t* cache, float* scales, int b, int h) {
+  if (n <= 0 || L < 0 || L + n > Lmax || kv_block <= 0 || b >= B || h >= Hkv) return 1;
+  int64_t head = (int64_t)b * Hkv + h;
+  int nblk = (Lmax + kv_block - 1) / kv_block;
+  for (int blk = L / kv_block; blk * kv_block < L + n; ++blk) {
+    int b0 = blk * kv_block;
+    int t0 = L > b0 ? L : b0;                               /* first new token of the block */
+    int t1 = L + n < b0 + kv_block ? L + n : b0 + kv_block; /* one past the last */
+    float a = 0.0f;
+    for (int t = t0; t < t1; ++t)
+      for (int d = 0; d < D; ++d) {
+        float v = fabsf(orc_bf16_to_f32(x[(head * n + (t - L)) * D + d]));
+        if (v > a) a = v;
+      }
+    float s_old = t0 > b0 ? scales[head * nblk + blk] : 0.0f;
+    float s1 = a / 127.0f;
+    float s = s1 > s_old ? s1 : s_old;
+    if (s > s_old && t0 > b0) {
+      for (int t = b0; t < t0; ++t)
+        for (int d = 0; d < D; ++d) {
+          int8_t* c = &cache[(head * Lmax + t) * D + d];
+          float y = (float)(*c) * s_old;                    /* one float32 rounding */
+          float q = rintf(y / s);
+          if (q > 127.0f) q = 127.0f;
+          if (q < -127.0f) q = -127.0f;
+          *c = (int8_t)q;
+        }
+    }
+    for (int t = t0; t < t1; ++t)
+      for (int d = 0; d < D; ++d) {
+        float q = 0.0f;
+        if (s != 0.0f) {
+          q = rintf(orc_bf16_to_f32(x[(head * n + (t - L)) * D + d]) / s);
+          if (q > 127.0f) q = 127.0f;
+          if (q < -127.0f) q = -127.0f;
+        }
+        cache[(head * Lmax + t) * D + d] = (int8_t)q;
+      }
+    scales[head * nblk + blk] = s;
+  }
+  return 0;
+}
+
+/*
+ * Packed INT4 cache ("ops-transformer INT8/INT4 量化推理", 5.1: one fp16 scale
+ * per group of `group` elements; 5.2: two codes per byte, element 2i in the
+ * low nibble): each new token gets its own scales, one per group along D.
+ *   a = max |x| over the group;  s16 = fp16(a / 7) (float32 division, then
+ *   RNE to fp16);  s = (float) s16
+ *   c = clamp(RNE(x / s), -7, 7) (float32 division); s == 0 gives zero codes
+ * x: bf16 [B, H_kv, n, D]; cache: bytes [B, H_kv, L_max, D/2]; scales: fp16
+ * bits [B, H_kv, L_max, D/group]. Updates (b, h) in place.
+ */
+int orc_kv_append_int4(const uint16_t* x, int B, int Hkv, int n, int D, int L, int Lmax, int group,
+                       uint8_t* cache, uint16_t* scales, int b, int h) {
+  if (n <= 0 || L < 0 || L + n > Lmax || group <= 0 || D % group || D % 2 || b >= B || h >= Hkv) return 1;
+  int64_t head = (int64_t)b * Hkv + h;
+  int ng = D / group;
+  int codes[1024];
+  if (D > 1024) return 1;
+  for (int t = L; t < L + n; ++t) {
+    const uint16_t* xr = x + (head * n + (t - L)) * D;
+    for (int g = 0; g < ng; ++g) {
+      float a = 0.0f;
+      for (int d = g * group; d < (g + 1) * group; ++d) {
+        float v = fabsf(orc_bf16_to_f32(xr[d]));
+        if (v > a) a = v;
+      }
+      uint16_t s16 = orc_f32_to_f16(a / 7.0f);
+      float s = orc_f16_to_f32(s16);
+      scales[(head * Lmax + t) * ng + g] = s16;
+      for (int d = g * group; d < (g + 1) * group; ++d) {
+        float q = 0.0f;
+        if (s != 0.0f) {
+          q = rintf(orc_bf16_to_f32(xr[d]) / s);
+          if (q > 7.0f) q = 7.0f;
+          if (q < -7.0f) q = -7.0f;
+        }
+        codes[d] = (int)q;
+      }
+    }
+    uint8_t* row = cache + (head * Lmax + t) * (D / 2);
+    for (int i = 0; i < D / 2; ++i) row[i] = orc_int4_pack(codes[2 * i], codes[2 * i + 1]);
+  }
+  return 0;
+}
+
 int orc_abi_version(void) { return 1; }
