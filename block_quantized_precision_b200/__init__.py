@@ -7,7 +7,7 @@ fails, an exception is raised.
 
 Function names follow the C ABI:
     qattn_rotate_block_quant, qattn_prefill, qattn_decode_workspace_size,
-    qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_device_error,
+    qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_kv_append, qattn_device_error,
     qattn_selftest_wait_timeout,
     qattn_abi_version, qattn_status_string.
 """
@@ -33,7 +33,7 @@ QATTN_BNSD, QATTN_BSND = 0, 1
 QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 3, 4
 
 EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
-            "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc",
+            "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc", "qattn_kv_append",
             "qattn_device_error", "qattn_selftest_wait_timeout")
 
 # Fixed scratch of qattn_decode_kvq_noalloc (bytes).
@@ -67,6 +67,8 @@ def lib() -> C.CDLL:
         L.qattn_decode_kvq.restype = i
         L.qattn_decode_kvq_noalloc.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, P, P]
         L.qattn_decode_kvq_noalloc.restype = i
+        L.qattn_kv_append.argtypes = [P, i, i, i, i, i, i, i, P, P, i, i, P]
+        L.qattn_kv_append.restype = i
         L.qattn_device_error.argtypes, L.qattn_device_error.restype = [P], i
         L.qattn_selftest_wait_timeout.argtypes, L.qattn_selftest_wait_timeout.restype = [i, P], i
         _lib = L
@@ -187,6 +189,20 @@ def qattn_decode_kvq_noalloc(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: 
                                         _ptr(out), _stream(stream))
     _check(st, "qattn_decode_kvq_noalloc")
     return out
+
+
+def qattn_kv_append(x_new, cache, scales, L: int, kv_dtype: int, kv_block: int = 256, group: int = 128,
+                    stream=None):
+    """Quantizes x_new (bf16 [B, H_kv, n, D]) into the cache at tokens
+    [L, L + n), in place. INT8: cache int8 [B, H_kv, L_max, D], scales
+    float32 [B, H_kv, ceil(L_max / kv_block)]. INT4_PACKED: cache uint8
+    [B, H_kv, L_max, D/2], scales float16 [B, H_kv, L_max, D/group]."""
+    B, Hkv, n, D = x_new.shape
+    Lmax = cache.shape[2]
+    st = lib().qattn_kv_append(_ptr(x_new), B, Hkv, n, D, kv_dtype, int(L), Lmax, _ptr(cache), _ptr(scales),
+                               kv_block, group, _stream(stream))
+    _check(st, "qattn_kv_append")
+    return cache, scales
 
 
 def qattn_device_error(stream=None) -> int:

@@ -1,0 +1,174 @@
+// kv_append.cu -- quantize new K or V rows into the decode cache.
+//
+// Method: "INT8 量化算子", ops-transformer item 3 (KV Cache 也量化): in the
+// decode phase new K/V rows are written into the cache as INT8 codes; packed
+// INT4 with one fp16 scale per group of channels: "ops-transformer INT8/INT4
+// 量化推理", 5.1 (group scales) and 5.2 (two codes per byte, element 2i in
+// the low nibble).
+//
+// INT8 cache, one float32 scale per 256-token block of each (b, h_kv): the
+// block scale stays absmax / 127 of every token written to the block so far.
+//   kv_append_int8_kernel: one CTA per (touched block, h_kv, b).
+//     a = max |x| over the block's new tokens; s = max(s_old, a / 127);
+//     if s grew and the block already held tokens, each of their codes c is
+//     replaced by RNE(f32(c * s_old) / s); new codes RNE(x / s); all float32
+//     with IEEE division, clamped to [-127, 127].
+// Packed INT4 cache, one fp16 scale per token per group:
+//   kv_append_int4_kernel: one warp per new token; lane l owns channels
+//     4l..4l+3. s16 = fp16(absmax_group / 7), codes RNE(x / s16) clamped to
+//     [-7, 7], packed two per byte.
+// Both are small, memory-bound kernels (the new rows are read once, the
+// codes written once; a growing INT8 block also rewrites its earlier codes).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "qattn_device.cuh"
+#include "qattn_internal.h"
+
+namespace qattn {
+
+namespace {
+
+constexpr int kAppendThreads = 256;
+
+__device__ __forceinline__ int rne_clamp(float v, int lim) {
+  return max(-lim, min(lim, __float2int_rn(v)));
+}
+
+// x: bf16 [B, H_kv, n, D]; cache int8 [B, H_kv, L_max, D]; scales float32
+// [B, H_kv, nblk]. D is a multiple of 8 (16-byte vectors of x, 8-byte code
+// stores).
+__global__ void __launch_bounds__(kAppendThreads)
+    kv_append_int8_kernel(const uint16_t* __restrict__ x, int Hkv, int n, int D, int L, int Lmax, int kv_block,
+                          int8_t* __restrict__ cache, float* __restrict__ scales) {
+  __shared__ float red[kAppendThreads / 32];
+  const int blk = L / kv_block + static_cast<int>(blockIdx.x);
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t head = static_cast<int64_t>(b) * Hkv + h;
+  const int nblk = (Lmax + kv_block - 1) / kv_block;
+  const int b0 = blk * kv_block;
+  const int t0 = max(L, b0), t1 = min(L + n, b0 + kv_block);
+  if (t0 >= t1) return;                                 // (uniform per CTA)
+  const int vecs = D / 8;
+  const int64_t total = static_cast<int64_t>(t1 - t0) * vecs;
+  const uint16_t* xb = x + (head * n + (t0 - L)) * D;
+
+  float m = 0.0f;
+  for (int64_t i = threadIdx.x; i < total; i += kAppendThreads) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xb + i * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[k] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[k] >> 16))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kAppendThreads / 32; ++i) a = fmaxf(a, red[i]);
+
+  const float s_old = t0 > b0 ? scales[head * nblk + blk] : 0.0f;
+  const float s1 = __fdiv_rn(a, 127.0f);
+  const float s = s1 > s_old ? s1 : s_old;
+
+  // earlier tokens of a block whose scale grew
+  if (s > s_old && t0 > b0) {
+    int8_t* cb = cache + (head * Lmax + b0) * D;
+    const int64_t old_total = static_cast<int64_t>(t0 - b0) * vecs;
+    for (int64_t i = threadIdx.x; i < old_total; i += kAppendThreads) {
+      const uint2 c = *reinterpret_cast<const uint2*>(cb + i * 8);
+      const uint32_t w[2] = {c.x, c.y};
+      uint32_t o[2] = {0, 0};
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float y = __fmul_rn(static_cast<float>(static_cast<int8_t>((w[k] >> (8 * e)) & 0xFFu)), s_old);
+          o[k] |= (static_cast<uint32_t>(rne_clamp(__fdiv_rn(y, s), 127)) & 0xFFu) << (8 * e);
+        }
+      *reinterpret_cast<uint2*>(cb + i * 8) = make_uint2(o[0], o[1]);
+    }
+  }
+  // new tokens
+  int8_t* cn = cache + (head * Lmax + t0) * D;
+  for (int64_t i = threadIdx.x; i < total; i += kAppendThreads) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xb + i * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2] = {0, 0};
+    if (s != 0.0f) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = static_cast<uint32_t>(rne_clamp(__fdiv_rn(bf16_bits_to_f32(w[k] & 0xFFFFu), s), 127)) & 0xFFu;
+        const uint32_t hi = static_cast<uint32_t>(rne_clamp(__fdiv_rn(bf16_bits_to_f32(w[k] >> 16), s), 127)) & 0xFFu;
+        o[k >> 1] |= (lo | (hi << 8)) << (16 * (k & 1));
+      }
+    }
+    *reinterpret_cast<uint2*>(cn + i * 8) = make_uint2(o[0], o[1]);
+  }
+  if (threadIdx.x == 0) scales[head * nblk + blk] = s;
+}
+
+// x: bf16 [B, H_kv, n, D], D = 128 (lane l: channels 4l..4l+3); cache bytes
+// [B, H_kv, L_max, D/2]; scales fp16 [B, H_kv, L_max, D/group], group 128 or
+// 64 (all lanes or one half-warp per group).
+__global__ void __launch_bounds__(kAppendThreads)
+    kv_append_int4_kernel(const uint16_t* __restrict__ x, int B, int Hkv, int n, int L, int Lmax, int group,
+                          uint8_t* __restrict__ cache, uint16_t* __restrict__ scales) {
+  constexpr int D = 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (kAppendThreads / 32) + (threadIdx.x >> 5);
+  const int64_t rows = static_cast<int64_t>(B) * Hkv * n;
+  if (row >= rows) return;                              // (uniform per warp)
+  const int64_t head = row / n;
+  const int t = L + static_cast<int>(row % n);
+  const uint2 raw = *reinterpret_cast<const uint2*>(x + row * D + lane * 4);
+  const float f[4] = {bf16_bits_to_f32(raw.x & 0xFFFFu), bf16_bits_to_f32(raw.x >> 16),
+                      bf16_bits_to_f32(raw.y & 0xFFFFu), bf16_bits_to_f32(raw.y >> 16)};
+  float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+  // reduce over the lanes of this lane's group (16 lanes for group 64)
+  const int width = group / 4;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float other = __shfl_xor_sync(0xffffffffu, m, o);
+    if (o < width) m = fmaxf(m, other);
+  }
+  const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
+  const float s = __half2float(s16);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) packed |= (static_cast<uint32_t>(rne_clamp(__fdiv_rn(f[e], s), 7)) & 0xFu) << (4 * e);
+  }
+  *reinterpret_cast<uint16_t*>(cache + (head * Lmax + t) * (D / 2) + lane * 2) = static_cast<uint16_t>(packed);
+  const int ng = D / group;
+  if ((lane % width) == 0)
+    scales[(head * Lmax + t) * ng + lane / width] = __half_as_ushort(s16);
+}
+
+}  // namespace
+
+bool kv_append_supported(int D, bool int4, int kv_block, int group) {
+  if (int4) return D == 128 && (group == 128 || group == 64);
+  return D % 8 == 0 && D <= 1024 && kv_block == 256;
+}
+
+cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st) {
+  if (!a.int4) {
+    const int first = a.L / a.kv_block, last = (a.L + a.n - 1) / a.kv_block;
+    dim3 grid(static_cast<unsigned>(last - first + 1), a.Hkv, a.B);
+    kv_append_int8_kernel<<<grid, kAppendThreads, 0, st>>>(static_cast<const uint16_t*>(a.x), a.Hkv, a.n, a.D, a.L,
+                                                            a.Lmax, a.kv_block, static_cast<int8_t*>(a.cache),
+                                                            static_cast<float*>(a.scales));
+  } else {
+    const int64_t rows = static_cast<int64_t>(a.B) * a.Hkv * a.n;
+    const int64_t ctas = (rows + kAppendThreads / 32 - 1) / (kAppendThreads / 32);
+    kv_append_int4_kernel<<<static_cast<unsigned>(ctas), kAppendThreads, 0, st>>>(
+        static_cast<const uint16_t*>(a.x), a.B, a.Hkv, a.n, a.L, a.Lmax, a.group, static_cast<uint8_t*>(a.cache),
+        static_cast<uint16_t*>(a.scales));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace qattn

@@ -245,6 +245,34 @@ qattn_status_t qattn_decode_kvq(const void* q, const void* k_cache, const void* 
   return from_cuda(launch_decode(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
 }
 
+qattn_status_t qattn_kv_append(const void* x_new, int B, int H_kv, int n, int D, qattn_dtype_t kv_dtype, int L,
+                               int L_max, void* cache, void* scales, int kv_block, int group,
+                               qattn_stream_t stream) {
+  if (B < 0 || H_kv < 0 || n < 0 || D <= 0 || L < 0 || L_max < 0) return QATTN_ERR_INVALID_ARG;
+  if (kv_dtype != QATTN_INT8 && kv_dtype != QATTN_INT4_PACKED) return QATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(L) + n > L_max) return QATTN_ERR_INVALID_ARG;
+  const bool int4 = kv_dtype == QATTN_INT4_PACKED;
+  if (int4 && (group <= 0 || D % group)) return QATTN_ERR_INVALID_ARG;
+  if (!int4 && kv_block <= 0) return QATTN_ERR_INVALID_ARG;
+  if (!kv_append_supported(D, int4, kv_block, group)) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H_kv * n == 0) return QATTN_OK;
+  if (!x_new || !cache || !scales) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(x_new) || !aligned16(cache)) return QATTN_ERR_ALIGNMENT;
+  if (static_cast<int64_t>(B) * H_kv * n >= (1LL << 31) * 8) return QATTN_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  KvAppendArgs a;
+  a.x = x_new;
+  a.int4 = int4;
+  a.B = B; a.Hkv = H_kv; a.n = n; a.D = D; a.L = L; a.Lmax = L_max;
+  a.kv_block = int4 ? 256 : kv_block;
+  a.group = int4 ? group : D;
+  a.cache = cache;
+  a.scales = scales;
+  return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qattn_status_t qattn_device_error(qattn_stream_t stream) {
   DeviceState* ds = nullptr;
   qattn_status_t s = device_state(&ds);

@@ -67,6 +67,18 @@ int decode_splits(int B, int Hkv, int L, int num_sms);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int D, int num_sms);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, int num_sms, int* err);
 
+struct KvAppendArgs {
+  const void* x;      // bf16 [B, H_kv, n, D]
+  int int4;           // 1: packed INT4 cache, 0: INT8 cache
+  int B, Hkv, n, D, L, Lmax;
+  int kv_block, group;
+  void* cache;
+  void* scales;
+};
+
+bool kv_append_supported(int D, bool int4, int kv_block, int group);
+cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st);
+
 cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err);
 
 }  // namespace qattn

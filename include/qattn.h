@@ -225,6 +225,41 @@ qattn_status_t qattn_decode_kvq_noalloc(const void* q, const void* k_cache, cons
                                         void* out, qattn_stream_t stream);
 
 /*
+ * Quantize-on-append: writes n new K (or V) rows into a quantized decode
+ * cache at token positions [L, L + n) of every (b, h_kv).
+ * "INT8 量化算子", ops-transformer item 3 (KV Cache 也量化: in the decode phase
+ * the new K/V rows are stored as INT8); packed INT4 with fp16 group scales:
+ * "ops-transformer INT8/INT4 量化推理", 5.1 and 5.2.
+ *
+ * x_new:   bfloat16 [B, H_kv, n, D], 16-byte aligned.
+ * kv_dtype QATTN_INT8:
+ *   cache  int8 [B, H_kv, L_max, D] (16-byte aligned); scales float32
+ *          [B, H_kv, ceil(L_max / kv_block)]; kv_block must be 256; D a
+ *          multiple of 8 up to 1024. A block's scale is absmax / 127 of
+ *          every token written to it so far: for each block touched,
+ *          s = max(s_old, a / 127) with a the largest |x| of its new rows
+ *          (s_old ignored for a block that held no token before L); if s
+ *          grew and the block held tokens, their codes become
+ *          RNE(f32(c * s_old) / s); new codes RNE(x / s). float32, IEEE
+ *          division, codes clamped to [-127, 127]; s == 0 gives zero codes.
+ * kv_dtype QATTN_INT4_PACKED:
+ *   cache  bytes [B, H_kv, L_max, D/2] (two codes per byte, element 2i in
+ *          the low nibble); scales fp16 [B, H_kv, L_max, D/group]; D = 128,
+ *          group 128 or 64. Per new token and group: s = fp16(absmax / 7)
+ *          (float32 division, RNE to fp16), codes RNE(x / s) clamped to
+ *          [-7, 7]; s == 0 gives zero codes.
+ * Requires L >= 0, n >= 0 and L + n <= L_max. The caller owns all memory;
+ * cache and scales are updated in place on `stream`; rows outside
+ * [L, L + n) are not written except the earlier rows of a growing INT8
+ * block. Errors: QATTN_ERR_INVALID_ARG (ranges, null pointers),
+ * QATTN_ERR_UNSUPPORTED (D, kv_block, group), QATTN_ERR_ALIGNMENT; nothing
+ * is launched on error. n == 0 returns QATTN_OK without a launch.
+ */
+qattn_status_t qattn_kv_append(const void* x_new, int B, int H_kv, int n, int D,
+                               qattn_dtype_t kv_dtype, int L, int L_max, void* cache,
+                               void* scales, int kv_block, int group, qattn_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the per-device error word that
  * kernels set when a bounded barrier wait runs out. Returns QATTN_OK,
  * QATTN_ERR_TIMEOUT, or QATTN_ERR_CUDA if the synchronisation itself failed.

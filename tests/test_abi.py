@@ -118,3 +118,22 @@ def test_oracle_and_library_share_no_code():
         assert "oracle" not in src.lower().replace("oracle-only", "")
     pkg = open(os.path.join(ROOT, "block_quantized_precision_b200", "__init__.py")).read()
     assert "import oracle" not in pkg and "from oracle" not in pkg
+
+
+def test_kv_append_validation(L):
+    f = L.qattn_kv_append
+    p = 0x1000
+
+    def call(B=2, H=8, n=1, D=128, kv=qa.QATTN_INT8, Lk=10, Lmax=256, kvb=256, grp=128, x=p, c=p, s=p):
+        return f(x, B, H, n, D, kv, Lk, Lmax, c, s, kvb, grp, None)
+    assert call(Lk=256) == qa.QATTN_ERR_INVALID_ARG              # L + n > L_max
+    assert call(Lk=-1) == qa.QATTN_ERR_INVALID_ARG
+    assert call(kv=qa.QATTN_FP8_E4M3) == qa.QATTN_ERR_INVALID_ARG
+    assert call(kvb=128) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(D=12) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(kv=qa.QATTN_INT4_PACKED, grp=96) == qa.QATTN_ERR_INVALID_ARG
+    assert call(kv=qa.QATTN_INT4_PACKED, grp=32) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(kv=qa.QATTN_INT4_PACKED, D=64, grp=64) == qa.QATTN_ERR_UNSUPPORTED
+    assert call(n=0) == qa.QATTN_OK
+    assert call(c=None) == qa.QATTN_ERR_INVALID_ARG
+    assert call(x=p + 2) == qa.QATTN_ERR_ALIGNMENT
