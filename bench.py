@@ -267,7 +267,7 @@ def gpu_arm(args):
 
     extra = {}
     if not args.no_extra:
-        extra = extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak)
+        extra = extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak, flush=l2_flush)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -313,7 +313,7 @@ def load_traffic(kernel):
         return None
 
 
-def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak):
+def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak, flush=None):
     import torch
     res = {}
     n = max(5, args.steps // 2)
@@ -324,7 +324,7 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         ts = []
         for _ in range(reps):
             if flush is not None:
-                flush.zero_()
+                flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
@@ -355,6 +355,30 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                     "roofline": {"bound": "hbm", "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
         del k, v, dd
         torch.cuda.empty_cache()
+
+    # KV-cache quantize-on-append: a 256-token chunk of new K rows written
+    # into the INT8 cache of the INT8 decode problem (block-aligned: one
+    # fresh block per (b, h_kv)) and into the INT4 cache of the INT4 problem
+    for key, p, kvt in (("kv_append_int8", synth.INT8_KV_DECODE, qa.QATTN_INT8),
+                        ("kv_append_int4", synth.INT4_KV_DECODE, qa.QATTN_INT4_PACKED)):
+        n_new, L0 = 256, 1024
+        g = torch.Generator(device=dev).manual_seed(7)
+        xn = torch.randn((p.B, p.Hkv, n_new, p.D), generator=g, device=dev).to(torch.bfloat16)
+        if kvt == qa.QATTN_INT8:
+            cache = torch.zeros((p.B, p.Hkv, L0 + n_new, p.D), dtype=torch.int8, device=dev)
+            scl = torch.zeros((p.B, p.Hkv, (L0 + n_new) // 256), dtype=torch.float32, device=dev)
+            by = xn.numel() * 2 + xn.numel() + p.B * p.Hkv * 4
+        else:
+            cache = torch.zeros((p.B, p.Hkv, L0 + n_new, p.D // 2), dtype=torch.uint8, device=dev)
+            scl = torch.zeros((p.B, p.Hkv, L0 + n_new, p.D // p.group), dtype=torch.float16, device=dev)
+            by = xn.numel() * 2 + xn.numel() // 2 + p.B * p.Hkv * n_new * (p.D // p.group) * 2
+        fn = lambda: qa.qattn_kv_append(xn, cache, scl, L0, kvt, group=p.group)
+        ms = timeit(fn, n, flush)
+        gbs = by / (ms * 1e-3) / 1e9
+        res[key] = {"workload": "%s, append %d tokens at %d" % (p.name, n_new, L0), "ms": round(ms, 4),
+                    "GB/s": round(gbs, 1), "bytes": by,
+                    "roofline": {"bound": "hbm", "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
+        del cache, scl, xn
 
     # FP8 long-sequence prefill path (inputs larger than L2)
     p = synth.FP8_LONG
