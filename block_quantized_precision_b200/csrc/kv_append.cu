@@ -11,10 +11,11 @@
 //   kv_append_int8_kernel: one CTA per (touched block, h_kv, b).
 //     a = max |x| over the block's new tokens; s = max(s_old, a / 127);
 //     if s grew and the block already held tokens, each of their codes c is
-//     replaced by RNE(f32(c * s_old) / s); new codes RNE(x / s); all float32
-//     with IEEE division, clamped to [-127, 127].
+//     replaced by RNE(f32(c * s_old) / s); new codes RNE(x / s); float32,
+//     each code as the IEEE quotient decides it (code_fast), clamped to
+//     [-127, 127].
 // Packed INT4 cache, one fp16 scale per token per group:
-//   kv_append_int4_kernel: one warp per new token; lane l owns channels
+//   kv_append_int4_kernel: one warp per 4 new tokens; lane l owns channels
 //     4l..4l+3. s16 = fp16(absmax_group / 7), codes RNE(x / s16) clamped to
 //     [-7, 7], packed two per byte.
 // Both are small, memory-bound kernels (the new rows are read once, the
@@ -33,6 +34,18 @@ constexpr int kAppendThreads = 256;
 
 __device__ __forceinline__ int rne_clamp(float v, int lim) {
   return max(-lim, min(lim, __float2int_rn(v)));
+}
+
+// RNE(y / s) as the IEEE quotient decides it, mostly without dividing: the
+// product y * RN(1/s) is within 1.5 ulp of the rounded quotient, so its
+// integer rounding agrees unless it lies within 1e-4 of a half-integer (for
+// |y/s| <= 128); those, and scales below the smallest normal float32
+// (`slow`), use the IEEE division.
+__device__ __forceinline__ int code_fast(float y, float s, float rcp, bool slow, int lim) {
+  float v = y * rcp;
+  const float r = (v + 12582912.0f) - 12582912.0f;
+  if (slow || fabsf(v - r) > 0.4999f) v = __fdiv_rn(y, s);
+  return rne_clamp(v, lim);
 }
 
 // x: bf16 [B, H_kv, n, D]; cache int8 [B, H_kv, L_max, D]; scales float32
@@ -72,6 +85,8 @@ __global__ void __launch_bounds__(kAppendThreads)
   const float s_old = t0 > b0 ? scales[head * nblk + blk] : 0.0f;
   const float s1 = __fdiv_rn(a, 127.0f);
   const float s = s1 > s_old ? s1 : s_old;
+  const float rcp = __frcp_rn(s);
+  const bool slow = s < 1.17549435e-38f;
 
   // earlier tokens of a block whose scale grew
   if (s > s_old && t0 > b0) {
@@ -86,7 +101,7 @@ __global__ void __launch_bounds__(kAppendThreads)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float y = __fmul_rn(static_cast<float>(static_cast<int8_t>((w[k] >> (8 * e)) & 0xFFu)), s_old);
-          o[k] |= (static_cast<uint32_t>(rne_clamp(__fdiv_rn(y, s), 127)) & 0xFFu) << (8 * e);
+          o[k] |= (static_cast<uint32_t>(code_fast(y, s, rcp, slow, 127)) & 0xFFu) << (8 * e);
         }
       *reinterpret_cast<uint2*>(cb + i * 8) = make_uint2(o[0], o[1]);
     }
@@ -100,8 +115,8 @@ __global__ void __launch_bounds__(kAppendThreads)
     if (s != 0.0f) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = static_cast<uint32_t>(rne_clamp(__fdiv_rn(bf16_bits_to_f32(w[k] & 0xFFFFu), s), 127)) & 0xFFu;
-        const uint32_t hi = static_cast<uint32_t>(rne_clamp(__fdiv_rn(bf16_bits_to_f32(w[k] >> 16), s), 127)) & 0xFFu;
+        const uint32_t lo = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] & 0xFFFFu), s, rcp, slow, 127)) & 0xFFu;
+        const uint32_t hi = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] >> 16), s, rcp, slow, 127)) & 0xFFu;
         o[k >> 1] |= (lo | (hi << 8)) << (16 * (k & 1));
       }
     }
@@ -113,38 +128,50 @@ __global__ void __launch_bounds__(kAppendThreads)
 // x: bf16 [B, H_kv, n, D], D = 128 (lane l: channels 4l..4l+3); cache bytes
 // [B, H_kv, L_max, D/2]; scales fp16 [B, H_kv, L_max, D/group], group 128 or
 // 64 (all lanes or one half-warp per group).
+constexpr int kInt4RowsPerWarp = 4;
+
 __global__ void __launch_bounds__(kAppendThreads)
     kv_append_int4_kernel(const uint16_t* __restrict__ x, int B, int Hkv, int n, int L, int Lmax, int group,
                           uint8_t* __restrict__ cache, uint16_t* __restrict__ scales) {
   constexpr int D = 128;
   const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (kAppendThreads / 32) + (threadIdx.x >> 5);
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * (kAppendThreads / 32) + (threadIdx.x >> 5)) * kInt4RowsPerWarp;
   const int64_t rows = static_cast<int64_t>(B) * Hkv * n;
-  if (row >= rows) return;                              // (uniform per warp)
-  const int64_t head = row / n;
-  const int t = L + static_cast<int>(row % n);
-  const uint2 raw = *reinterpret_cast<const uint2*>(x + row * D + lane * 4);
-  const float f[4] = {bf16_bits_to_f32(raw.x & 0xFFFFu), bf16_bits_to_f32(raw.x >> 16),
-                      bf16_bits_to_f32(raw.y & 0xFFFFu), bf16_bits_to_f32(raw.y >> 16)};
-  float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
-  // reduce over the lanes of this lane's group (16 lanes for group 64)
-  const int width = group / 4;
+  // the warp's rows are loaded first (in flight together), then coded
+  uint2 raw[kInt4RowsPerWarp];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float other = __shfl_xor_sync(0xffffffffu, m, o);
-    if (o < width) m = fmaxf(m, other);
-  }
-  const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
-  const float s = __half2float(s16);
-  uint32_t packed = 0;
-  if (s != 0.0f) {
+  for (int i = 0; i < kInt4RowsPerWarp; ++i)
+    raw[i] = row0 + i < rows ? *reinterpret_cast<const uint2*>(x + (row0 + i) * D + lane * 4) : make_uint2(0, 0);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) packed |= (static_cast<uint32_t>(rne_clamp(__fdiv_rn(f[e], s), 7)) & 0xFu) << (4 * e);
+  for (int i = 0; i < kInt4RowsPerWarp; ++i) {
+    const int64_t row = row0 + i;
+    if (row >= rows) break;                             // (uniform per warp)
+    const int64_t head = row / n;
+    const int t = L + static_cast<int>(row % n);
+    const float f[4] = {bf16_bits_to_f32(raw[i].x & 0xFFFFu), bf16_bits_to_f32(raw[i].x >> 16),
+                        bf16_bits_to_f32(raw[i].y & 0xFFFFu), bf16_bits_to_f32(raw[i].y >> 16)};
+    float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+    // reduce over the lanes of this lane's group (16 lanes for group 64)
+    const int width = group / 4;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float other = __shfl_xor_sync(0xffffffffu, m, o);
+      if (o < width) m = fmaxf(m, other);
+    }
+    const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
+    const float s = __half2float(s16);
+    uint32_t packed = 0;
+    if (s != 0.0f) {
+      const float rcp = __frcp_rn(s);
+      const bool slow = s < 1.17549435e-38f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) packed |= (static_cast<uint32_t>(code_fast(f[e], s, rcp, slow, 7)) & 0xFu) << (4 * e);
+    }
+    *reinterpret_cast<uint16_t*>(cache + (head * Lmax + t) * (D / 2) + lane * 2) = static_cast<uint16_t>(packed);
+    const int ng = D / group;
+    if ((lane % width) == 0)
+      scales[(head * Lmax + t) * ng + lane / width] = __half_as_ushort(s16);
   }
-  *reinterpret_cast<uint16_t*>(cache + (head * Lmax + t) * (D / 2) + lane * 2) = static_cast<uint16_t>(packed);
-  const int ng = D / group;
-  if ((lane % width) == 0)
-    scales[(head * Lmax + t) * ng + lane / width] = __half_as_ushort(s16);
 }
 
 }  // namespace
@@ -163,7 +190,8 @@ cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st) {
                                                             static_cast<float*>(a.scales));
   } else {
     const int64_t rows = static_cast<int64_t>(a.B) * a.Hkv * a.n;
-    const int64_t ctas = (rows + kAppendThreads / 32 - 1) / (kAppendThreads / 32);
+    const int64_t per_cta = static_cast<int64_t>(kAppendThreads / 32) * kInt4RowsPerWarp;
+    const int64_t ctas = (rows + per_cta - 1) / per_cta;
     kv_append_int4_kernel<<<static_cast<unsigned>(ctas), kAppendThreads, 0, st>>>(
         static_cast<const uint16_t*>(a.x), a.B, a.Hkv, a.n, a.L, a.Lmax, a.group, static_cast<uint8_t*>(a.cache),
         static_cast<uint16_t*>(a.scales));
