@@ -30,7 +30,9 @@
 //               here it may compute PV_j. Finally O / l as bfloat16 (and the
 //               LSE).
 // With two tiles per CTA the tensor core works on one tile's products while
-// the other tile's rows are in their softmax. Every wait is bounded.
+// the other tile's rows are in their softmax. With FP8 codes the two tiles
+// also take turns in step (2), so one tile's row max and fold overlap the
+// other's exponentials. Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -68,6 +70,12 @@ constexpr float kLog2_127 = 6.988684686772166f;
 // and rounding on the FMA pipe, is fastest with none.
 template <bool kInt8>
 constexpr uint32_t kPolyPairs = kInt8 ? 0x00u : 0x02u;
+// Whether the two tiles of a CTA take turns in the probability pass.
+// Measured: FP8, whose pass is MUFU-heavy (exponentials and e4m3
+// conversions), gains from it; INT8 loses, its pass being bound by integer
+// and float32 issue that the other tile's row max and fold compete for.
+template <bool kInt8>
+constexpr bool kPingPong = !kInt8;
 
 struct PrefillParams {
   const float* qs;
@@ -166,21 +174,29 @@ struct TileBars {
   uint64_t p_full;    // P_j in shared memory      (128 row threads)
   uint64_t pv_full;   // PV_j in TMEM              (MMA commit)
   uint64_t pv_free;   // PV_j read by the rows     (128 row threads)
+  uint64_t turn;      // the other tile's probability pass is done (its 128 row threads)
 };
 
-// Calls body(c, v) for the 16-column chunks c = 0..N-1 of this thread's TMEM
-// lane starting at taddr; chunk c + 1 is loaded while chunk c is processed.
-template <int N, typename F>
+// Calls body(c, v) for the W-column chunks c = 0..N-1 of this thread's TMEM
+// lane starting at taddr (W = 16 or 32); chunk c + 1 is loaded while chunk c
+// is processed.
+template <int W>
+__device__ __forceinline__ void tmem_ld_w(uint32_t taddr, uint32_t (&r)[W]) {
+  if constexpr (W == 16) tmem_ld16(taddr, r);
+  else tmem_ld32(taddr, r);
+}
+
+template <int N, int W, typename F>
 __device__ __forceinline__ void tmem_chunks(uint32_t taddr, F&& body) {
-  uint32_t a[16], b[16];
-  tmem_ld16(taddr, a);
+  uint32_t a[W], b[W];
+  tmem_ld_w<W>(taddr, a);
   tmem_wait_ld();
   reg_fence(a);
 #pragma unroll
   for (int c = 0; c < N; ++c) {
-    uint32_t(&cur)[16] = (c & 1) ? b : a;
-    uint32_t(&nxt)[16] = (c & 1) ? a : b;
-    if (c + 1 < N) tmem_ld16(taddr + (c + 1) * 16, nxt);
+    uint32_t(&cur)[W] = (c & 1) ? b : a;
+    uint32_t(&nxt)[W] = (c & 1) ? a : b;
+    if (c + 1 < N) tmem_ld_w<W>(taddr + (c + 1) * W, nxt);
     body(c, cur);
     if (c + 1 < N) {
       tmem_wait_ld();
@@ -189,22 +205,24 @@ __device__ __forceinline__ void tmem_chunks(uint32_t taddr, F&& body) {
   }
 }
 
-// O = alpha * O + g * PV for this thread's row (kScaleO false: alpha == 1
-// for every lane of the warp).
+// Columns per TMEM load in the fold and in the row max (double-buffered).
+constexpr int kFoldW = 16;
+constexpr int kMaxW = 16;
+
 template <int D, bool kInt8, bool kScaleO>
 __device__ __forceinline__ void fold_pv(float (&O)[D], uint32_t tPV, float alpha, float g) {
   const float2 a2 = make_float2(alpha, alpha);
   const float2 g2 = make_float2(g, g);
-  tmem_chunks<D / 16>(tPV, [&](int c, uint32_t(&pv)[16]) {
+  tmem_chunks<D / kFoldW, kFoldW>(tPV, [&](int i, uint32_t(&pv)[kFoldW]) {
 #pragma unroll
-    for (int e = 0; e < 16; e += 2) {
+    for (int e = 0; e < kFoldW; e += 2) {
       const float2 x = kInt8 ? s32x2_to_f32x2(pv[e], pv[e + 1])
                              : make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
-      float2 o = make_float2(O[c * 16 + e], O[c * 16 + e + 1]);
+      float2 o = make_float2(O[i * kFoldW + e], O[i * kFoldW + e + 1]);
       if constexpr (kScaleO) o = fmul2(o, a2);
       o = ffma2(x, g2, o);
-      O[c * 16 + e] = o.x;
-      O[c * 16 + e + 1] = o.y;
+      O[i * kFoldW + e] = o.x;
+      O[i * kFoldW + e + 1] = o.y;
     }
   });
 }
@@ -216,14 +234,14 @@ template <bool kInt8, bool kPartial>
 __device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc) {
   if constexpr (kInt8) {
     int i0 = INT_MIN, i1 = INT_MIN, i2 = INT_MIN, i3 = INT_MIN;
-    tmem_chunks<kTileN / 16>(tS, [&](int c, uint32_t(&v)[16]) {
+    tmem_chunks<kTileN / kMaxW, kMaxW>(tS, [&](int c, uint32_t(&v)[kMaxW]) {
       if constexpr (kPartial) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (c * 16 + e >= kmax) v[e] = 0x80000000u;
+        for (int e = 0; e < kMaxW; ++e)
+          if (c * kMaxW + e >= kmax) v[e] = 0x80000000u;
       }
 #pragma unroll
-      for (int e = 0; e < 16; e += 4) {
+      for (int e = 0; e < kMaxW; e += 4) {
         i0 = max(i0, static_cast<int>(v[e]));
         i1 = max(i1, static_cast<int>(v[e + 1]));
         i2 = max(i2, static_cast<int>(v[e + 2]));
@@ -234,14 +252,14 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc) 
     return im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
   } else {
     float f0 = -CUDART_INF_F, f1 = -CUDART_INF_F, f2 = -CUDART_INF_F, f3 = -CUDART_INF_F;
-    tmem_chunks<kTileN / 16>(tS, [&](int c, uint32_t(&v)[16]) {
+    tmem_chunks<kTileN / kMaxW, kMaxW>(tS, [&](int c, uint32_t(&v)[kMaxW]) {
       if constexpr (kPartial) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (c * 16 + e >= kmax) v[e] = 0xFF800000u;        // -inf
+        for (int e = 0; e < kMaxW; ++e)
+          if (c * kMaxW + e >= kmax) v[e] = 0xFF800000u;        // -inf
       }
 #pragma unroll
-      for (int e = 0; e < 16; e += 8) {
+      for (int e = 0; e < kMaxW; e += 8) {
         f0 = fmax3(f0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
         f1 = fmax3(f1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
         f2 = fmax3(f2, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
@@ -263,7 +281,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
   const float2 t2 = make_float2(toff, toff);
   int ri0 = 0, ri1 = 0;
   float rf0 = 0.0f, rf1 = 0.0f, rf2 = 0.0f, rf3 = 0.0f;
-  tmem_chunks<kTileN / 16>(tS, [&](int c, uint32_t(&v)[16]) {
+  tmem_chunks<kTileN / 16, 16>(tS, [&](int c, uint32_t(&v)[16]) {
     uint32_t packed[4];
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -329,10 +347,18 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
 }
 
 // The rows of one query tile (4 warps, one row per thread).
+//
+// The two tiles of a CTA take turns in pass (2), which keeps the MUFU unit
+// busiest: A(0), B(0), A(1), B(1), ... Each tile's row max and fold run while
+// the other tile computes its probabilities. Tile A waits before pass (2) of
+// tile j for B's pass of tile j - 1, tile B for A's pass of tile j; a tile
+// arrives only where its partner will wait (the causal tile B has one key
+// tile more than A, and a pair may lack B).
 template <int D, bool kInt8>
-__device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars, uint32_t tS, uint32_t tPV,
-                                          uint8_t* sP, const float* sKsc, const float* sVsc, int qt, int ntiles,
-                                          int bh, int b, int h, int quarter, int lane, volatile int* abort_flag) {
+__device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars, TileBars& partner, uint32_t tS,
+                                          uint32_t tPV, uint8_t* sP, const float* sKsc, const float* sVsc, int qt,
+                                          int ntiles, int x, int nt_partner, int bh, int b, int h, int quarter,
+                                          int lane, volatile int* abort_flag) {
   const int r = quarter * 32 + lane;            // row within the tile (= TMEM lane)
   const int q0 = qt * kTileM;
   const int qrow = q0 + r;
@@ -377,12 +403,18 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     }
 
     // ---- (2) probabilities, 8-bit rounding, P to shared memory ----
+    const bool my_turn_waits = kPingPong<kInt8> && (x == 0 ? (j >= 1 && j - 1 < nt_partner) : (j < nt_partner));
+    if (my_turn_waits) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars.turn, (x == 0 ? j - 1 : j) & 1, abort_flag, p.err));
+      if (!ok) break;
+    }
     const float toff = (kInt8 ? kLog2_127 : 0.0f) - m_use;
     const float rowsum = partial ? tile_probs<kInt8, true>(tS, prow, rsw, ksc, toff, kmax)
                                  : tile_probs<kInt8, false>(tS, prow, rsw, ksc, toff, kmax);
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(&bars.p_full);
+    if (kPingPong<kInt8> && (x == 0 ? j < nt_partner : j + 1 < nt_partner)) mbar_arrive(&partner.turn);
     l_run = l_run * alpha + rowsum;
     m_run = m_new;
 
@@ -477,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[x].p_full, 128);
       mbar_init(&bars[x].pv_full, 1);
       mbar_init(&bars[x].pv_free, 128);
+      mbar_init(&bars[x].turn, 128);
     }
     mbar_init(&bar_drain[0], 1);
     mbar_init(&bar_drain[1], 1);
@@ -615,8 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 256);
     if (qt2[x] >= 0)
-      tile_rows<D, kInt8>(p, bars[x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN, sKsc, sVsc,
-                          qt2[x], nt2[x], bh, b, h, warp & 3, lane, &abort_flag);
+      tile_rows<D, kInt8>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
+                          sKsc, sVsc, qt2[x], nt2[x], x, nt2[1 - x], bh, b, h, warp & 3, lane, &abort_flag);
   }
 
   tc_fence_before();

@@ -116,6 +116,68 @@ __device__ __forceinline__ int64_t row_offset(int layout, int H, int N, int D, i
 }
 
 // ---------------------------------------------------------------------------
+// Codes of eight values at a time
+// ---------------------------------------------------------------------------
+
+// Codes of 8 values by the fast path of code_of alone (v0 = y * rcp), packed
+// little-endian into lo (values 0..3) and hi (4..7). Returns false when any
+// value is too close to a rounding boundary (or, for e4m3, in the subnormal
+// range) for v0 to be trusted; the caller then takes the exact path.
+template <bool kInt8>
+__device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
+  bool ok = true;
+  uint32_t t[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float v0 = f[e] * rcp;
+    if constexpr (kInt8) {
+      const float m = v0 + 12582912.0f;                  // RNE integer in the low mantissa bits
+      ok = ok && fabsf(v0 - (m - 12582912.0f)) <= 0.4999f;
+      t[e] = __float_as_uint(m);
+    } else {
+      const uint32_t bb = __float_as_uint(v0) & 0x7FFFFFFFu;
+      ok = ok && bb >= 0x3C800000u && abs(static_cast<int>(bb & 0xFFFFFu) - 0x80000) > 16;
+      t[e] = __float_as_uint(v0);
+    }
+  }
+  if constexpr (kInt8) {
+    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+  } else {
+    lo = cvt_e4m3x2(__uint_as_float(t[0]), __uint_as_float(t[1])) |
+         (cvt_e4m3x2(__uint_as_float(t[2]), __uint_as_float(t[3])) << 16);
+    hi = cvt_e4m3x2(__uint_as_float(t[4]), __uint_as_float(t[5])) |
+         (cvt_e4m3x2(__uint_as_float(t[6]), __uint_as_float(t[7])) << 16);
+  }
+  return ok;
+}
+
+// Eight float32 values, passed by value to the rare exact path.
+struct F8 {
+  float v[8];
+};
+
+// Codes of 8 values with the IEEE quotient for every value, packed like
+// codes8_fast.
+template <bool kInt8>
+__device__ __noinline__ uint2 codes8_exact_f(F8 f, float scale) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f.v[j], scale, 0.0f, true) << (8 * j);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f.v[j + 4], scale, 0.0f, true) << (8 * j);
+  return make_uint2(lo, hi);
+}
+
+// The same for 8 raw 16-bit inputs.
+template <bool kInt8>
+__device__ __forceinline__ uint2 codes8_exact(uint4 raw, bool is_bf16, float scale) {
+  F8 f;
+  unpack8(raw, is_bf16, f.v);
+  return codes8_exact_f<kInt8>(f, scale);
+}
+
+// ---------------------------------------------------------------------------
 // With rotation
 // ---------------------------------------------------------------------------
 
@@ -236,23 +298,38 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
     const bool slow = scale < 1.17549435e-38f;
     if (tid == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
 
+    // Codes by the division-free fast path, one trust check per row of 8
+    // values; the rare rows it cannot decide (and blocks with a subnormal
+    // scale) are coded afterwards with IEEE divisions.
+    uint32_t fix = 0;
 #pragma unroll
     for (int i = 0; i < kRPT; ++i) {
       const int r = rg * kRPT + i;
       if (r >= rows) continue;
       uint32_t w0 = 0, w1 = 0;
       if (scale != 0.0f) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          w0 |= code_of<kInt8>(acc[i][j].x, scale, rcp, slow) << (16 * j);
-          w0 |= code_of<kInt8>(acc[i][j].y, scale, rcp, slow) << (16 * j + 8);
-          w1 |= code_of<kInt8>(acc[i][j + 2].x, scale, rcp, slow) << (16 * j);
-          w1 |= code_of<kInt8>(acc[i][j + 2].y, scale, rcp, slow) << (16 * j + 8);
+        const float f[8] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
+                            acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y};
+        if (!codes8_fast<kInt8>(f, rcp, w0, w1) || slow) {
+          fix |= 1u << i;
+          continue;
         }
       }
       uint8_t* crow = codes + row_offset(layout, H, N, D, b, h, n0 + r);
       *reinterpret_cast<uint32_t*>(crow + c0) = w0;
       *reinterpret_cast<uint32_t*>(crow + c1) = w1;
+    }
+    if (fix != 0) {
+#pragma unroll
+      for (int i = 0; i < kRPT; ++i) {
+        if (!((fix >> i) & 1u)) continue;
+        const F8 f = {{acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
+                       acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y}};
+        const uint2 w = codes8_exact_f<kInt8>(f, scale);
+        uint8_t* crow = codes + row_offset(layout, H, N, D, b, h, n0 + rg * kRPT + i);
+        *reinterpret_cast<uint32_t*>(crow + c0) = w.x;
+        *reinterpret_cast<uint32_t*>(crow + c1) = w.y;
+      }
     }
   }
 }
@@ -260,52 +337,6 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
 // ---------------------------------------------------------------------------
 // Without rotation
 // ---------------------------------------------------------------------------
-
-// Codes of 8 values by the fast path of code_of alone (v0 = y * rcp), packed
-// little-endian into lo (values 0..3) and hi (4..7). Returns false when any
-// value is too close to a rounding boundary (or, for e4m3, in the subnormal
-// range) for v0 to be trusted; the caller then takes the exact path.
-template <bool kInt8>
-__device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
-  bool ok = true;
-  uint32_t t[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float v0 = f[e] * rcp;
-    if constexpr (kInt8) {
-      const float m = v0 + 12582912.0f;                  // RNE integer in the low mantissa bits
-      ok = ok && fabsf(v0 - (m - 12582912.0f)) <= 0.4999f;
-      t[e] = __float_as_uint(m);
-    } else {
-      const uint32_t bb = __float_as_uint(v0) & 0x7FFFFFFFu;
-      ok = ok && bb >= 0x3C800000u && abs(static_cast<int>(bb & 0xFFFFFu) - 0x80000) > 16;
-      t[e] = __float_as_uint(v0);
-    }
-  }
-  if constexpr (kInt8) {
-    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
-  } else {
-    lo = cvt_e4m3x2(__uint_as_float(t[0]), __uint_as_float(t[1])) |
-         (cvt_e4m3x2(__uint_as_float(t[2]), __uint_as_float(t[3])) << 16);
-    hi = cvt_e4m3x2(__uint_as_float(t[4]), __uint_as_float(t[5])) |
-         (cvt_e4m3x2(__uint_as_float(t[6]), __uint_as_float(t[7])) << 16);
-  }
-  return ok;
-}
-
-// Codes of 8 values with the IEEE quotient for every value.
-template <bool kInt8>
-__device__ __noinline__ uint2 codes8_exact(uint4 raw, bool is_bf16, float scale) {
-  float f[8];
-  unpack8(raw, is_bf16, f);
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f[j], scale, 0.0f, true) << (8 * j);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f[j + 4], scale, 0.0f, true) << (8 * j);
-  return make_uint2(lo, hi);
-}
 
 // One CTA per block; each thread owns kVec = T*D/8/256 (rounded up) 16-byte
 // input vectors, kept in registers between the max and the code pass. Codes
