@@ -93,8 +93,10 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
-                   const uint32_t* box, CUtensorMapSwizzle swizzle) {
+namespace {
+
+bool encode_map(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const uint64_t* dims,
+                const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn enc = encode_fn();
   if (!enc || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], s[4];
@@ -105,9 +107,20 @@ bool encode_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t*
     e[i] = 1;
     if (i + 1 < rank) s[i] = strides[i];
   }
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), d, s, b, e,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(map, type, rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool encode_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                   const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides, box, swizzle);
+}
+
+bool encode_map_u16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
+                    const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, rank, base, dims, strides, box, swizzle);
 }
 
 cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err) {
@@ -160,7 +173,7 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype, qa
   a.int8 = code_dtype == QATTN_INT8;
   a.codes = codes;
   a.scales = scales;
-  return from_cuda(launch_rotate_block_quant(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms));
+  return from_cuda(launch_rotate_block_quant(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
 }
 
 qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,

@@ -342,6 +342,14 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
 // Packed float32 pairs (sm_100): one instruction, two IEEE float32 results
 // ---------------------------------------------------------------------------
 
+// Through the compiler's float2 builtins (fma/add/mul.rn.f32x2), which leave
+// the choice of register pairs to the compiler; QATTN_F32X2_ASM selects
+// inline PTX instead.
+#ifndef QATTN_F32X2_ASM
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+#else
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;"
@@ -366,6 +374,7 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
   return *reinterpret_cast<float2*>(&d);
 }
+#endif
 
 // Order-preserving map between float32 and int32 (an involution): a < b as
 // floats iff key(a) < key(b) as signed integers (-0 < +0; NaN not handled).

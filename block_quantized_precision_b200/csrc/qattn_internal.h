@@ -14,6 +14,9 @@ namespace qattn {
 // contiguous dimension; strides (bytes) are given for dims 1..rank-1.
 bool encode_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                    const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle);
+// The same over 16-bit data.
+bool encode_map_u16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                    const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle);
 
 struct RotQuantArgs {
   const void* x;      // F16/BF16 bits
@@ -27,7 +30,8 @@ struct RotQuantArgs {
 };
 
 bool rotate_block_quant_supported(int D, int T);
-cudaError_t launch_rotate_block_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms);
+// err: the library's device error word (timeouts of the pipelined quantizer).
+cudaError_t launch_rotate_block_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err);
 
 struct PrefillArgs {
   const void* q;

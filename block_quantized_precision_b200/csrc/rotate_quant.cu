@@ -17,8 +17,11 @@
 //                 float32) in shared memory and walk over blocks; each CTA
 //                 stages one block of x transposed in shared memory and
 //                 computes y with an 8-column register tile per thread.
-//   quant_kernel  (no R): HBM bound. One CTA per block; 16-byte loads, the
-//                 block max by warp shuffles, 8- or 16-byte code stores.
+//   quant_kernel  (no R): HBM bound. Persistent CTAs stream whole blocks
+//                 through a three-stage shared-memory ring by TMA (two blocks
+//                 ahead); block max on the raw 16-bit lanes, codes by the
+//                 division-free path, the rare undecided values redone one by
+//                 one from the IEEE quotient.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -29,7 +32,6 @@ namespace qattn {
 
 namespace {
 
-constexpr int kThreads = 256;                 // quant_kernel
 template <int D>
 struct RotqThreads {
   static constexpr int value = D == 128 ? 512 : 256;   // 16 warps per SM for D = 128
@@ -119,37 +121,115 @@ __device__ __forceinline__ int64_t row_offset(int layout, int H, int N, int D, i
 // Codes of eight values at a time
 // ---------------------------------------------------------------------------
 
-// Codes of 8 values by the fast path of code_of alone (v0 = y * rcp), packed
-// little-endian into lo (values 0..3) and hi (4..7). Returns false when any
-// value is too close to a rounding boundary (or, for e4m3, in the subnormal
-// range) for v0 to be trusted; the caller then takes the exact path.
-template <bool kInt8>
+// Codes of 8 values by the division-free path, packed little-endian into lo
+// (values 0..3) and hi (4..7). Returns false when any value is too close to a
+// rounding boundary (or, for e4m3, in the subnormal range) for the product
+// with rcp to be trusted; the caller then takes the exact path.
+//   INT8 (pairs of values per f32x2 FMA): m = RN(y * rcp + 1.5 * 2^23) holds
+//   RNE(y * rcp) in its low mantissa bits; d = y * rcp - that integer
+//   (the exact product, one rounding). y * rcp is within 1.5e-5 of the IEEE
+//   quotient (|quotient| <= 127.5), so every code agrees with it when
+//   max |d| <= 0.4999.
+//   e4m3: as code_of.
+// kPacked false: the same INT8 decision one value at a time (d from
+// y * rcp rounded first; the bound holds as well). The rotation kernel uses
+// it: the packed form measured slower there, its FMA loop being compiled
+// differently next to it.
+template <bool kInt8, bool kPacked = true>
 __device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
-  bool ok = true;
   uint32_t t[8];
+  if constexpr (kInt8 && !kPacked) {
+    bool ok = true;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float v0 = f[e] * rcp;
-    if constexpr (kInt8) {
+    for (int e = 0; e < 8; ++e) {
+      const float v0 = f[e] * rcp;
       const float m = v0 + 12582912.0f;                  // RNE integer in the low mantissa bits
       ok = ok && fabsf(v0 - (m - 12582912.0f)) <= 0.4999f;
       t[e] = __float_as_uint(m);
-    } else {
+    }
+    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    return ok;
+  } else if constexpr (kInt8) {
+    const float2 rc = make_float2(rcp, rcp);
+    const float2 mg = make_float2(12582912.0f, 12582912.0f);
+    float dmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 y = make_float2(f[2 * i], f[2 * i + 1]);
+      const float2 m = ffma2(y, rc, mg);
+      const float2 nr = ffma2(m, make_float2(-1.0f, -1.0f), mg);     // -RNE(y * rcp), exact
+      const float2 d = ffma2(y, rc, nr);
+      dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+      t[2 * i] = __float_as_uint(m.x);
+      t[2 * i + 1] = __float_as_uint(m.y);
+    }
+    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    return dmax <= 0.4999f;
+  } else {
+    bool ok = true;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float v0 = f[e] * rcp;
       const uint32_t bb = __float_as_uint(v0) & 0x7FFFFFFFu;
       ok = ok && bb >= 0x3C800000u && abs(static_cast<int>(bb & 0xFFFFFu) - 0x80000) > 16;
       t[e] = __float_as_uint(v0);
     }
+    lo = cvt_e4m3x2(__uint_as_float(t[0]), __uint_as_float(t[1])) |
+         (cvt_e4m3x2(__uint_as_float(t[2]), __uint_as_float(t[3])) << 16);
+    hi = cvt_e4m3x2(__uint_as_float(t[4]), __uint_as_float(t[5])) |
+         (cvt_e4m3x2(__uint_as_float(t[6]), __uint_as_float(t[7])) << 16);
+    return ok;
   }
+}
+
+// The packed INT8 / e4m3 fast path with one flag per value: bit e of the
+// result is set when value e's code must come from the IEEE quotient (same
+// bounds as codes8_fast). The codes of unflagged values are final.
+template <bool kInt8>
+__device__ __forceinline__ uint32_t codes8_flags(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
+  uint32_t t[8];
+  uint32_t flags = 0;
   if constexpr (kInt8) {
+    const float2 rc = make_float2(rcp, rcp);
+    const float2 mg = make_float2(12582912.0f, 12582912.0f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 y = make_float2(f[2 * i], f[2 * i + 1]);
+      const float2 m = ffma2(y, rc, mg);
+      const float2 nr = ffma2(m, make_float2(-1.0f, -1.0f), mg);     // -RNE(y * rcp), exact
+      const float2 d = ffma2(y, rc, nr);
+      flags |= (fabsf(d.x) > 0.4999f ? 1u : 0u) << (2 * i);
+      flags |= (fabsf(d.y) > 0.4999f ? 1u : 0u) << (2 * i + 1);
+      t[2 * i] = __float_as_uint(m.x);
+      t[2 * i + 1] = __float_as_uint(m.y);
+    }
     lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
     hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
   } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float v0 = f[e] * rcp;
+      const uint32_t bb = __float_as_uint(v0) & 0x7FFFFFFFu;
+      flags |= (bb < 0x3C800000u || abs(static_cast<int>(bb & 0xFFFFFu) - 0x80000) <= 16 ? 1u : 0u) << e;
+      t[e] = __float_as_uint(v0);
+    }
     lo = cvt_e4m3x2(__uint_as_float(t[0]), __uint_as_float(t[1])) |
          (cvt_e4m3x2(__uint_as_float(t[2]), __uint_as_float(t[3])) << 16);
     hi = cvt_e4m3x2(__uint_as_float(t[4]), __uint_as_float(t[5])) |
          (cvt_e4m3x2(__uint_as_float(t[6]), __uint_as_float(t[7])) << 16);
   }
-  return ok;
+  return flags;
+}
+
+// Code byte of one value from the IEEE quotient (the rare path; inline, as a
+// call per value measured far slower).
+template <bool kInt8>
+__device__ __forceinline__ uint32_t code_exact(float y, float scale) {
+  const float v = __fdiv_rn(y, scale);
+  if constexpr (kInt8) return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(v)))) & 0xFFu;
+  else return cvt_e4m3x2(v, 0.0f) & 0xFFu;
 }
 
 // Eight float32 values, passed by value to the rare exact path.
@@ -167,14 +247,6 @@ __device__ __noinline__ uint2 codes8_exact_f(F8 f, float scale) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) hi |= code_of<kInt8>(f.v[j + 4], scale, 0.0f, true) << (8 * j);
   return make_uint2(lo, hi);
-}
-
-// The same for 8 raw 16-bit inputs.
-template <bool kInt8>
-__device__ __forceinline__ uint2 codes8_exact(uint4 raw, bool is_bf16, float scale) {
-  F8 f;
-  unpack8(raw, is_bf16, f.v);
-  return codes8_exact_f<kInt8>(f, scale);
 }
 
 // ---------------------------------------------------------------------------
@@ -301,34 +373,39 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
     // Codes by the division-free fast path, one trust check per row of 8
     // values; the rare rows it cannot decide (and blocks with a subnormal
     // scale) are coded afterwards with IEEE divisions.
+    // All codes first, with no branch between the rows, then the stores.
+    uint2 w[kRPT];
     uint32_t fix = 0;
 #pragma unroll
     for (int i = 0; i < kRPT; ++i) {
-      const int r = rg * kRPT + i;
-      if (r >= rows) continue;
-      uint32_t w0 = 0, w1 = 0;
-      if (scale != 0.0f) {
-        const float f[8] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
-                            acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y};
-        if (!codes8_fast<kInt8>(f, rcp, w0, w1) || slow) {
-          fix |= 1u << i;
-          continue;
-        }
-      }
-      uint8_t* crow = codes + row_offset(layout, H, N, D, b, h, n0 + r);
-      *reinterpret_cast<uint32_t*>(crow + c0) = w0;
-      *reinterpret_cast<uint32_t*>(crow + c1) = w1;
+      const float f[8] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
+                          acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y};
+      fix |= codes8_fast<kInt8, false>(f, rcp, w[i].x, w[i].y) ? 0u : 1u << i;
+    }
+    if (scale == 0.0f) {                              // all-zero block: zero codes
+      fix = 0;
+#pragma unroll
+      for (int i = 0; i < kRPT; ++i) w[i] = make_uint2(0, 0);
+    } else if (slow) {
+      fix = (1u << kRPT) - 1;
+    }
+    uint8_t* crow0 = codes + row_offset(layout, H, N, D, b, h, n0 + rg * kRPT);
+    const int64_t rstride = layout == 0 ? D : static_cast<int64_t>(H) * D;   // between token rows
+#pragma unroll
+    for (int i = 0; i < kRPT; ++i) {
+      if (((fix >> i) & 1u) || rg * kRPT + i >= rows) continue;
+      *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c0) = w[i].x;
+      *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c1) = w[i].y;
     }
     if (fix != 0) {
 #pragma unroll
       for (int i = 0; i < kRPT; ++i) {
-        if (!((fix >> i) & 1u)) continue;
+        if (!((fix >> i) & 1u) || rg * kRPT + i >= rows) continue;
         const F8 f = {{acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
                        acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y}};
-        const uint2 w = codes8_exact_f<kInt8>(f, scale);
-        uint8_t* crow = codes + row_offset(layout, H, N, D, b, h, n0 + rg * kRPT + i);
-        *reinterpret_cast<uint32_t*>(crow + c0) = w.x;
-        *reinterpret_cast<uint32_t*>(crow + c1) = w.y;
+        const uint2 we = codes8_exact_f<kInt8>(f, scale);
+        *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c0) = we.x;
+        *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c1) = we.y;
       }
     }
   }
@@ -338,76 +415,159 @@ __global__ void __launch_bounds__(RotqThreads<D>::value, 1)
 // Without rotation
 // ---------------------------------------------------------------------------
 
-// One CTA per block; each thread owns kVec = T*D/8/256 (rounded up) 16-byte
-// input vectors, kept in registers between the max and the code pass. Codes
-// are formed by the division-free fast path; the few vectors holding a value
-// it cannot decide are reloaded and coded with IEEE divisions afterwards,
-// which keeps the unrolled main loop small and branch-free.
-template <int D, int T, bool kInt8>
-__global__ void __launch_bounds__(kThreads)
-    quant_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
-                 uint8_t* __restrict__ codes, float* __restrict__ scales) {
-  constexpr int kCG = D / 8;
-  constexpr int kVec = (T * kCG + kThreads - 1) / kThreads;
-  static_assert(kVec <= 32, "fix-up mask");
-  __shared__ float red[kThreads / 32];
-  const int nblk = (N + T - 1) / T;
-  const int blk = blockIdx.x % nblk;
-  const int bh = blockIdx.x / nblk;
-  const int b = bh / H, h = bh % H;
-  const int n0 = blk * T;
-  const int rows = min(T, N - n0);
-  const bool bf = is_bf16 != 0;
+// Persistent, one CTA per SM: whole blocks stream through a three-stage
+// shared-memory ring by TMA, issued two blocks ahead, so the HBM reads of
+// later blocks overlap the coding of the current one. Each of the 512
+// threads keeps its kVec 16-byte input vectors of the current block in
+// registers between the max and the code pass. The block max is taken on
+// the raw 16-bit lanes (|x| of bf16 and fp16 values orders like the bits
+// with the sign cleared); codes come from the division-free path, the rare
+// vectors it cannot decide from IEEE divisions. Every wait is bounded: a
+// timeout is decided for the whole CTA at the next barrier.
+constexpr int kQThreads = 512;
+constexpr int kQStages = 3;
 
-  uint4 v[kVec];
-  // all loads first (16 bytes each, in flight together), then the max
-#pragma unroll
-  for (int i = 0; i < kVec; ++i) {
-    const int idx = threadIdx.x + i * kThreads;
-    const int r = idx / kCG, c = idx % kCG;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (idx < T * kCG && r < rows)
-      v[i] = __ldcs(reinterpret_cast<const uint4*>(x + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8));
+// Lane-wise max of two pairs of unsigned 16-bit integers.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+template <int D, int T>
+struct QuantSmem {
+  static constexpr int kStage = T * D * 2;             // one block of 16-bit inputs
+  static constexpr int kBytes = kQStages * kStage + 128;
+};
+
+template <int D, int T, bool kInt8, bool kBf16>
+__global__ void __launch_bounds__(kQThreads, 1)
+    quant_kernel(const __grid_constant__ CUtensorMap tmX, int layout, int B, int H, int N,
+                 uint8_t* __restrict__ codes, float* __restrict__ scales, int* err) {
+  constexpr int kCG = D / 8;                           // 16-byte vectors per row
+  constexpr int kVec = T * kCG / kQThreads;            // per thread
+  static_assert(kVec * kQThreads == T * kCG && kVec <= 32, "vectors per thread");
+  using L = QuantSmem<D, T>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ __align__(8) uint64_t full[kQStages];
+  __shared__ float red[2][kQThreads / 32];
+  __shared__ int abort_flag;
+
+  const int tid = threadIdx.x;
+  const int nblk = (N + T - 1) / T;
+  const int64_t total = static_cast<int64_t>(B) * H * nblk;
+  constexpr bool bf = kBf16;
+  if (tid == 0) {
+    for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
+    abort_flag = 0;
+    mbar_fence_init();
   }
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < kVec; ++i) {
-    float f[8];
-    unpack8(v[i], bf, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+  __syncthreads();
+  auto issue = [&](int64_t id, int slot) {
+    const int blk_ = static_cast<int>(id % nblk);
+    const int bh_ = static_cast<int>(id / nblk);
+    mbar_arrive_expect_tx(&full[slot], L::kStage);
+    tma_load_4d(smem + slot * L::kStage, &tmX, &full[slot], 0, blk_ * T, bh_ % H, bh_ / H);
+  };
+  int64_t issued = blockIdx.x;                         // next block to load
+  if (tid == 0) {
+    tma_prefetch_desc(&tmX);
+    for (int st = 0; st < kQStages - 1 && issued < total; ++st, issued += gridDim.x) issue(issued, st);
   }
-  const float amax = block_max<kThreads>(m, red);
-  const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
-  const float rcp = __frcp_rn(scale);
-  const bool slow = scale < 1.17549435e-38f;          // zero or subnormal scale: exact path
-  if (threadIdx.x == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
-  uint32_t fix = 0;
+
+  int it = 0;
+  for (int64_t id = blockIdx.x; id < total; id += gridDim.x, ++it) {
+    const int slot = it % kQStages;
+    const uint32_t parity = (it / kQStages) & 1;
+    // One thread waits (bounded); the barrier releases the others, whose own
+    // completed test of the phase then orders their reads after the copy.
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait(&full[slot], parity, &abort_flag, err);
+    if (!__syncthreads_and(ok)) break;
+    mbar_try_wait(&full[slot], parity);
+    const int blk = static_cast<int>(id % nblk);
+    const int bh = static_cast<int>(id / nblk);
+    const int b = bh / H, h = bh % H;
+    const int n0 = blk * T;
+    const int rows = min(T, N - n0);                   // rows beyond N were zero-filled
+
+    const uint4* src = reinterpret_cast<const uint4*>(smem + slot * L::kStage);
+    uint4 v[kVec];
+    uint32_t mb0 = 0, mb1 = 0;
 #pragma unroll
-  for (int i = 0; i < kVec; ++i) {
-    const int idx = threadIdx.x + i * kThreads;
-    const int r = idx / kCG, c = idx % kCG;
-    if (idx < T * kCG && r < rows) {
+    for (int i = 0; i < kVec; ++i) {
+      v[i] = src[tid + i * kQThreads];
+      mb0 = max_u16x2(mb0, max_u16x2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu));
+      mb1 = max_u16x2(mb1, max_u16x2(v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu));
+    }
+    const uint32_t mb = max_u16x2(mb0, mb1);
+    const uint32_t m16 = max(mb & 0xFFFFu, mb >> 16);
+    float m = bf ? bf16_bits_to_f32(m16) : f16_bits_to_f32(m16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) red[it & 1][tid >> 5] = m;
+    __syncthreads();  // also: every thread is done with the slot of block it - 1
+    float amax = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kQThreads / 32; ++w) amax = fmaxf(amax, red[it & 1][w]);
+    if (tid == 0) {
+      if (issued < total) issue(issued, (it + kQStages - 1) % kQStages);
+      issued += gridDim.x;
+    }
+    const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
+    const float rcp = __frcp_rn(scale);
+    const bool slow = scale < 1.17549435e-38f;        // zero or subnormal scale: exact path
+    if (tid == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
+
+    // Vector i of this thread: row r0 + i * kRowStep, channels 8c .. 8c + 7.
+    constexpr int kRowStep = kQThreads / kCG;
+    const int r0 = tid / kCG, c = tid % kCG;
+    const int64_t rstride = layout == 0 ? D : static_cast<int64_t>(H) * D;   // between token rows
+    uint8_t* out = codes + row_offset(layout, H, N, D, b, h, n0 + r0) + c * 8;
+    // All codes first, with no branch between the vectors (so their
+    // dependent arithmetic interleaves), stored at once; then the few values
+    // too close to a rounding boundary for the fast path are recomputed from
+    // the IEEE quotient one by one (re-read from the stage, which stays until
+    // the next barrier) and their bytes rewritten. A zero scale gives zero
+    // codes; a subnormal one sends every value to the exact path.
+    uint32_t flagged = 0;                                  // vectors with a value to redo
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
       float f[8];
       unpack8(v[i], bf, f);
-      uint32_t lo, hi;
-      const bool ok = codes8_fast<kInt8>(f, rcp, lo, hi);
-      if (ok && !slow) {
-        *reinterpret_cast<uint2*>(codes + row_offset(layout, H, N, D, b, h, n0 + r) + c * 8) = make_uint2(lo, hi);
-      } else {
-        fix |= 1u << i;
+      uint2 w;
+      const bool ok = codes8_fast<kInt8>(f, rcp, w.x, w.y);
+      if (scale == 0.0f) w = make_uint2(0, 0);
+      else flagged |= (ok && !slow ? 0u : 1u) << i;
+      if (r0 + i * kRowStep < rows) *reinterpret_cast<uint2*>(out + i * kRowStep * rstride) = w;
+    }
+#pragma unroll 1
+    while (flagged != 0) {
+      const int i = __ffs(flagged) - 1;
+      flagged &= flagged - 1;
+      if (r0 + i * kRowStep >= rows) continue;
+      float f[8];
+      unpack8(src[tid + i * kQThreads], bf, f);
+      uint2 w;
+      uint32_t fl = slow ? 0xFFu : codes8_flags<kInt8>(f, rcp, w.x, w.y);
+      uint8_t* o = out + i * kRowStep * rstride;
+#pragma unroll 1
+      while (fl != 0) {
+        const int e = __ffs(fl) - 1;
+        fl &= fl - 1;
+        const uint16_t hv = reinterpret_cast<const uint16_t*>(src + tid + i * kQThreads)[e];
+        o[e] = static_cast<uint8_t>(code_exact<kInt8>(bf ? bf16_bits_to_f32(hv) : f16_bits_to_f32(hv), scale));
       }
     }
   }
-  while (fix != 0) {
-    const int i = __ffs(fix) - 1;
-    fix &= fix - 1;
-    const int idx = threadIdx.x + i * kThreads;
-    const int r = idx / kCG, c = idx % kCG;
-    const int64_t off = row_offset(layout, H, N, D, b, h, n0 + r) + c * 8;
-    uint2 w = make_uint2(0, 0);
-    if (scale != 0.0f) w = codes8_exact<kInt8>(*reinterpret_cast<const uint4*>(x + off), bf, scale);
-    *reinterpret_cast<uint2*>(codes + off) = w;
+  if (abort_flag && tid == 0) {
+    // Let the copies already issued land before the CTA exits (bounded).
+    for (int k = 0; k < kQStages; ++k) {
+      const int i2 = it + k;
+      if (blockIdx.x + static_cast<int64_t>(i2) * gridDim.x >= issued) break;
+      mbar_wait(&full[i2 % kQStages], (i2 / kQStages) & 1, nullptr, nullptr, 100000000ull);
+    }
   }
 }
 
@@ -424,32 +584,57 @@ cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
   return cudaGetLastError();
 }
 
+// 4-D map {D, N, H, B} over the 16-bit inputs; box {D, T, 1, 1}: one block of
+// T token rows of one head, unswizzled (rows beyond N read as zeros).
+bool make_map_x(CUtensorMap* m, const void* base, int layout, int B, int H, int N, int D, int T) {
+  const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(N), static_cast<uint64_t>(H),
+                            static_cast<uint64_t>(B)};
+  uint64_t strides[3];
+  if (layout == 0) {
+    strides[0] = static_cast<uint64_t>(D) * 2;
+    strides[1] = static_cast<uint64_t>(N) * D * 2;
+    strides[2] = static_cast<uint64_t>(H) * N * D * 2;
+  } else {
+    strides[0] = static_cast<uint64_t>(H) * D * 2;
+    strides[1] = static_cast<uint64_t>(D) * 2;
+    strides[2] = static_cast<uint64_t>(N) * H * D * 2;
+  }
+  const uint32_t box[4] = {static_cast<uint32_t>(D), static_cast<uint32_t>(T), 1, 1};
+  return encode_map_u16(m, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 template <int D, int T, bool kInt8>
-cudaError_t launch_quant(const RotQuantArgs& a, cudaStream_t st) {
+cudaError_t launch_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err) {
+  CUtensorMap tm;
+  if (!make_map_x(&tm, a.x, a.layout, a.B, a.H, a.N, D, T)) return cudaErrorInvalidValue;
+  using L = QuantSmem<D, T>;
+  auto k = a.is_bf16 ? quant_kernel<D, T, kInt8, true> : quant_kernel<D, T, kInt8, false>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+  if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
-  quant_kernel<D, T, kInt8><<<static_cast<unsigned>(nblocks), kThreads, 0, st>>>(
-      static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B, a.H, a.N,
-      static_cast<uint8_t*>(a.codes), a.scales);
+  const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
+  k<<<grid, kQThreads, L::kBytes, st>>>(tm, a.layout, a.B, a.H, a.N, static_cast<uint8_t*>(a.codes), a.scales,
+                                         err);
   return cudaGetLastError();
 }
 
 template <int D, int T>
-cudaError_t dispatch_t(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
+cudaError_t dispatch_t(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err) {
   if (a.rot) return a.int8 ? launch_rotq<D, T, true>(a, st, num_sms) : launch_rotq<D, T, false>(a, st, num_sms);
-  return a.int8 ? launch_quant<D, T, true>(a, st) : launch_quant<D, T, false>(a, st);
+  return a.int8 ? launch_quant<D, T, true>(a, st, num_sms, err) : launch_quant<D, T, false>(a, st, num_sms, err);
 }
 
 }  // namespace
 
 // Block sizes compiled: 128 and 256 tokens (the method's Q and K/V blocks);
 // D in {64, 128}.
-cudaError_t launch_rotate_block_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
+cudaError_t launch_rotate_block_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err) {
   if (a.D == 128) {
-    if (a.T == 128) return dispatch_t<128, 128>(a, st, num_sms);
-    if (a.T == 256) return dispatch_t<128, 256>(a, st, num_sms);
+    if (a.T == 128) return dispatch_t<128, 128>(a, st, num_sms, err);
+    if (a.T == 256) return dispatch_t<128, 256>(a, st, num_sms, err);
   } else if (a.D == 64) {
-    if (a.T == 128) return dispatch_t<64, 128>(a, st, num_sms);
-    if (a.T == 256) return dispatch_t<64, 256>(a, st, num_sms);
+    if (a.T == 128) return dispatch_t<64, 128>(a, st, num_sms, err);
+    if (a.T == 256) return dispatch_t<64, 256>(a, st, num_sms, err);
   }
   return cudaErrorInvalidValue;
 }
