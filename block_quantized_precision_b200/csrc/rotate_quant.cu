@@ -32,9 +32,11 @@ namespace qattn {
 
 namespace {
 
-template <int D>
+// 8 x 8 thread tiles: 256 threads for 128-token blocks (and D = 64), 512 for
+// 256-token blocks at D = 128.
+template <int D, int T>
 struct RotqThreads {
-  static constexpr int value = D == 128 ? 512 : 256;   // 16 warps per SM for D = 128
+  static constexpr int value = D == 128 && T == 256 ? 512 : 256;
 };
 
 __device__ __forceinline__ void unpack8(uint4 v, bool is_bf16, float (&f)[8]) {
@@ -258,11 +260,11 @@ __device__ __noinline__ uint2 codes8_exact_f(F8 f, float scale) {
 // consecutive across the warp, so the R reads are free of bank conflicts);
 // row group rg = tid / (D/8) owns rows rg*kRPT .. rg*kRPT + kRPT - 1.
 template <int D, int T, bool kInt8>
-__global__ void __launch_bounds__(RotqThreads<D>::value, 1)
+__global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
     rotq_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
                 const float* __restrict__ rot, uint8_t* __restrict__ codes,
                 float* __restrict__ scales) {
-  constexpr int kNT = RotqThreads<D>::value;
+  constexpr int kNT = RotqThreads<D, T>::value;
   constexpr int kCG = D / 8;               // column groups
   constexpr int kRG = kNT / kCG;           // row groups
   constexpr int kRPT = T / kRG;            // rows per thread
@@ -579,7 +581,7 @@ cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
   const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
-  k<<<grid, RotqThreads<D>::value, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B,
+  k<<<grid, RotqThreads<D, T>::value, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B,
                                                 a.H, a.N, a.rot, static_cast<uint8_t*>(a.codes), a.scales);
   return cudaGetLastError();
 }
