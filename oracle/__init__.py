@@ -58,7 +58,7 @@ def lib():
         L.orc_rotate_row.argtypes = [P, P, i, P]
         L.orc_quant_block.argtypes = [P, i, i, i, i, i, i, P, i, i, i, i, i, P, P]
         L.orc_quant_head.argtypes = [P, i, i, i, i, i, i, P, i, i, i, i, P, P]
-        L.orc_prefill_rows.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, f, i,
+        L.orc_prefill_rows.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, i, f, i,
                                        i, i, P, i, P, P, P]
         L.orc_exact_rows.argtypes = [P, P, P, i, i, i, i, i, i, i, i, d, i, i, P, i, P]
         L.orc_decode_one.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, i, i, i, P, P]
@@ -136,7 +136,8 @@ def rotate_row(x: np.ndarray, rot) -> np.ndarray:
 
 def rotate_block_quant(x_bits: np.ndarray, x_dtype: int, layout: int, rot, block: int,
                        code_dtype: int, heads=None, blocks=None):
-    """Codes (uint8, same shape as x) and scales float32 [B, H, nblk].
+    """Codes (uint8, same shape as x; INT4_PACKED: [..., D/2], two codes per
+    byte, element 2i in the low nibble) and scales float32 [B, H, nblk].
 
     heads: optional list of (b, h) to compute (others are left zero).
     blocks: optional list of (b, h, blk) to compute (overrides heads)."""
@@ -160,6 +161,9 @@ def rotate_block_quant(x_bits: np.ndarray, x_dtype: int, layout: int, rot, block
                                                    block, code_dtype, b, h, _p(codes), _p(scales)))
                 for (b, h) in hs]
     _run_all(jobs)
+    if code_dtype == INT4_PACKED:
+        c = codes & 0xF                                    # two's complement nibbles
+        codes = (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
     return codes, scales
 
 
@@ -170,11 +174,13 @@ def rotate_block_quant(x_bits: np.ndarray, x_dtype: int, layout: int, rot, block
 def prefill_rows(qc, qs, kc, ks, vc, vs, code_dtype: int, layout: int, causal: bool,
                  rows_by_head: dict, q_block=128, kv_block=256, kv_tile=128,
                  softmax_scale=0.0, p_quant=True, Nkv=None, want_f64=False, want_lse=False,
-                 row_chunk=None):
+                 row_chunk=None, v_dtype=None):
     """Output rows of quantized attention.
 
     qc/kc/vc: codes (uint8 for INT8/FP8 -- INT8 codes as their byte pattern --
-    or float32 for F32), shaped like the layout. rows_by_head: {(b, h): [rows]}.
+    or float32 for F32), shaped like the layout; Q and K have code_dtype, V
+    has v_dtype (default code_dtype; INT4_PACKED: [..., D/2] packed bytes).
+    rows_by_head: {(b, h): [rows]}.
     row_chunk: optional number of rows per parallel job (default: one job per
     head). Returns {(b, h): (bf16 bits [n, D], f64 [n, D] or None, lse [n] or
     None)}.
@@ -208,7 +214,8 @@ def prefill_rows(qc, qs, kc, ks, vc, vs, code_dtype: int, layout: int, causal: b
             lss = ls[s0:s1] if ls is not None else None
             jobs.append(lambda b=b, h=h, rr=rr, obs=obs, ofs=ofs, lss=lss: L.orc_prefill_rows(
                 _p(arrs[0]), _p(arrs[1]), _p(arrs[2]), _p(arrs[3]), _p(arrs[4]), _p(arrs[5]),
-                code_dtype, layout, B, H, Nq, Nk, D, q_block, kv_block, kv_tile, int(causal),
+                code_dtype, code_dtype if v_dtype is None else v_dtype, layout, B, H, Nq, Nk, D, q_block,
+                kv_block, kv_tile, int(causal),
                 float(softmax_scale), int(p_quant), b, h, _p(rr), len(rr), _p(obs), _p(ofs), _p(lss)))
     _run_all(jobs)
     return res

@@ -27,6 +27,12 @@
  *    "ops-transformer INT8/INT4 量化推理" page, sections 5.1 and 5.2.
  *  - float8_e4m3fn: OCP 8-bit floating point specification (E4M3: bias 7,
  *    no infinities, one NaN pattern per sign, largest finite 448).
+ *  - INT4 block codes for attention inputs (round(x / scale) clamped to the
+ *    INT4 range, scale per group) and INT4 widened to INT8 for the matmul:
+ *    "FlashAttention 的 INT8/INT4 量化" page, 第二层 (INT4); Q/K in INT8 with
+ *    V in INT4: same page, 第三层 (混合精度). Here the INT4 scale is dynamic
+ *    per block of tokens like the INT8/e4m3 ones (absmax / 7, codes in
+ *    [-7, 7], packed as above).
  *
  * Precision: every step whose result decides an integer code (rotation,
  * block absmax, scale, code rounding, the probabilities that are rounded to
@@ -228,7 +234,7 @@ int orc_quant_block(const uint16_t* x, int x_dtype, int layout, int B, int H, in
       if (a > amax) amax = a;
     }
   }
-  float qmax = code_dtype == ORC_INT8 ? 127.0f : 448.0f;
+  float qmax = code_dtype == ORC_INT8 ? 127.0f : code_dtype == ORC_INT4_PACKED ? 7.0f : 448.0f;
   float s = amax / qmax;
   int nblk = (N + T - 1) / T;
   scales[((int64_t)b * H + h) * nblk + blk] = s;
@@ -242,6 +248,11 @@ int orc_quant_block(const uint16_t* x, int x_dtype, int layout, int B, int H, in
           float q = rintf(v);                  /* default rounding: half to even */
           if (q > 127.0f) q = 127.0f;
           if (q < -127.0f) q = -127.0f;
+          c = (uint8_t)(int8_t)q;
+        } else if (code_dtype == ORC_INT4_PACKED) {
+          float q = rintf(v);                  /* one signed code per byte here; */
+          if (q > 7.0f) q = 7.0f;              /* the caller packs two per byte  */
+          if (q < -7.0f) q = -7.0f;
           c = (uint8_t)(int8_t)q;
         } else {
           c = orc_e4m3_from_f32(v);
@@ -273,6 +284,10 @@ int orc_quant_head(const uint16_t* x, int x_dtype, int layout, int B, int H, int
 
 static double code_value(const void* c, int dtype, int64_t i) {
   if (dtype == ORC_INT8) return (double)((const int8_t*)c)[i];
+  if (dtype == ORC_INT4_PACKED) {              /* element i of a packed array */
+    uint8_t b = ((const uint8_t*)c)[i >> 1];
+    return (double)((i & 1) ? orc_int4_hi(b) : orc_int4_lo(b));
+  }
   if (dtype == ORC_FP8_E4M3) return (double)orc_e4m3_to_f32(((const uint8_t*)c)[i]);
   return (double)((const float*)c)[i];       /* ORC_F32 */
 }
@@ -281,7 +296,8 @@ static double code_value(const void* c, int dtype, int64_t i) {
  * Output rows of quantized attention for one (b, h).
  *
  * Inputs are the codes and per-block scales of Q (blocks of q_block tokens),
- * K and V (blocks of kv_block tokens), laid out as the quantizer writes them.
+ * K and V (blocks of kv_block tokens), laid out as the quantizer writes them;
+ * Q and K have code_dtype, V has v_dtype (INT4_PACKED: two codes per byte).
  * For each requested query row i:
  *
  *   for each key tile t of kv_tile keys, ascending (tiles whose keys are all
@@ -293,9 +309,9 @@ static double code_value(const void* c, int dtype, int64_t i) {
  *     m_new  = max(m, max_j s_j)                           (float32)
  *     alpha  = expf(m - m_new)                             (float32; 0 at start)
  *     p_j    = expf(s_j - m_new)                           (float32)
- *     P_j    = Q(p_j): e4m3(p_j) for FP8 codes, RNE(p_j * 127) / 127 for INT8
- *              codes (computed as rintf(p_j * 127.0f)), p_j itself when
- *              p_quant == 0
+ *     P_j    = Q(p_j): e4m3(p_j) when V has e4m3 codes, RNE(p_j * 127) / 127
+ *              when V has INT8 or INT4 codes (computed as rintf(p_j *
+ *              127.0f)), p_j itself when p_quant == 0
  *     l      = l * alpha + sum_j P_j                       (float64)
  *     O      = O * alpha + sum_j P_j * vcode[j] * sV[j / kv_block] (float64)
  *   out = O / l, rounded to bfloat16 (RNE); lse = m + ln(l).
@@ -304,7 +320,7 @@ static double code_value(const void* c, int dtype, int64_t i) {
  * lse: optional [nrows, D] / [nrows].
  */
 int orc_prefill_rows(const void* qc, const float* qs, const void* kc, const float* ks,
-                     const void* vc, const float* vs, int code_dtype, int layout,
+                     const void* vc, const float* vs, int code_dtype, int v_dtype, int layout,
                      int B, int H, int Nq, int Nkv, int D, int q_block, int kv_block,
                      int kv_tile, int causal, float softmax_scale, int p_quant,
                      int b, int h, const int* rows, int nrows,
@@ -348,7 +364,7 @@ int orc_prefill_rows(const void* qc, const float* qs, const void* kc, const floa
         double pq;
         if (!p_quant)
           pq = (double)p;
-        else if (code_dtype == ORC_INT8)
+        else if (v_dtype == ORC_INT8 || v_dtype == ORC_INT4_PACKED)
           pq = (double)rintf(p * 127.0f) / 127.0;
         else
           pq = (double)orc_e4m3_to_f32(orc_e4m3_from_f32(p));
@@ -356,7 +372,7 @@ int orc_prefill_rows(const void* qc, const float* qs, const void* kc, const floa
         if (pq != 0.0) {
           int64_t voff = row_off(layout, B, H, Nkv, D, b, h, j);
           double sv = (double)vs[((int64_t)b * H + h) * nkb + j / kv_block];
-          for (int d = 0; d < D; ++d) O[d] += pq * code_value(vc, code_dtype, voff + d) * sv;
+          for (int d = 0; d < D; ++d) O[d] += pq * code_value(vc, v_dtype, voff + d) * sv;
         }
       }
       l = l * (double)alpha + tile_l;
