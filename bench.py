@@ -404,6 +404,31 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                                "TFLOPS_path": round(ops / (ms_full * 1e-3) / 1e12, 1),
                                "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TFLOP/s",
                                             "frac": round(ops / (ms_pf * 1e-3) / 1e12 / int8_peak, 4)}}
+    del x, codes, out, d
+
+    # Mixed precision on the INT8 causal problem: Q/K INT8 (rotated), V in
+    # packed INT4 or e4m3 (L2 flushed before every timed call)
+    p = synth.INT8_CAUSAL
+    d = synth.make_prefill(p)
+    x = {nm: torch.from_numpy(d[nm].view(np.int16)).to(dev).view(torch.bfloat16) for nm in ("q", "k", "v")}
+    rot = torch.from_numpy(d["rot"]).to(dev)
+    qk = {nm: qa.qattn_rotate_block_quant(x[nm], p.layout, rot, 128 if nm == "q" else 256, qa.QATTN_INT8)
+          for nm in ("q", "k")}
+    out = torch.empty(p.shape(), dtype=torch.bfloat16, device=dev)
+    ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
+    for key, vt in (("prefill_mixed_int4v", qa.QATTN_INT4_PACKED), ("prefill_mixed_fp8v", qa.QATTN_FP8_E4M3)):
+        vcodes = qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, vt)
+        qv = lambda: qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, vt, vcodes[0], vcodes[1])
+        ms_qv = timeit(qv, n, flush)
+        pf = lambda: qa.qattn_prefill_mixed(qk["q"][0], qk["q"][1], qk["k"][0], qk["k"][1], vcodes[0], vcodes[1],
+                                            qa.QATTN_INT8, vt, p.layout, p.causal, out=out)
+        ms_pf = timeit(pf, n, flush)
+        v_bytes = x["v"].numel() * 2 + vcodes[0].numel()
+        tops = ops / (ms_pf * 1e-3) / 1e12
+        res[key] = {"workload": "%s, V %s" % (p.name, "int4 packed" if vt == qa.QATTN_INT4_PACKED else "e4m3"),
+                    "ms_prefill": round(ms_pf, 4), "TOPS_prefill": round(tops, 1),
+                    "ms_quant_v": round(ms_qv, 4), "GB/s_quant_v": round(v_bytes / (ms_qv * 1e-3) / 1e9, 1),
+                    "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TOPS", "frac": round(tops / int8_peak, 4)}}
     return res
 
 
@@ -500,15 +525,17 @@ def profile_case(args):
         for _ in range(args.warmup + args.steps):
             qa.qattn_decode_kvq(q, k, v, ks, vs, kvt, kv_block=p.kv_block, group=p.group)
     else:
-        p = synth.INT8_CAUSAL if c == "prefill_int8" else synth.FP8_LONG
+        p = synth.FP8_LONG if c == "prefill_fp8" else synth.INT8_CAUSAL
+        # prefill_int4v: the INT8 causal problem with V in packed INT4
+        vt = qa.QATTN_INT4_PACKED if c == "prefill_int4v" else p.code_dtype
         d = synth.make_prefill(p)
         x = {n: torch.from_numpy(d[n].view(np.int16)).to(dev).view(torch.bfloat16) for n in ("q", "k", "v")}
         rot = torch.from_numpy(d["rot"]).to(dev)
         for _ in range(args.warmup + args.steps):
             qc = qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, p.code_dtype)
             kc = qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, p.code_dtype)
-            vc = qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, p.code_dtype)
-            qa.qattn_prefill(*qc, *kc, *vc, p.code_dtype, p.layout, p.causal)
+            vc = qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, vt)
+            qa.qattn_prefill_mixed(*qc, *kc, *vc, p.code_dtype, vt, p.layout, p.causal)
     torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
     print("case %s: ok" % c)
@@ -524,7 +551,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-heads", type=int, default=4, help="heads per reference-arm step")
-    ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "decode_int8kv", "decode_int4kv"],
+    ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "prefill_int4v", "decode_int8kv",
+                                                           "decode_int4kv"],
                     help="run one workload only (for profiler captures); prints no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

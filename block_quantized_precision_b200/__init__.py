@@ -6,7 +6,7 @@ memory and streams. There is no fallback: if libqattn.so is missing or a call
 fails, an exception is raised.
 
 Function names follow the C ABI:
-    qattn_rotate_block_quant, qattn_prefill, qattn_decode_workspace_size,
+    qattn_rotate_block_quant, qattn_prefill, qattn_prefill_mixed, qattn_decode_workspace_size,
     qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_kv_append, qattn_device_error,
     qattn_selftest_wait_timeout,
     qattn_abi_version, qattn_status_string.
@@ -33,6 +33,7 @@ QATTN_BNSD, QATTN_BSND = 0, 1
 QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 3, 4
 
 EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
+            "qattn_prefill_mixed",
             "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc", "qattn_kv_append",
             "qattn_device_error", "qattn_selftest_wait_timeout")
 
@@ -62,6 +63,8 @@ def lib() -> C.CDLL:
         L.qattn_rotate_block_quant.restype = i
         L.qattn_prefill.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
         L.qattn_prefill.restype = i
+        L.qattn_prefill_mixed.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
+        L.qattn_prefill_mixed.restype = i
         L.qattn_decode_workspace_size.argtypes, L.qattn_decode_workspace_size.restype = [i, i, i, i, i], z
         L.qattn_decode_kvq.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, P, P, z, P]
         L.qattn_decode_kvq.restype = i
@@ -115,13 +118,15 @@ def qattn_rotate_block_quant(x, layout: int, rot, block_tokens: int, code_dtype:
     """Rotation (optional) + dynamic block quantization of one tensor.
 
     x: CUDA bfloat16/float16 tensor in `layout`; rot: CUDA float32 [D, D] or
-    None. Returns (codes uint8 like x, scales float32 [B, H, nblk])."""
+    None. Returns (codes uint8 like x -- [..., D/2] for QATTN_INT4_PACKED --,
+    scales float32 [B, H, nblk])."""
     import torch
     B, H, N, D = _dims(x, layout)
     x_dtype = {torch.bfloat16: QATTN_BF16, torch.float16: QATTN_F16}[x.dtype]
     nblk = -(-N // block_tokens)
     if codes is None:
-        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+        shape = tuple(x.shape[:-1]) + ((D // 2,) if code_dtype == QATTN_INT4_PACKED else (D,))
+        codes = torch.empty(shape, dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((B, H, nblk), dtype=torch.float32, device=x.device)
     st = lib().qattn_rotate_block_quant(_ptr(x), x_dtype, layout, B, H, N, D, _ptr(rot), block_tokens,
@@ -143,6 +148,24 @@ def qattn_prefill(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, code_
                              _ptr(v_scales), code_dtype, layout, B, H, Nq, Nkv, D, q_block, kv_block,
                              int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "qattn_prefill")
+    return out
+
+
+def qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, qk_dtype: int, v_dtype: int,
+                        layout: int, causal: bool, softmax_scale: float = 0.0, out=None, lse=None,
+                        q_block: int = 128, kv_block: int = 256, stream=None):
+    """Quantized attention with V in its own code type (INT4 V: [..., D/2]
+    packed bytes); returns the bfloat16 output (layout of Q)."""
+    import torch
+    B, H, Nq, D = _dims(q_codes, layout)
+    Nkv = _dims(k_codes, layout)[2]
+    if out is None:
+        out = torch.empty(q_codes.shape, dtype=torch.bfloat16, device=q_codes.device)
+    st = lib().qattn_prefill_mixed(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                   _ptr(v_scales), qk_dtype, v_dtype, layout, B, H, Nq, Nkv, D, q_block,
+                                   kv_block, int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse),
+                                   _stream(stream))
+    _check(st, "qattn_prefill_mixed")
     return out
 
 

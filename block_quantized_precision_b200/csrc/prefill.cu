@@ -68,14 +68,14 @@ constexpr float kLog2_127 = 6.988684686772166f;
 // Measured: one pair in eight shortens the FP8 probability pass (MUFU is
 // its busiest unit); the INT8 pass, with its integer-to-float conversions
 // and rounding on the FMA pipe, is fastest with none.
-template <bool kInt8>
-constexpr uint32_t kPolyPairs = kInt8 ? 0x00u : 0x02u;
+template <bool kPInt8>
+constexpr uint32_t kPolyPairs = kPInt8 ? 0x00u : 0x02u;
 // Whether the two tiles of a CTA take turns in the probability pass.
 // Measured: FP8, whose pass is MUFU-heavy (exponentials and e4m3
 // conversions), gains from it; INT8 loses, its pass being bound by integer
 // and float32 issue that the other tile's row max and fold compete for.
-template <bool kInt8>
-constexpr bool kPingPong = !kInt8;
+template <bool kPInt8>
+constexpr bool kPingPong = !kPInt8;
 
 struct PrefillParams {
   const float* qs;
@@ -91,14 +91,17 @@ struct PrefillParams {
   int* err;
 };
 
-template <int D>
+// kVCode: V code type (0 e4m3, 1 INT8, 2 packed INT4 widened on chip).
+template <int D, int kVCode>
 struct Smem {
   static constexpr int kTileBytes = kTileM * D;       // one 128-row code tile
+  static constexpr int kVTileBytes = kVCode == 2 ? kTileN * D / 2 : kTileBytes;   // one V tile as loaded
   static constexpr int kQ = 0;                        // two Q tiles
   static constexpr int kP = kQ + 2 * kTileBytes;      // two P tiles: 128 rows x 128 keys
   static constexpr int kK = kP + 2 * kTileM * kTileN;
   static constexpr int kV = kK + kStagesKV * kTileBytes;
-  static constexpr int kEnd = kV + kStagesKV * kTileBytes;
+  static constexpr int kW = kV + kStagesKV * kVTileBytes;  // INT4: two widened (INT8) V tiles
+  static constexpr int kEnd = kW + (kVCode == 2 ? 2 * kTileBytes : 0);
   static constexpr int kBytes = kEnd + 1024;          // slack for 1024-byte alignment
 };
 
@@ -209,14 +212,14 @@ __device__ __forceinline__ void tmem_chunks(uint32_t taddr, F&& body) {
 constexpr int kFoldW = 16;
 constexpr int kMaxW = 16;
 
-template <int D, bool kInt8, bool kScaleO>
+template <int D, bool kPInt8, bool kScaleO>
 __device__ __forceinline__ void fold_pv(float (&O)[D], uint32_t tPV, float alpha, float g) {
   const float2 a2 = make_float2(alpha, alpha);
   const float2 g2 = make_float2(g, g);
   tmem_chunks<D / kFoldW, kFoldW>(tPV, [&](int i, uint32_t(&pv)[kFoldW]) {
 #pragma unroll
     for (int e = 0; e < kFoldW; e += 2) {
-      const float2 x = kInt8 ? s32x2_to_f32x2(pv[e], pv[e + 1])
+      const float2 x = kPInt8 ? s32x2_to_f32x2(pv[e], pv[e + 1])
                              : make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1]));
       float2 o = make_float2(O[i * kFoldW + e], O[i * kFoldW + e + 1]);
       if constexpr (kScaleO) o = fmul2(o, a2);
@@ -275,7 +278,7 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc) 
 // row of P in shared memory (128-byte swizzled K-major rows); returns the row
 // sum of the rounded values. t = S * ksc + toff; INT8: code = RNE(2^t) with
 // toff = log2(127) - m (so 2^t = 127 p); FP8: e4m3(2^t) with toff = -m.
-template <bool kInt8, bool kPartial>
+template <bool kSInt8, bool kPInt8, bool kPartial>
 __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw, float ksc, float toff, int kmax) {
   const float2 k2 = make_float2(ksc, ksc);
   const float2 t2 = make_float2(toff, toff);
@@ -286,7 +289,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       float2 t01, t23;
-      if constexpr (kInt8) {
+      if constexpr (kSInt8) {
         t01 = ffma2(s32x2_to_f32x2(v[4 * w], v[4 * w + 1]), k2, t2);
         t23 = ffma2(s32x2_to_f32x2(v[4 * w + 2], v[4 * w + 3]), k2, t2);
       } else {
@@ -295,7 +298,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
       }
       // the pairs marked in kPolyPairs go to the FMA pipe, the rest to MUFU
       float pr[4];
-      if ((kPolyPairs<kInt8> >> (2 * w)) & 1) {
+      if ((kPolyPairs<kPInt8> >> (2 * w)) & 1) {
         const float2 e = exp2_poly2(t01);
         pr[0] = e.x;
         pr[1] = e.y;
@@ -303,7 +306,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
         pr[0] = ex2(t01.x);
         pr[1] = ex2(t01.y);
       }
-      if ((kPolyPairs<kInt8> >> (2 * w + 1)) & 1) {
+      if ((kPolyPairs<kPInt8> >> (2 * w + 1)) & 1) {
         const float2 e = exp2_poly2(t23);
         pr[2] = e.x;
         pr[3] = e.y;
@@ -315,7 +318,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
 #pragma unroll
         for (int e = 0; e < 4; ++e) pr[e] = c * 16 + w * 4 + e < kmax ? pr[e] : 0.0f;
       }
-      if constexpr (kInt8) {
+      if constexpr (kPInt8) {
         // adding 1.5 * 2^23 rounds to an integer (half to even) and leaves it
         // in the low mantissa byte
         const float2 q01 = fadd2(make_float2(pr[0], pr[1]), make_float2(12582912.0f, 12582912.0f));
@@ -343,7 +346,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
     // keys 16c .. 16c+15 = 16-byte chunk c of this row
     *reinterpret_cast<uint4*>(prow + ((c ^ rsw) << 4)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   });
-  return kInt8 ? static_cast<float>(ri0 + ri1) * (1.0f / 127.0f) : (rf0 + rf1) + (rf2 + rf3);
+  return kPInt8 ? static_cast<float>(ri0 + ri1) * (1.0f / 127.0f) : (rf0 + rf1) + (rf2 + rf3);
 }
 
 // The rows of one query tile (4 warps, one row per thread).
@@ -354,7 +357,7 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
 // tile j for B's pass of tile j - 1, tile B for A's pass of tile j; a tile
 // arrives only where its partner will wait (the causal tile B has one key
 // tile more than A, and a pair may lack B).
-template <int D, bool kInt8>
+template <int D, bool kSInt8, bool kPInt8>
 __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars, TileBars& partner, uint32_t tS,
                                           uint32_t tPV, uint8_t* sP, const float* sKsc, const float* sVsc, int qt,
                                           int ntiles, int x, int nt_partner, int bh, int b, int h, int quarter,
@@ -390,7 +393,7 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     if (p.causal) kmax = min(kmax, qrow - key0 + 1);
 
     // ---- (1) row max ----
-    const float tmax = partial ? tile_row_max<kInt8, true>(tS, kmax, ksc) : tile_row_max<kInt8, false>(tS, kmax, ksc);
+    const float tmax = partial ? tile_row_max<kSInt8, true>(tS, kmax, ksc) : tile_row_max<kSInt8, false>(tS, kmax, ksc);
     const float m_new = fmaxf(m_run, tmax);
     const float m_use = m_new == -CUDART_INF_F ? 0.0f : m_new;
     const float alpha = ex2(m_run - m_use);     // 0 on the first tile
@@ -403,37 +406,37 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     }
 
     // ---- (2) probabilities, 8-bit rounding, P to shared memory ----
-    const bool my_turn_waits = kPingPong<kInt8> && (x == 0 ? (j >= 1 && j - 1 < nt_partner) : (j < nt_partner));
+    const bool my_turn_waits = kPingPong<kPInt8> && (x == 0 ? (j >= 1 && j - 1 < nt_partner) : (j < nt_partner));
     if (my_turn_waits) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.turn, (x == 0 ? j - 1 : j) & 1, abort_flag, p.err));
       if (!ok) break;
     }
-    const float toff = (kInt8 ? kLog2_127 : 0.0f) - m_use;
-    const float rowsum = partial ? tile_probs<kInt8, true>(tS, prow, rsw, ksc, toff, kmax)
-                                 : tile_probs<kInt8, false>(tS, prow, rsw, ksc, toff, kmax);
+    const float toff = (kPInt8 ? kLog2_127 : 0.0f) - m_use;
+    const float rowsum = partial ? tile_probs<kSInt8, kPInt8, true>(tS, prow, rsw, ksc, toff, kmax)
+                                 : tile_probs<kSInt8, kPInt8, false>(tS, prow, rsw, ksc, toff, kmax);
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(&bars.p_full);
-    if (kPingPong<kInt8> && (x == 0 ? j < nt_partner : j + 1 < nt_partner)) mbar_arrive(&partner.turn);
+    if (kPingPong<kPInt8> && (x == 0 ? j < nt_partner : j + 1 < nt_partner)) mbar_arrive(&partner.turn);
     l_run = l_run * alpha + rowsum;
     m_run = m_new;
 
     // ---- (3) fold PV_{j-1}: O <- alpha_j (O + g_{j-1} PV_{j-1}) ----
     // (O is kept relative to the newest running max.)
     if (j > 0) {
-      if (__all_sync(0xffffffffu, alpha == 1.0f)) fold_pv<D, kInt8, false>(O, tPV, alpha, alpha * g_prev);
-      else fold_pv<D, kInt8, true>(O, tPV, alpha, alpha * g_prev);
+      if (__all_sync(0xffffffffu, alpha == 1.0f)) fold_pv<D, kPInt8, false>(O, tPV, alpha, alpha * g_prev);
+      else fold_pv<D, kPInt8, true>(O, tPV, alpha, alpha * g_prev);
       tc_fence_before();
       mbar_arrive(&bars.pv_free);
     }
-    g_prev = vscale * (kInt8 ? (1.0f / 127.0f) : 1.0f);
+    g_prev = vscale * (kPInt8 ? (1.0f / 127.0f) : 1.0f);
   }
   if (!ok || ntiles == 0) return;
   // last product: O += g_{n-1} PV_{n-1}
   ok = __all_sync(0xffffffffu, mbar_wait(&bars.pv_full, (ntiles - 1) & 1, abort_flag, p.err));
   if (!ok) return;
   tc_fence_after();
-  fold_pv<D, kInt8, false>(O, tPV, 1.0f, g_prev);
+  fold_pv<D, kPInt8, false>(O, tPV, 1.0f, g_prev);
 
   // epilogue: out = O / l (bf16), lse
   if (qrow < p.Nq) {
@@ -453,33 +456,62 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
   }
 }
 
+// Four bytes each holding a 4-bit two's complement code (0..15) -> the same
+// codes as signed bytes: bit 3 times 0x1E spreads to 0xF0 within each byte.
+__device__ __forceinline__ uint32_t sext_nibbles(uint32_t x) { return x | ((x & 0x08080808u) * 0x1Eu); }
+
+// 32 packed INT4 codes (16 bytes; element 2i in the low nibble of byte i)
+// -> 32 INT8 codes in element order (two 16-byte chunks).
+__device__ __forceinline__ void widen_int4x32(uint4 w, uint4& lo16, uint4& hi16) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t lo = sext_nibbles(in[k] & 0x0F0F0F0Fu);          // elements 8k, 8k+2, 8k+4, 8k+6
+    const uint32_t hi = sext_nibbles((in[k] >> 4) & 0x0F0F0F0Fu);   // elements 8k+1, 8k+3, ...
+    o[2 * k] = __byte_perm(lo, hi, 0x5140);
+    o[2 * k + 1] = __byte_perm(lo, hi, 0x7362);
+  }
+  lo16 = make_uint4(o[0], o[1], o[2], o[3]);
+  hi16 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 // Grid: one CTA per pair of consecutive query tiles (2i, 2i+1) of one (b, h),
-// the pairs with the most key tiles first (causal).
-template <int D, bool kInt8>
+// the pairs with the most key tiles first (causal). kSInt8: Q/K codes INT8
+// (else e4m3); kVCode: V codes e4m3 (0), INT8 (1) or packed INT4 (2, widened
+// to INT8 in shared memory by warp 3 before the P.V products). P is rounded
+// to INT8 codes for integer V and to e4m3 for e4m3 V.
+template <int D, bool kSInt8, int kVCode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using L = Smem<D>;
+  constexpr bool kPInt8 = kVCode != 0;
+  constexpr bool kV4 = kVCode == 2;
+  using L = Smem<D, kVCode>;
   constexpr uint32_t kSwz = D == 128 ? 2u : 4u;       // descriptor swizzle: 128B / 64B
   constexpr uint32_t kRowB = D;                        // bytes per code row
   constexpr uint32_t kSBO = 8 * kRowB;                 // 8-row core-matrix group stride
   // S = Q K^T: A = Q (K-major), B = K (K-major), M = N = 128.
-  constexpr uint32_t kIdescQK = instr_desc(kInt8 ? 2u : 1u, kInt8 ? 1u : 0u, kInt8 ? 1u : 0u, 0u, 0u, kTileN, kTileM);
+  constexpr uint32_t kIdescQK =
+      instr_desc(kSInt8 ? 2u : 1u, kSInt8 ? 1u : 0u, kSInt8 ? 1u : 0u, 0u, 0u, kTileN, kTileM);
   // PV = P V: A = P (K-major over keys), B = V (MN-major: channels contiguous), N = D.
-  constexpr uint32_t kIdescPV = instr_desc(kInt8 ? 2u : 1u, kInt8 ? 1u : 0u, kInt8 ? 1u : 0u, 0u, 1u, D, kTileM);
+  constexpr uint32_t kIdescPV = instr_desc(kPInt8 ? 2u : 1u, kPInt8 ? 1u : 0u, kPInt8 ? 1u : 0u, 0u, 1u, D, kTileM);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + L::kQ;                          // [2][128 x D]
   uint8_t* sP = smem + L::kP;                          // [2][128 x 128]
   uint8_t* sK = smem + L::kK;                          // [stages][128 x D]
-  uint8_t* sV = smem + L::kV;                          // [stages][128 x D]
+  uint8_t* sV = smem + L::kV;                          // [stages][128 x D] (INT4: 128 x D/2)
+  uint8_t* sW = smem + L::kW;                          // INT4: [2][128 x D] widened V
 
   __shared__ __align__(8) uint64_t bar_q_full;
   __shared__ __align__(8) uint64_t bar_kv_full[kStagesKV];
   __shared__ __align__(8) uint64_t bar_kv_empty[kStagesKV];
   __shared__ __align__(8) TileBars bars[2];
   __shared__ __align__(8) uint64_t bar_drain[2];
+  __shared__ __align__(8) uint64_t bar_wv_full[2];     // INT4: widened V(j) in sW[j & 1] (warp 3)
+  __shared__ __align__(8) uint64_t bar_wv_empty[2];    // INT4: sW[j & 1] read by both tiles' P.V
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ float sKsc[kMaxBlk], sVsc[kMaxBlk];
@@ -513,6 +545,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bar_drain[0], 1);
     mbar_init(&bar_drain[1], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar_wv_full[x], 1);
+      mbar_init(&bar_wv_empty[x], 2);
+    }
     abort_flag = 0;
     mbar_fence_init();
   }
@@ -544,9 +580,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_kv_full[st], 2 * L::kTileBytes);
+        mbar_arrive_expect_tx(&bar_kv_full[st], L::kTileBytes + L::kVTileBytes);
         tma_load_4d(sK + st * L::kTileBytes, &tmK, &bar_kv_full[st], 0, j * kTileN, h, b);
-        tma_load_4d(sV + st * L::kTileBytes, &tmV, &bar_kv_full[st], 0, j * kTileN, h, b);
+        tma_load_4d(sV + st * L::kVTileBytes, &tmV, &bar_kv_full[st], 0, j * kTileN, h, b);
       }
       __syncwarp();
     }
@@ -569,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = warp - 1;
     const int nt = nt2[x];
     const uint32_t aQ = smem_u32(sQ) + x * L::kTileBytes, aP = smem_u32(sP) + x * kTileM * kTileN;
-    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aW = smem_u32(sW);
     const uint32_t tS = tmem + x * 256, tPV = tmem + x * 256 + 128;
     TileBars& tb = bars[x];
     auto issue_s = [&](int j) {
@@ -579,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < D / 32; ++kk) {
           const uint64_t da = smem_desc(aQ + kk * 32, 16, kSBO, kSwz);
           const uint64_t db = smem_desc(kbase + kk * 32, 16, kSBO, kSwz);
-          mma_ss<kInt8>(tS, da, db, kIdescQK, kk > 0 ? 1u : 0u);
+          mma_ss<kSInt8>(tS, da, db, kIdescQK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&tb.s_full);
       }
@@ -591,7 +627,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err));
       if (!ok) break;
       if (j >= nt) {
-        if (lane == 0) mbar_arrive(&bar_kv_empty[st]);
+        // (INT4: arrive only once the widened tile is there, so that this
+        // early arrival cannot count toward the buffer's previous use.)
+        if constexpr (kV4) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar_wv_full[j & 1], (j >> 1) & 1, &abort_flag, p.err));
+          if (!ok) break;
+        }
+        if (lane == 0) {
+          mbar_arrive(&bar_kv_empty[st]);
+          if constexpr (kV4) mbar_arrive(&bar_wv_empty[j & 1]);
+        }
         __syncwarp();
         continue;
       }
@@ -611,18 +656,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&tb.pv_free, (j - 1) & 1, &abort_flag, p.err));
         if (!ok) break;
       }
+      if constexpr (kV4) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar_wv_full[j & 1], (j >> 1) & 1, &abort_flag, p.err));
+        if (!ok) break;
+      }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vbase = aV + st * L::kTileBytes;
+        const uint32_t vbase = kV4 ? aW + (j & 1) * L::kTileBytes : aV + st * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kTileN / 32; ++kk) {
           const uint64_t da = smem_desc(aP + kk * 32, 16, 1024, 2u);
           // MN-major V: 32 keys per MMA = 4 groups of 8 key rows, SBO apart.
           const uint64_t db = smem_desc(vbase + kk * 32 * kRowB, kTileN * kRowB, kSBO, kSwz);
-          mma_ss<kInt8>(tPV, da, db, kIdescPV, kk > 0 ? 1u : 0u);
+          mma_ss<kPInt8>(tPV, da, db, kIdescPV, kk > 0 ? 1u : 0u);
         }
         mma_commit(&tb.pv_full);
         mma_commit(&bar_kv_empty[st]);
+        if constexpr (kV4) mma_commit(&bar_wv_empty[j & 1]);
       }
       __syncwarp();
     }
@@ -634,6 +684,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 3) {
     regs_dec<kRegsLow>();
+    if constexpr (kV4) {
+      // ------------------------------------------------------------ INT4 V widening
+      // Packed V tile j (stage j % 3, D/2 bytes per key row) -> INT8 codes in
+      // sW[j & 1], laid out as a TMA load of INT8 codes with the same swizzle
+      // would leave them (16-byte chunk c of row t at chunk c ^ swz(t)).
+      constexpr int kPC = D / 32;                      // packed 16-byte chunks per row
+      for (int j = 0; j < nt_max; ++j) {
+        const int st = j % kStagesKV;
+        bool ok = mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err);
+        if (ok && j >= 2) ok = mbar_wait(&bar_wv_empty[j & 1], ((j >> 1) - 1) & 1, &abort_flag, p.err);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const uint4* src = reinterpret_cast<const uint4*>(sV + st * L::kVTileBytes);
+        uint8_t* dst = sW + (j & 1) * L::kTileBytes;
+#pragma unroll 4
+        for (int q = lane; q < kTileN * kPC; q += 32) {
+          const int t = q / kPC, c = q % kPC;
+          uint4 lo16, hi16;
+          widen_int4x32(src[q], lo16, hi16);
+          const int swz = D == 128 ? (t & 7) : ((t >> 1) & 3);
+          *reinterpret_cast<uint4*>(dst + t * D + (((2 * c) ^ swz) << 4)) = lo16;
+          *reinterpret_cast<uint4*>(dst + t * D + (((2 * c + 1) ^ swz) << 4)) = hi16;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_wv_full[j & 1]);
+      }
+    }
   } else {
     // ------------------------------------------------------------ softmax rows
     regs_inc<kRegsHigh>();
@@ -648,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 256);
     if (qt2[x] >= 0)
-      tile_rows<D, kInt8>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
+      tile_rows<D, kSInt8, kPInt8>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
                           sKsc, sVsc, qt2[x], nt2[x], x, nt2[1 - x], bh, b, h, warp & 3, lane, &abort_flag);
   }
 
@@ -684,11 +761,32 @@ bool make_map(CUtensorMap* m, const void* base, int layout, int B, int H, int N,
                        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int D, bool kInt8>
+// Packed INT4 V: {D/2, N, H, B} bytes, box {D/2, 128, 1, 1}, unswizzled (the
+// widening warp reads it linearly).
+bool make_map_v4(CUtensorMap* m, const void* base, int layout, int B, int H, int N, int D) {
+  const uint64_t Db = static_cast<uint64_t>(D / 2);
+  const uint64_t dims[4] = {Db, static_cast<uint64_t>(N), static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
+  uint64_t strides[3];
+  if (layout == 0) {
+    strides[0] = Db;
+    strides[1] = static_cast<uint64_t>(N) * Db;
+    strides[2] = static_cast<uint64_t>(H) * N * Db;
+  } else {
+    strides[0] = static_cast<uint64_t>(H) * Db;
+    strides[1] = Db;
+    strides[2] = static_cast<uint64_t>(N) * H * Db;
+  }
+  const uint32_t box[4] = {static_cast<uint32_t>(Db), static_cast<uint32_t>(kTileN), 1, 1};
+  return encode_map_u8(m, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int D, bool kSInt8, int kVCode>
 cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   CUtensorMap mq, mk, mv;
+  const bool v_ok = kVCode == 2 ? make_map_v4(&mv, a.v, a.layout, a.B, a.H, a.Nkv, D)
+                                : make_map(&mv, a.v, a.layout, a.B, a.H, a.Nkv, D);
   if (!make_map(&mq, a.q, a.layout, a.B, a.H, a.Nq, D) || !make_map(&mk, a.k, a.layout, a.B, a.H, a.Nkv, D) ||
-      !make_map(&mv, a.v, a.layout, a.B, a.H, a.Nkv, D))
+      !v_ok)
     return cudaErrorInvalidValue;
   PrefillParams p;
   p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
@@ -703,8 +801,9 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   p.layout = a.layout;
   p.scale_log2 = a.scale_log2;
   p.err = err;
-  auto k = prefill_kernel<D, kInt8>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::kBytes);
+  auto k = prefill_kernel<D, kSInt8, kVCode>;
+  constexpr int kSmem = Smem<D, kVCode>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   // The register split inside the kernel needs at least kRegsNeeded
   // registers per thread at launch; never launch with fewer.
@@ -713,19 +812,36 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   if (e != cudaSuccess) return e;
   if (fa.numRegs < kRegsNeeded) return cudaErrorInvalidConfiguration;
   const int64_t grid = static_cast<int64_t>(p.npairs) * a.B * a.H;
-  k<<<static_cast<unsigned>(grid), kThreads, Smem<D>::kBytes, st>>>(mq, mk, mv, p);
+  k<<<static_cast<unsigned>(grid), kThreads, kSmem, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int* err) {
+  if (a.int8) {
+    if (a.v_code == 1) return launch_t<D, true, 1>(a, st, err);
+    if (a.v_code == 0) return launch_t<D, true, 0>(a, st, err);
+    if (a.v_code == 2) return launch_t<D, true, 2>(a, st, err);
+  } else if (a.v_code == 0) {
+    return launch_t<D, false, 0>(a, st, err);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 bool prefill_supported(int D) { return D == 64 || D == 128; }
 
+// Q/K INT8 with V e4m3, INT8 or packed INT4; Q/K e4m3 with V e4m3.
+bool prefill_codes_supported(int qk_int8, int v_code) { return qk_int8 ? (v_code >= 0 && v_code <= 2) : v_code == 0; }
+
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st, int num_sms, int* err) {
   (void)num_sms;
-  if (a.D == 128) return a.int8 ? launch_t<128, true>(a, st, err) : launch_t<128, false>(a, st, err);
-  if (a.D == 64) return a.int8 ? launch_t<64, true>(a, st, err) : launch_t<64, false>(a, st, err);
+  if (!prefill_codes_supported(a.int8, a.v_code)) return cudaErrorInvalidValue;
+  if (a.D == 128) return launch_d<128>(a, st, err);
+  if (a.D == 64) return launch_d<64>(a, st, err);
   return cudaErrorInvalidValue;
 }
+
 
 }  // namespace qattn

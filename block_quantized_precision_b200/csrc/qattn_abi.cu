@@ -155,9 +155,11 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype, qa
                                         qattn_stream_t stream) {
   if (B < 0 || H < 0 || N < 0 || D <= 0 || block_tokens <= 0) return QATTN_ERR_INVALID_ARG;
   if (x_dtype != QATTN_F16 && x_dtype != QATTN_BF16) return QATTN_ERR_INVALID_ARG;
-  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3 && code_dtype != QATTN_INT4_PACKED)
+    return QATTN_ERR_INVALID_ARG;
   if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
   if (!rotate_block_quant_supported(D, block_tokens)) return QATTN_ERR_UNSUPPORTED;
+  if (code_dtype == QATTN_INT4_PACKED && rot) return QATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * N == 0) return QATTN_OK;
   if (!x || !codes || !scales) return QATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes) || (rot && !aligned16(rot))) return QATTN_ERR_ALIGNMENT;
@@ -170,21 +172,26 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype, qa
   a.layout = layout;
   a.B = B; a.H = H; a.N = N; a.D = D; a.T = block_tokens;
   a.rot = rot;
-  a.int8 = code_dtype == QATTN_INT8;
+  a.int8 = code_dtype == QATTN_INT8 || code_dtype == QATTN_INT4_PACKED;
+  a.int4 = code_dtype == QATTN_INT4_PACKED;
   a.codes = codes;
   a.scales = scales;
   return from_cuda(launch_rotate_block_quant(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
 }
 
-qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,
-                             const void* v_codes, const float* v_scales, qattn_dtype_t code_dtype,
-                             qattn_layout_t layout, int B, int H, int N_q, int N_kv, int D, int q_block,
-                             int kv_block, int causal, float softmax_scale, void* out, float* lse,
-                             qattn_stream_t stream) {
+qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, const void* k_codes,
+                                   const float* k_scales, const void* v_codes, const float* v_scales,
+                                   qattn_dtype_t qk_dtype, qattn_dtype_t v_dtype, qattn_layout_t layout, int B,
+                                   int H, int N_q, int N_kv, int D, int q_block, int kv_block, int causal,
+                                   float softmax_scale, void* out, float* lse, qattn_stream_t stream) {
   if (B < 0 || H < 0 || N_q < 0 || N_kv < 0 || D <= 0) return QATTN_ERR_INVALID_ARG;
-  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (qk_dtype != QATTN_INT8 && qk_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (v_dtype != QATTN_INT8 && v_dtype != QATTN_FP8_E4M3 && v_dtype != QATTN_INT4_PACKED)
+    return QATTN_ERR_INVALID_ARG;
   if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return QATTN_ERR_INVALID_ARG;
+  const int v_code = v_dtype == QATTN_FP8_E4M3 ? 0 : v_dtype == QATTN_INT8 ? 1 : 2;
+  if (!prefill_codes_supported(qk_dtype == QATTN_INT8, v_code)) return QATTN_ERR_UNSUPPORTED;
   if (causal && N_q != N_kv) return QATTN_ERR_UNSUPPORTED;
   if (q_block != 128 || kv_block != 256) return QATTN_ERR_UNSUPPORTED;
   if (!prefill_supported(D)) return QATTN_ERR_UNSUPPORTED;
@@ -202,7 +209,8 @@ qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const v
   a.q = q_codes; a.qs = q_scales;
   a.k = k_codes; a.ks = k_scales;
   a.v = v_codes; a.vs = v_scales;
-  a.int8 = code_dtype == QATTN_INT8;
+  a.int8 = qk_dtype == QATTN_INT8;
+  a.v_code = v_code;
   a.layout = layout;
   a.B = B; a.H = H; a.Nq = N_q; a.Nkv = N_kv; a.D = D;
   a.causal = causal;
@@ -210,6 +218,17 @@ qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const v
   a.out = out;
   a.lse = lse;
   return from_cuda(launch_prefill(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
+}
+
+qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const void* k_codes, const float* k_scales,
+                             const void* v_codes, const float* v_scales, qattn_dtype_t code_dtype,
+                             qattn_layout_t layout, int B, int H, int N_q, int N_kv, int D, int q_block,
+                             int kv_block, int causal, float softmax_scale, void* out, float* lse,
+                             qattn_stream_t stream) {
+  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  return qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, code_dtype, code_dtype,
+                             layout, B, H, N_q, N_kv, D, q_block, kv_block, causal, softmax_scale, out, lse,
+                             stream);
 }
 
 size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D) {

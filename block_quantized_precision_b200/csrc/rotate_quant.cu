@@ -123,6 +123,15 @@ __device__ __forceinline__ int64_t row_offset(int layout, int H, int N, int D, i
 // Codes of eight values at a time
 // ---------------------------------------------------------------------------
 
+// Eight integer codes held in the low bits of t[e] (two's complement, |c| <= 7)
+// -> one word of nibbles, element e in bits 4e .. 4e+3.
+__device__ __forceinline__ uint32_t pack_nibbles8(const uint32_t (&t)[8]) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) w |= (t[e] & 0xFu) << (4 * e);
+  return w;
+}
+
 // Codes of 8 values by the division-free path, packed little-endian into lo
 // (values 0..3) and hi (4..7). Returns false when any value is too close to a
 // rounding boundary (or, for e4m3, in the subnormal range) for the product
@@ -137,7 +146,7 @@ __device__ __forceinline__ int64_t row_offset(int layout, int H, int N, int D, i
 // y * rcp rounded first; the bound holds as well). The rotation kernel uses
 // it: the packed form measured slower there, its FMA loop being compiled
 // differently next to it.
-template <bool kInt8, bool kPacked = true>
+template <bool kInt8, bool kPacked = true, bool kInt4 = false>
 __device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
   uint32_t t[8];
   if constexpr (kInt8 && !kPacked) {
@@ -166,8 +175,13 @@ __device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint
       t[2 * i] = __float_as_uint(m.x);
       t[2 * i + 1] = __float_as_uint(m.y);
     }
-    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    if constexpr (kInt4) {
+      lo = pack_nibbles8(t);
+      hi = 0;
+    } else {
+      lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+      hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    }
     return dmax <= 0.4999f;
   } else {
     bool ok = true;
@@ -189,7 +203,9 @@ __device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint
 // The packed INT8 / e4m3 fast path with one flag per value: bit e of the
 // result is set when value e's code must come from the IEEE quotient (same
 // bounds as codes8_fast). The codes of unflagged values are final.
-template <bool kInt8>
+// kInt4 (with kInt8): the same integer codes (|quotient| <= 7.5), packed two
+// per byte into lo (element 2i in the low nibble of byte i); hi is unused.
+template <bool kInt8, bool kInt4 = false>
 __device__ __forceinline__ uint32_t codes8_flags(const float (&f)[8], float rcp, uint32_t& lo, uint32_t& hi) {
   uint32_t t[8];
   uint32_t flags = 0;
@@ -207,8 +223,13 @@ __device__ __forceinline__ uint32_t codes8_flags(const float (&f)[8], float rcp,
       t[2 * i] = __float_as_uint(m.x);
       t[2 * i + 1] = __float_as_uint(m.y);
     }
-    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    if constexpr (kInt4) {
+      lo = pack_nibbles8(t);
+      hi = 0;
+    } else {
+      lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+      hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    }
   } else {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -227,10 +248,11 @@ __device__ __forceinline__ uint32_t codes8_flags(const float (&f)[8], float rcp,
 
 // Code byte of one value from the IEEE quotient (the rare path; inline, as a
 // call per value measured far slower).
-template <bool kInt8>
+template <bool kInt8, bool kInt4 = false>
 __device__ __forceinline__ uint32_t code_exact(float y, float scale) {
   const float v = __fdiv_rn(y, scale);
-  if constexpr (kInt8) return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(v)))) & 0xFFu;
+  if constexpr (kInt4) return static_cast<uint32_t>(max(-7, min(7, __float2int_rn(v)))) & 0xFu;
+  else if constexpr (kInt8) return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(v)))) & 0xFFu;
   else return cvt_e4m3x2(v, 0.0f) & 0xFFu;
 }
 
@@ -442,7 +464,8 @@ struct QuantSmem {
   static constexpr int kBytes = kQStages * kStage + 128;
 };
 
-template <int D, int T, bool kInt8, bool kBf16>
+// kInt4 (with kInt8): INT4 codes, scale absmax / 7, two per byte.
+template <int D, int T, bool kInt8, bool kBf16, bool kInt4>
 __global__ void __launch_bounds__(kQThreads, 1)
     quant_kernel(const __grid_constant__ CUtensorMap tmX, int layout, int B, int H, int N,
                  uint8_t* __restrict__ codes, float* __restrict__ scales, int* err) {
@@ -517,32 +540,39 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (issued < total) issue(issued, (it + kQStages - 1) % kQStages);
       issued += gridDim.x;
     }
-    const float scale = __fdiv_rn(amax, kInt8 ? 127.0f : 448.0f);
+    const float scale = __fdiv_rn(amax, kInt4 ? 7.0f : kInt8 ? 127.0f : 448.0f);
     const float rcp = __frcp_rn(scale);
     const bool slow = scale < 1.17549435e-38f;        // zero or subnormal scale: exact path
     if (tid == 0) scales[static_cast<int64_t>(bh) * nblk + blk] = scale;
 
-    // Vector i of this thread: row r0 + i * kRowStep, channels 8c .. 8c + 7.
+    // Vector i of this thread: row r0 + i * kRowStep, channels 8c .. 8c + 7
+    // (code bytes 8c .. 8c + 7; INT4: bytes 4c .. 4c + 3).
     constexpr int kRowStep = kQThreads / kCG;
+    constexpr int kCB = kInt4 ? 4 : 8;                 // code bytes per vector
     const int r0 = tid / kCG, c = tid % kCG;
-    const int64_t rstride = layout == 0 ? D : static_cast<int64_t>(H) * D;   // between token rows
-    uint8_t* out = codes + row_offset(layout, H, N, D, b, h, n0 + r0) + c * 8;
+    const int64_t rstride = (layout == 0 ? D : static_cast<int64_t>(H) * D) / (kInt4 ? 2 : 1);
+    uint8_t* out = codes + row_offset(layout, H, N, D, b, h, n0 + r0) / (kInt4 ? 2 : 1) + c * kCB;
+    auto store = [&](int i, uint2 w) {
+      if constexpr (kInt4) *reinterpret_cast<uint32_t*>(out + i * kRowStep * rstride) = w.x;
+      else *reinterpret_cast<uint2*>(out + i * kRowStep * rstride) = w;
+    };
     // All codes first, with no branch between the vectors (so their
-    // dependent arithmetic interleaves), stored at once; then the few values
-    // too close to a rounding boundary for the fast path are recomputed from
-    // the IEEE quotient one by one (re-read from the stage, which stays until
-    // the next barrier) and their bytes rewritten. A zero scale gives zero
-    // codes; a subnormal one sends every value to the exact path.
+    // dependent arithmetic interleaves), stored at once; then the vectors
+    // holding a value too close to a rounding boundary for the fast path are
+    // recomputed (re-read from the stage, which stays until the next
+    // barrier), the flagged values taken from the IEEE quotient, and stored
+    // again. A zero scale gives zero codes; a subnormal one sends every value
+    // to the exact path.
     uint32_t flagged = 0;                                  // vectors with a value to redo
 #pragma unroll
     for (int i = 0; i < kVec; ++i) {
       float f[8];
       unpack8(v[i], bf, f);
       uint2 w;
-      const bool ok = codes8_fast<kInt8>(f, rcp, w.x, w.y);
+      const bool ok = codes8_fast<kInt8, true, kInt4>(f, rcp, w.x, w.y);
       if (scale == 0.0f) w = make_uint2(0, 0);
       else flagged |= (ok && !slow ? 0u : 1u) << i;
-      if (r0 + i * kRowStep < rows) *reinterpret_cast<uint2*>(out + i * kRowStep * rstride) = w;
+      if (r0 + i * kRowStep < rows) store(i, w);
     }
 #pragma unroll 1
     while (flagged != 0) {
@@ -552,15 +582,25 @@ __global__ void __launch_bounds__(kQThreads, 1)
       float f[8];
       unpack8(src[tid + i * kQThreads], bf, f);
       uint2 w;
-      uint32_t fl = slow ? 0xFFu : codes8_flags<kInt8>(f, rcp, w.x, w.y);
-      uint8_t* o = out + i * kRowStep * rstride;
+      uint32_t fl = codes8_flags<kInt8, kInt4>(f, rcp, w.x, w.y);
+      if (slow) fl = 0xFFu;
 #pragma unroll 1
       while (fl != 0) {
         const int e = __ffs(fl) - 1;
         fl &= fl - 1;
-        const uint16_t hv = reinterpret_cast<const uint16_t*>(src + tid + i * kQThreads)[e];
-        o[e] = static_cast<uint8_t>(code_exact<kInt8>(bf ? bf16_bits_to_f32(hv) : f16_bits_to_f32(hv), scale));
+        float y = f[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) y = e == k ? f[k] : y;
+        const uint32_t cd = code_exact<kInt8, kInt4>(y, scale);
+        if constexpr (kInt4) {
+          w.x = (w.x & ~(0xFu << (4 * e))) | (cd << (4 * e));
+        } else {
+          const int sh = 8 * (e & 3);
+          if (e < 4) w.x = (w.x & ~(0xFFu << sh)) | (cd << sh);
+          else w.y = (w.y & ~(0xFFu << sh)) | (cd << sh);
+        }
       }
+      store(i, w);
     }
   }
   if (abort_flag && tid == 0) {
@@ -610,7 +650,8 @@ cudaError_t launch_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, in
   CUtensorMap tm;
   if (!make_map_x(&tm, a.x, a.layout, a.B, a.H, a.N, D, T)) return cudaErrorInvalidValue;
   using L = QuantSmem<D, T>;
-  auto k = a.is_bf16 ? quant_kernel<D, T, kInt8, true> : quant_kernel<D, T, kInt8, false>;
+  auto k = a.int4 ? (a.is_bf16 ? quant_kernel<D, T, true, true, true> : quant_kernel<D, T, true, false, true>)
+                  : (a.is_bf16 ? quant_kernel<D, T, kInt8, true, false> : quant_kernel<D, T, kInt8, false, false>);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);

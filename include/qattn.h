@@ -105,8 +105,14 @@ const char* qattn_status_string(qattn_status_t status);
  *               [B,H,N,D] or [B,N,H,D].
  * rot:          D x D float32 row-major (rot[k*D + j] = R[k][j]), or NULL.
  * block_tokens: tokens per block: 128 (Q) or 256 (K/V).
- * code_dtype:   QATTN_INT8 or QATTN_FP8_E4M3.
- * codes:        output, 1 byte per element, same layout and shape as x.
+ * code_dtype:   QATTN_INT8, QATTN_FP8_E4M3, or QATTN_INT4_PACKED (no
+ *               rotation: rot must be NULL, else QATTN_ERR_UNSUPPORTED):
+ *               scale = max|x| / 7, codes RNE(x / scale) clamped to [-7, 7]
+ *               ("FlashAttention 的 INT8/INT4 量化", 第二层, with the block
+ *               scales above), two per byte, element 2i in the low nibble
+ *               ("ops-transformer INT8/INT4 量化推理", 5.2).
+ * codes:        output, 1 byte per element (INT4: per 2 elements), same
+ *               layout as x ([..., D/2] for INT4).
  * scales:       output, float32 [B, H, ceil(N / block_tokens)].
  */
 qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype,
@@ -143,12 +149,38 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype,
  * softmax_scale: <= 0 selects 1/sqrt(D) (computed in float32).
  * out:          bfloat16, same layout as Q.
  * lse:          optional (NULL) float32 [B, H, N_q].
+ * code_dtype:   QATTN_INT8 or QATTN_FP8_E4M3 (Q, K and V alike; see
+ *               qattn_prefill_mixed for V in another type).
  */
 qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const void* k_codes,
                              const float* k_scales, const void* v_codes, const float* v_scales,
                              qattn_dtype_t code_dtype, qattn_layout_t layout, int B, int H,
                              int N_q, int N_kv, int D, int q_block, int kv_block, int causal,
                              float softmax_scale, void* out, float* lse, qattn_stream_t stream);
+
+/*
+ * Quantized prefill attention with V in its own code type (mixed precision).
+ *
+ * Defined by: "FlashAttention 的 INT8/INT4 量化", 第三层 (混合精度: Q/K in
+ * INT8 for the scores, V in a narrower format for the weighted sum) and
+ * 第二层 (INT4 codes widened to INT8 for the matmul).
+ *
+ * Same computation and arguments as qattn_prefill, with:
+ *   qk_dtype: QATTN_INT8 or QATTN_FP8_E4M3 (Q and K codes);
+ *   v_dtype:  QATTN_INT8, QATTN_FP8_E4M3 or QATTN_INT4_PACKED (V codes,
+ *             [B,H,N_kv,D/2] or [B,N_kv,H,D/2] bytes for INT4, as written by
+ *             qattn_rotate_block_quant). Supported pairs: INT8 Q/K with any V;
+ *             e4m3 Q/K with e4m3 V (else QATTN_ERR_UNSUPPORTED).
+ *   P is rounded to INT8 codes (round(127 p) / 127) when V is INT8 or INT4
+ *   (INT4 V is widened to INT8 on chip) and to e4m3 when V is e4m3.
+ * v_scales: float32 [B, H, ceil(N_kv / kv_block)] for every V type.
+ */
+qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, const void* k_codes,
+                                   const float* k_scales, const void* v_codes, const float* v_scales,
+                                   qattn_dtype_t qk_dtype, qattn_dtype_t v_dtype, qattn_layout_t layout,
+                                   int B, int H, int N_q, int N_kv, int D, int q_block, int kv_block,
+                                   int causal, float softmax_scale, void* out, float* lse,
+                                   qattn_stream_t stream);
 
 /*
  * Bytes of device workspace qattn_decode_kvq needs for these sizes on the

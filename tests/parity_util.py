@@ -42,6 +42,10 @@ def dequant_v_max(vc: np.ndarray, vs: np.ndarray, code_dtype: int, layout: int, 
     codes = head_rows(vc, layout, b, h)
     if code_dtype == synth.INT8:
         vals = np.abs(codes.view(np.int8).astype(np.float64))
+    elif code_dtype == synth.INT4_PACKED:
+        lo = ((codes & 0xF).astype(np.int16) ^ 8) - 8
+        hi = ((codes >> 4).astype(np.int16) ^ 8) - 8
+        vals = np.abs(np.concatenate([lo, hi], axis=1).astype(np.float64))
     else:
         vals = np.abs(orc.e4m3_decode(codes).astype(np.float64))
     per_tok = vals.max(axis=1)
