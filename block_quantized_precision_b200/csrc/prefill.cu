@@ -357,7 +357,11 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
 // tile j for B's pass of tile j - 1, tile B for A's pass of tile j; a tile
 // arrives only where its partner will wait (the causal tile B has one key
 // tile more than A, and a pair may lack B).
-template <int D, bool kSInt8, bool kPInt8>
+// kVBias: V arrives as code + 8 (INT4 widened to unsigned bytes); the
+// output then carries 8 * g * (sum of the row's P codes) per tile in every
+// channel, which the scalar C accumulates with the same rescaling as O and
+// removes at the end (O_true = O + C).
+template <int D, bool kSInt8, bool kPInt8, bool kVBias>
 __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars, TileBars& partner, uint32_t tS,
                                           uint32_t tPV, uint8_t* sP, const float* sKsc, const float* sVsc, int qt,
                                           int ntiles, int x, int nt_partner, int bh, int b, int h, int quarter,
@@ -376,6 +380,8 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
   for (int d = 0; d < D; ++d) O[d] = 0.0f;
   float m_run = -CUDART_INF_F, l_run = 0.0f;
   float g_prev = 0.0f;                          // V dequantization factor of the previous tile
+  float r_prev = 0.0f;                          // kVBias: sum of the previous tile's P codes
+  float C = 0.0f;                               // kVBias: -8 * accumulated g * P-code sums
   bool ok = true;
   for (int j = 0; j < ntiles; ++j) {
     ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full, j & 1, abort_flag, p.err));
@@ -428,8 +434,10 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
       else fold_pv<D, kPInt8, true>(O, tPV, alpha, alpha * g_prev);
       tc_fence_before();
       mbar_arrive(&bars.pv_free);
+      if constexpr (kVBias) C = alpha * (C - 8.0f * g_prev * r_prev);
     }
     g_prev = vscale * (kPInt8 ? (1.0f / 127.0f) : 1.0f);
+    if constexpr (kVBias) r_prev = rintf(rowsum * 127.0f);    // the integer sum of the P codes
   }
   if (!ok || ntiles == 0) return;
   // last product: O += g_{n-1} PV_{n-1}
@@ -437,6 +445,11 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
   if (!ok) return;
   tc_fence_after();
   fold_pv<D, kPInt8, false>(O, tPV, 1.0f, g_prev);
+  if constexpr (kVBias) {
+    C -= 8.0f * g_prev * r_prev;
+#pragma unroll
+    for (int d = 0; d < D; ++d) O[d] += C;
+  }
 
   // epilogue: out = O / l (bf16), lse
   if (qrow < p.Nq) {
@@ -456,19 +469,18 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
   }
 }
 
-// Four bytes each holding a 4-bit two's complement code (0..15) -> the same
-// codes as signed bytes: bit 3 times 0x1E spreads to 0xF0 within each byte.
-__device__ __forceinline__ uint32_t sext_nibbles(uint32_t x) { return x | ((x & 0x08080808u) * 0x1Eu); }
-
-// 32 packed INT4 codes (16 bytes; element 2i in the low nibble of byte i)
-// -> 32 INT8 codes in element order (two 16-byte chunks).
-__device__ __forceinline__ void widen_int4x32(uint4 w, uint4& lo16, uint4& hi16) {
+// 32 packed INT4 codes (16 bytes; element 2i in the low nibble of byte i,
+// two's complement) -> the 32 values code + 8 (0..15) as unsigned bytes in
+// element order (two 16-byte chunks). Flipping bit 3 of every nibble adds 8
+// to it modulo 16, which maps -8..7 onto 0..15.
+__device__ __forceinline__ void widen_int4x32_biased(uint4 w, uint4& lo16, uint4& hi16) {
   const uint32_t in[4] = {w.x, w.y, w.z, w.w};
   uint32_t o[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const uint32_t lo = sext_nibbles(in[k] & 0x0F0F0F0Fu);          // elements 8k, 8k+2, 8k+4, 8k+6
-    const uint32_t hi = sext_nibbles((in[k] >> 4) & 0x0F0F0F0Fu);   // elements 8k+1, 8k+3, ...
+    const uint32_t u = in[k] ^ 0x88888888u;
+    const uint32_t lo = u & 0x0F0F0F0Fu;                // elements 8k, 8k+2, 8k+4, 8k+6
+    const uint32_t hi = (u >> 4) & 0x0F0F0F0Fu;         // elements 8k+1, 8k+3, ...
     o[2 * k] = __byte_perm(lo, hi, 0x5140);
     o[2 * k + 1] = __byte_perm(lo, hi, 0x7362);
   }
@@ -479,8 +491,10 @@ __device__ __forceinline__ void widen_int4x32(uint4 w, uint4& lo16, uint4& hi16)
 // Grid: one CTA per pair of consecutive query tiles (2i, 2i+1) of one (b, h),
 // the pairs with the most key tiles first (causal). kSInt8: Q/K codes INT8
 // (else e4m3); kVCode: V codes e4m3 (0), INT8 (1) or packed INT4 (2, widened
-// to INT8 in shared memory by warp 3 before the P.V products). P is rounded
-// to INT8 codes for integer V and to e4m3 for e4m3 V.
+// in shared memory by warp 3 before the P.V products, as code + 8 in unsigned
+// bytes; the 8 * sum(P codes) this adds to every output channel of a row is
+// removed by a per-row scalar). P is rounded to INT8 codes for integer V and
+// to e4m3 for e4m3 V.
 template <int D, bool kSInt8, int kVCode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -495,7 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kIdescQK =
       instr_desc(kSInt8 ? 2u : 1u, kSInt8 ? 1u : 0u, kSInt8 ? 1u : 0u, 0u, 0u, kTileN, kTileM);
   // PV = P V: A = P (K-major over keys), B = V (MN-major: channels contiguous), N = D.
-  constexpr uint32_t kIdescPV = instr_desc(kPInt8 ? 2u : 1u, kPInt8 ? 1u : 0u, kPInt8 ? 1u : 0u, 0u, 1u, D, kTileM);
+  // (INT4 V is widened to unsigned bytes: B format u8.)
+  constexpr uint32_t kIdescPV =
+      instr_desc(kPInt8 ? 2u : 1u, kPInt8 ? 1u : 0u, kPInt8 && !kV4 ? 1u : 0u, 0u, 1u, D, kTileM);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -701,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = lane; q < kTileN * kPC; q += 32) {
           const int t = q / kPC, c = q % kPC;
           uint4 lo16, hi16;
-          widen_int4x32(src[q], lo16, hi16);
+          widen_int4x32_biased(src[q], lo16, hi16);
           const int swz = D == 128 ? (t & 7) : ((t >> 1) & 3);
           *reinterpret_cast<uint4*>(dst + t * D + (((2 * c) ^ swz) << 4)) = lo16;
           *reinterpret_cast<uint4*>(dst + t * D + (((2 * c + 1) ^ swz) << 4)) = hi16;
@@ -725,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 256);
     if (qt2[x] >= 0)
-      tile_rows<D, kSInt8, kPInt8>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
+      tile_rows<D, kSInt8, kPInt8, kV4>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
                           sKsc, sVsc, qt2[x], nt2[x], x, nt2[1 - x], bh, b, h, warp & 3, lane, &abort_flag);
   }
 
