@@ -193,6 +193,8 @@ def prefill_rows(qc, qs, kc, ks, vc, vs, code_dtype: int, layout: int, causal: b
         Nk = kc.shape[1]
     if Nkv is not None:
         Nk = Nkv
+    if code_dtype == INT4_PACKED:                          # packed: D/2 bytes per row
+        D *= 2
     arrs = [np.ascontiguousarray(a) for a in (qc, qs, kc, ks, vc, vs)]
     for a in arrs[1::2]:
         assert a.dtype == np.float32

@@ -144,3 +144,24 @@ def test_constant_v_reproduces_the_row(orc, v_dtype):
     out = orc.prefill_rows(qc, qs, kc, ks, vc, vs, synth.INT8, synth.BNSD, True, rows, want_f64=True,
                            v_dtype=v_dtype)[(0, 0)][1]
     assert np.allclose(out, deq[None, :], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_int4_qkv_equals_the_same_codes_held_as_int8(orc, causal):
+    """INT4 Q, K and V (rotated Q/K): identical outputs to the INT8 path fed
+    the same codes one per byte with the same scales -- INT4 codes widened to
+    INT8 for the matmul, as the page's INT4 layer states."""
+    B, H, N, D = 1, 2, 300, 64
+    rng = np.random.default_rng(21 + causal)
+    R = synth.haar_orthogonal(5, 0, D)
+    x = {n: _bf16(rng, (B, H, N, D)) for n in ("q", "k", "v")}
+    q4, qs = orc.rotate_block_quant(x["q"], synth.BF16, synth.BNSD, R, 128, synth.INT4_PACKED)
+    k4, ks = orc.rotate_block_quant(x["k"], synth.BF16, synth.BNSD, R, 256, synth.INT4_PACKED)
+    v4, vs = orc.rotate_block_quant(x["v"], synth.BF16, synth.BNSD, None, 256, synth.INT4_PACKED)
+    as8 = lambda c: _unpack(c).astype(np.int8).view(np.uint8)
+    rows = {(b, h): list(range(0, N, 4)) + [N - 1] for b in range(B) for h in range(H)}
+    a = orc.prefill_rows(q4, qs, k4, ks, v4, vs, synth.INT4_PACKED, synth.BNSD, causal, rows, want_f64=True)
+    b = orc.prefill_rows(as8(q4), qs, as8(k4), ks, as8(v4), vs, synth.INT8, synth.BNSD, causal, rows,
+                         want_f64=True)
+    for key in rows:
+        assert np.array_equal(a[key][1], b[key][1])
