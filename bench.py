@@ -429,6 +429,26 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                     "ms_prefill": round(ms_pf, 4), "TOPS_prefill": round(tops, 1),
                     "ms_quant_v": round(ms_qv, 4), "GB/s_quant_v": round(v_bytes / (ms_qv * 1e-3) / 1e9, 1),
                     "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TOPS", "frac": round(tops / int8_peak, 4)}}
+
+    # INT4 Q/K/V on the same problem (Q/K rotated), widened to INT8 on chip
+    c4 = {nm: qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
+                                          qa.QATTN_INT4_PACKED) for nm in ("q", "k", "v")}
+    pf4 = lambda: qa.qattn_prefill_mixed(*c4["q"], *c4["k"], *c4["v"], qa.QATTN_INT4_PACKED, qa.QATTN_INT4_PACKED,
+                                         p.layout, p.causal, out=out)
+    ms_pf4 = timeit(pf4, n, flush)
+
+    def full4():
+        for nm in ("q", "k", "v"):
+            qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
+                                        qa.QATTN_INT4_PACKED, c4[nm][0], c4[nm][1])
+        pf4()
+    ms_full4 = timeit(full4, n, flush)
+    tops4 = ops / (ms_pf4 * 1e-3) / 1e12
+    res["prefill_int4_qkv"] = {"workload": "%s, Q/K/V int4 packed" % p.name, "ms_prefill": round(ms_pf4, 4),
+                               "TOPS_prefill": round(tops4, 1), "ms_path": round(ms_full4, 4),
+                               "TOPS_path": round(ops / (ms_full4 * 1e-3) / 1e12, 1),
+                               "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TOPS",
+                                            "frac": round(tops4 / int8_peak, 4)}}
     return res
 
 
@@ -526,16 +546,18 @@ def profile_case(args):
             qa.qattn_decode_kvq(q, k, v, ks, vs, kvt, kv_block=p.kv_block, group=p.group)
     else:
         p = synth.FP8_LONG if c == "prefill_fp8" else synth.INT8_CAUSAL
-        # prefill_int4v: the INT8 causal problem with V in packed INT4
-        vt = qa.QATTN_INT4_PACKED if c == "prefill_int4v" else p.code_dtype
+        # prefill_int4v: the INT8 causal problem with V in packed INT4;
+        # prefill_int4: with Q, K and V in packed INT4
+        vt = qa.QATTN_INT4_PACKED if c in ("prefill_int4v", "prefill_int4") else p.code_dtype
+        qkt = qa.QATTN_INT4_PACKED if c == "prefill_int4" else p.code_dtype
         d = synth.make_prefill(p)
         x = {n: torch.from_numpy(d[n].view(np.int16)).to(dev).view(torch.bfloat16) for n in ("q", "k", "v")}
         rot = torch.from_numpy(d["rot"]).to(dev)
         for _ in range(args.warmup + args.steps):
-            qc = qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, p.code_dtype)
-            kc = qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, p.code_dtype)
+            qc = qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, qkt)
+            kc = qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, qkt)
             vc = qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, vt)
-            qa.qattn_prefill_mixed(*qc, *kc, *vc, p.code_dtype, vt, p.layout, p.causal)
+            qa.qattn_prefill_mixed(*qc, *kc, *vc, qkt, vt, p.layout, p.causal)
     torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
     print("case %s: ok" % c)
@@ -551,7 +573,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-heads", type=int, default=4, help="heads per reference-arm step")
-    ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "prefill_int4v", "decode_int8kv",
+    ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "prefill_int4v", "prefill_int4", "decode_int8kv",
                                                            "decode_int4kv"],
                     help="run one workload only (for profiler captures); prints no JSON")
     args = ap.parse_args()

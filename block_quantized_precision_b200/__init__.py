@@ -154,13 +154,15 @@ def qattn_prefill(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, code_
 def qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, qk_dtype: int, v_dtype: int,
                         layout: int, causal: bool, softmax_scale: float = 0.0, out=None, lse=None,
                         q_block: int = 128, kv_block: int = 256, stream=None):
-    """Quantized attention with V in its own code type (INT4 V: [..., D/2]
-    packed bytes); returns the bfloat16 output (layout of Q)."""
+    """Quantized attention with V in its own code type (packed INT4 codes:
+    [..., D/2] bytes); returns the bfloat16 output (layout of Q, D channels)."""
     import torch
     B, H, Nq, D = _dims(q_codes, layout)
+    if qk_dtype == QATTN_INT4_PACKED:
+        D *= 2
     Nkv = _dims(k_codes, layout)[2]
     if out is None:
-        out = torch.empty(q_codes.shape, dtype=torch.bfloat16, device=q_codes.device)
+        out = torch.empty(tuple(q_codes.shape[:-1]) + (D,), dtype=torch.bfloat16, device=q_codes.device)
     st = lib().qattn_prefill_mixed(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
                                    _ptr(v_scales), qk_dtype, v_dtype, layout, B, H, Nq, Nkv, D, q_block,
                                    kv_block, int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse),

@@ -91,17 +91,23 @@ struct PrefillParams {
   int* err;
 };
 
-// kVCode: V code type (0 e4m3, 1 INT8, 2 packed INT4 widened on chip).
-template <int D, int kVCode>
+// kQKCode / kVCode: code type of Q and K / of V (0 e4m3, 1 INT8, 2 packed
+// INT4 widened to INT8 on chip).
+template <int D, int kQKCode, int kVCode>
 struct Smem {
-  static constexpr int kTileBytes = kTileM * D;       // one 128-row code tile
-  static constexpr int kVTileBytes = kVCode == 2 ? kTileN * D / 2 : kTileBytes;   // one V tile as loaded
-  static constexpr int kQ = 0;                        // two Q tiles
+  static constexpr bool kK4 = kQKCode == 2, kV4 = kVCode == 2;
+  static constexpr int kTileBytes = kTileM * D;       // one 128-row tile of 8-bit codes
+  static constexpr int kQTileBytes = kK4 ? kTileM * D / 2 : kTileBytes;    // one Q tile as loaded
+  static constexpr int kKTileBytes = kK4 ? kTileN * D / 2 : kTileBytes;    // one K tile as loaded
+  static constexpr int kVTileBytes = kV4 ? kTileN * D / 2 : kTileBytes;    // one V tile as loaded
+  static constexpr int kQ = 0;                        // two Q tiles (8-bit codes)
   static constexpr int kP = kQ + 2 * kTileBytes;      // two P tiles: 128 rows x 128 keys
-  static constexpr int kK = kP + 2 * kTileM * kTileN;
-  static constexpr int kV = kK + kStagesKV * kTileBytes;
-  static constexpr int kW = kV + kStagesKV * kVTileBytes;  // INT4: two widened (INT8) V tiles
-  static constexpr int kEnd = kW + (kVCode == 2 ? 2 * kTileBytes : 0);
+  static constexpr int kK = kP + 2 * kTileM * kTileN; // K stages as loaded
+  static constexpr int kV = kK + kStagesKV * kKTileBytes;
+  static constexpr int kW = kV + kStagesKV * kVTileBytes;        // INT4 V: two widened tiles
+  static constexpr int kKw = kW + (kV4 ? 2 * kTileBytes : 0);    // INT4 K: two widened tiles
+  static constexpr int kQp = kKw + (kK4 ? 2 * kTileBytes : 0);   // INT4 Q: the two packed tiles
+  static constexpr int kEnd = kQp + (kK4 ? 2 * kQTileBytes : 0);
   static constexpr int kBytes = kEnd + 1024;          // slack for 1024-byte alignment
 };
 
@@ -234,7 +240,7 @@ __device__ __forceinline__ void fold_pv(float (&O)[D], uint32_t tPV, float alpha
 // INT32 scores, FP8 the float max; keys >= kmax are masked when kPartial.
 // Returns -inf if every key is masked.
 template <bool kInt8, bool kPartial>
-__device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc) {
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc, int sub) {
   if constexpr (kInt8) {
     int i0 = INT_MIN, i1 = INT_MIN, i2 = INT_MIN, i3 = INT_MIN;
     tmem_chunks<kTileN / kMaxW, kMaxW>(tS, [&](int c, uint32_t(&v)[kMaxW]) {
@@ -252,7 +258,7 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int kmax, float ksc) 
       }
     });
     const int im = max(max(i0, i1), max(i2, i3));
-    return im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im) * ksc;
+    return im == INT_MIN ? -CUDART_INF_F : static_cast<float>(im - sub) * ksc;
   } else {
     float f0 = -CUDART_INF_F, f1 = -CUDART_INF_F, f2 = -CUDART_INF_F, f3 = -CUDART_INF_F;
     tmem_chunks<kTileN / kMaxW, kMaxW>(tS, [&](int c, uint32_t(&v)[kMaxW]) {
@@ -361,11 +367,15 @@ __device__ __forceinline__ float tile_probs(uint32_t tS, uint8_t* prow, int rsw,
 // output then carries 8 * g * (sum of the row's P codes) per tile in every
 // channel, which the scalar C accumulates with the same rescaling as O and
 // removes at the end (O_true = O + C).
-template <int D, bool kSInt8, bool kPInt8, bool kVBias>
+// kKBias: K arrives as code + 8 (INT4 widened to unsigned bytes); every
+// score of row i then carries 8 * sum_d Q[i][d], subtracted with the scale
+// (q_wide: completes when the widened Q tile qrows is in shared memory).
+template <int D, bool kSInt8, bool kPInt8, bool kVBias, bool kKBias>
 __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars, TileBars& partner, uint32_t tS,
                                           uint32_t tPV, uint8_t* sP, const float* sKsc, const float* sVsc, int qt,
                                           int ntiles, int x, int nt_partner, int bh, int b, int h, int quarter,
-                                          int lane, volatile int* abort_flag) {
+                                          int lane, volatile int* abort_flag, uint64_t* q_wide,
+                                          const uint8_t* qrows) {
   const int r = quarter * 32 + lane;            // row within the tile (= TMEM lane)
   const int q0 = qt * kTileM;
   const int qrow = q0 + r;
@@ -383,6 +393,15 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
   float r_prev = 0.0f;                          // kVBias: sum of the previous tile's P codes
   float C = 0.0f;                               // kVBias: -8 * accumulated g * P-code sums
   bool ok = true;
+  int sub = 0;                                  // kKBias: 8 * sum of this row's Q codes
+  if constexpr (kKBias) {
+    ok = __all_sync(0xffffffffu, mbar_wait(q_wide, 0, abort_flag, p.err));
+    if (!ok) return;
+    const int* qr = reinterpret_cast<const int*>(qrows + r * D);   // (chunk order does not matter)
+#pragma unroll
+    for (int w = 0; w < D / 4; ++w) sub = __dp4a(qr[w], 0x01010101, sub);
+    sub *= 8;
+  }
   for (int j = 0; j < ntiles; ++j) {
     ok = __all_sync(0xffffffffu, mbar_wait(&bars.s_full, j & 1, abort_flag, p.err));
     if (!ok) break;
@@ -399,7 +418,8 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
     if (p.causal) kmax = min(kmax, qrow - key0 + 1);
 
     // ---- (1) row max ----
-    const float tmax = partial ? tile_row_max<kSInt8, true>(tS, kmax, ksc) : tile_row_max<kSInt8, false>(tS, kmax, ksc);
+    const float tmax = partial ? tile_row_max<kSInt8, true>(tS, kmax, ksc, sub)
+                               : tile_row_max<kSInt8, false>(tS, kmax, ksc, sub);
     const float m_new = fmaxf(m_run, tmax);
     const float m_use = m_new == -CUDART_INF_F ? 0.0f : m_new;
     const float alpha = ex2(m_run - m_use);     // 0 on the first tile
@@ -417,7 +437,8 @@ __device__ __forceinline__ void tile_rows(const PrefillParams& p, TileBars& bars
       ok = __all_sync(0xffffffffu, mbar_wait(&bars.turn, (x == 0 ? j - 1 : j) & 1, abort_flag, p.err));
       if (!ok) break;
     }
-    const float toff = (kPInt8 ? kLog2_127 : 0.0f) - m_use;
+    // (kKBias: the scores' offset 8 * sum(Q codes) leaves with the scale)
+    const float toff = (kPInt8 ? kLog2_127 : 0.0f) - m_use - (kKBias ? static_cast<float>(sub) * ksc : 0.0f);
     const float rowsum = partial ? tile_probs<kSInt8, kPInt8, true>(tS, prow, rsw, ksc, toff, kmax)
                                  : tile_probs<kSInt8, kPInt8, false>(tS, prow, rsw, ksc, toff, kmax);
     fence_proxy_async_smem();
@@ -488,26 +509,69 @@ __device__ __forceinline__ void widen_int4x32_biased(uint4 w, uint4& lo16, uint4
   hi16 = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// The same, as signed bytes (INT4 Q, widened once per CTA): bit 3 of each
+// nibble times 0x1E spreads to 0xF0 within its byte.
+__device__ __forceinline__ void widen_int4x32_signed(uint4 w, uint4& lo16, uint4& hi16) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t lo = in[k] & 0x0F0F0F0Fu;
+    uint32_t hi = (in[k] >> 4) & 0x0F0F0F0Fu;
+    lo |= (lo & 0x08080808u) * 0x1Eu;
+    hi |= (hi & 0x08080808u) * 0x1Eu;
+    o[2 * k] = __byte_perm(lo, hi, 0x5140);
+    o[2 * k + 1] = __byte_perm(lo, hi, 0x7362);
+  }
+  lo16 = make_uint4(o[0], o[1], o[2], o[3]);
+  hi16 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Widens one 128-row tile of packed INT4 codes (D/2 bytes per row, linear)
+// into 8-bit codes laid out as a TMA load of 8-bit codes with the tile's
+// swizzle would leave them (16-byte chunk c of row t at chunk c ^ swz(t)).
+// One warp; kBiased: code + 8 as unsigned bytes, else signed codes.
+template <int D, bool kBiased>
+__device__ __forceinline__ void widen_tile(const uint8_t* packed, uint8_t* dst, int lane) {
+  constexpr int kPC = D / 32;                          // packed 16-byte chunks per row
+  const uint4* src = reinterpret_cast<const uint4*>(packed);
+#pragma unroll 4
+  for (int q = lane; q < kTileN * kPC; q += 32) {
+    const int t = q / kPC, c = q % kPC;
+    uint4 lo16, hi16;
+    if constexpr (kBiased) widen_int4x32_biased(src[q], lo16, hi16);
+    else widen_int4x32_signed(src[q], lo16, hi16);
+    const int swz = D == 128 ? (t & 7) : ((t >> 1) & 3);
+    *reinterpret_cast<uint4*>(dst + t * D + (((2 * c) ^ swz) << 4)) = lo16;
+    *reinterpret_cast<uint4*>(dst + t * D + (((2 * c + 1) ^ swz) << 4)) = hi16;
+  }
+}
+
 // Grid: one CTA per pair of consecutive query tiles (2i, 2i+1) of one (b, h),
-// the pairs with the most key tiles first (causal). kSInt8: Q/K codes INT8
-// (else e4m3); kVCode: V codes e4m3 (0), INT8 (1) or packed INT4 (2, widened
-// in shared memory by warp 3 before the P.V products, as code + 8 in unsigned
+// the pairs with the most key tiles first (causal). kQKCode: Q/K codes e4m3
+// (0), INT8 (1) or packed INT4 (2: Q widened once to INT8 by warp 3, each K
+// tile widened to code + 8 in unsigned bytes, and the 8 * sum(Q codes) this
+// adds to every score of a row subtracted with the scale); kVCode: V codes
+// e4m3 (0), INT8 (1) or packed INT4 (2, widened in shared memory by warp 3 before the P.V products, as code + 8 in unsigned
 // bytes; the 8 * sum(P codes) this adds to every output channel of a row is
 // removed by a per-row scalar). P is rounded to INT8 codes for integer V and
 // to e4m3 for e4m3 V.
-template <int D, bool kSInt8, int kVCode>
+template <int D, int kQKCode, int kVCode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  constexpr bool kSInt8 = kQKCode != 0;
+  constexpr bool kK4 = kQKCode == 2;
   constexpr bool kPInt8 = kVCode != 0;
   constexpr bool kV4 = kVCode == 2;
-  using L = Smem<D, kVCode>;
+  using L = Smem<D, kQKCode, kVCode>;
   constexpr uint32_t kSwz = D == 128 ? 2u : 4u;       // descriptor swizzle: 128B / 64B
   constexpr uint32_t kRowB = D;                        // bytes per code row
   constexpr uint32_t kSBO = 8 * kRowB;                 // 8-row core-matrix group stride
   // S = Q K^T: A = Q (K-major), B = K (K-major), M = N = 128.
+  // (INT4 K is widened to unsigned bytes: B format u8.)
   constexpr uint32_t kIdescQK =
-      instr_desc(kSInt8 ? 2u : 1u, kSInt8 ? 1u : 0u, kSInt8 ? 1u : 0u, 0u, 0u, kTileN, kTileM);
+      instr_desc(kSInt8 ? 2u : 1u, kSInt8 ? 1u : 0u, kSInt8 && !kK4 ? 1u : 0u, 0u, 0u, kTileN, kTileM);
   // PV = P V: A = P (K-major over keys), B = V (MN-major: channels contiguous), N = D.
   // (INT4 V is widened to unsigned bytes: B format u8.)
   constexpr uint32_t kIdescPV =
@@ -520,6 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sK = smem + L::kK;                          // [stages][128 x D]
   uint8_t* sV = smem + L::kV;                          // [stages][128 x D] (INT4: 128 x D/2)
   uint8_t* sW = smem + L::kW;                          // INT4: [2][128 x D] widened V
+  uint8_t* sKw = smem + L::kKw;                        // INT4: [2][128 x D] widened K
+  uint8_t* sQp = smem + L::kQp;                        // INT4: [2][128 x D/2] packed Q
 
   __shared__ __align__(8) uint64_t bar_q_full;
   __shared__ __align__(8) uint64_t bar_kv_full[kStagesKV];
@@ -528,6 +594,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_drain[2];
   __shared__ __align__(8) uint64_t bar_wv_full[2];     // INT4: widened V(j) in sW[j & 1] (warp 3)
   __shared__ __align__(8) uint64_t bar_wv_empty[2];    // INT4: sW[j & 1] read by both tiles' P.V
+  __shared__ __align__(8) uint64_t bar_wk_full[2];     // INT4: widened K(j) in sKw[j & 1]
+  __shared__ __align__(8) uint64_t bar_wk_empty[2];    // INT4: sKw[j & 1] read by both tiles' S
+  __shared__ __align__(8) uint64_t bar_q_wide;         // INT4: both Q tiles widened into sQ
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ float sKsc[kMaxBlk], sVsc[kMaxBlk];
@@ -564,7 +633,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bar_wv_full[x], 1);
       mbar_init(&bar_wv_empty[x], 2);
+      mbar_init(&bar_wk_full[x], 1);
+      mbar_init(&bar_wk_empty[x], 2);
     }
+    mbar_init(&bar_q_wide, 1);
     abort_flag = 0;
     mbar_fence_init();
   }
@@ -584,9 +656,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar_q_full, (qt2[1] >= 0 ? 2 : 1) * L::kTileBytes);
+      mbar_arrive_expect_tx(&bar_q_full, (qt2[1] >= 0 ? 2 : 1) * L::kQTileBytes);
+      uint8_t* qdst = kK4 ? sQp : sQ;                  // INT4: packed, widened by warp 3
       for (int x = 0; x < 2; ++x)
-        if (qt2[x] >= 0) tma_load_4d(sQ + x * L::kTileBytes, &tmQ, &bar_q_full, 0, qt2[x] * kTileM, h, b);
+        if (qt2[x] >= 0) tma_load_4d(qdst + x * L::kQTileBytes, &tmQ, &bar_q_full, 0, qt2[x] * kTileM, h, b);
     }
     int j = 0;
     for (; j < nt_max; ++j) {
@@ -596,8 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bar_kv_full[st], L::kTileBytes + L::kVTileBytes);
-        tma_load_4d(sK + st * L::kTileBytes, &tmK, &bar_kv_full[st], 0, j * kTileN, h, b);
+        mbar_arrive_expect_tx(&bar_kv_full[st], L::kKTileBytes + L::kVTileBytes);
+        tma_load_4d(sK + st * L::kKTileBytes, &tmK, &bar_kv_full[st], 0, j * kTileN, h, b);
         tma_load_4d(sV + st * L::kVTileBytes, &tmV, &bar_kv_full[st], 0, j * kTileN, h, b);
       }
       __syncwarp();
@@ -621,12 +694,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = warp - 1;
     const int nt = nt2[x];
     const uint32_t aQ = smem_u32(sQ) + x * L::kTileBytes, aP = smem_u32(sP) + x * kTileM * kTileN;
-    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aW = smem_u32(sW);
+    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aW = smem_u32(sW), aKw = smem_u32(sKw);
     const uint32_t tS = tmem + x * 256, tPV = tmem + x * 256 + 128;
     TileBars& tb = bars[x];
+    // (INT4 K: the caller has waited for the widened tile.)
     auto issue_s = [&](int j) {
       if (lane == 0) {
-        const uint32_t kbase = aK + (j % kStagesKV) * L::kTileBytes;
+        const uint32_t kbase = kK4 ? aKw + (j & 1) * L::kTileBytes : aK + (j % kStagesKV) * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const uint64_t da = smem_desc(aQ + kk * 32, 16, kSBO, kSwz);
@@ -634,30 +708,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss<kSInt8>(tS, da, db, kIdescQK, kk > 0 ? 1u : 0u);
         }
         mma_commit(&tb.s_full);
+        if constexpr (kK4) mma_commit(&bar_wk_empty[j & 1]);
       }
       __syncwarp();
     };
-    bool ok = nt == 0 || __all_sync(0xffffffffu, mbar_wait(&bar_q_full, 0, &abort_flag, p.err));
+    bool ok = nt == 0 || __all_sync(0xffffffffu, mbar_wait(kK4 ? &bar_q_wide : &bar_q_full, 0, &abort_flag, p.err));
     for (int j = 0; ok && j < nt_max; ++j) {
       const int st = j % kStagesKV;
       ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err));
       if (!ok) break;
       if (j >= nt) {
-        // (INT4: arrive only once the widened tile is there, so that this
-        // early arrival cannot count toward the buffer's previous use.)
+        // (INT4: arrive only once the widened tiles are there, so that these
+        // early arrivals cannot count toward a buffer's previous use.)
+        if constexpr (kK4) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar_wk_full[j & 1], (j >> 1) & 1, &abort_flag, p.err));
+          if (!ok) break;
+        }
         if constexpr (kV4) {
           ok = __all_sync(0xffffffffu, mbar_wait(&bar_wv_full[j & 1], (j >> 1) & 1, &abort_flag, p.err));
           if (!ok) break;
         }
         if (lane == 0) {
           mbar_arrive(&bar_kv_empty[st]);
+          if constexpr (kK4) mbar_arrive(&bar_wk_empty[j & 1]);
           if constexpr (kV4) mbar_arrive(&bar_wv_empty[j & 1]);
         }
         __syncwarp();
         continue;
       }
-      tc_fence_after();
-      if (j == 0) issue_s(0);
+      if (j == 0) {
+        if constexpr (kK4) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar_wk_full[0], 0, &abort_flag, p.err));
+          if (!ok) break;
+        }
+        tc_fence_after();
+        issue_s(0);
+      }
       // S(j) consumed: P(j) is in shared memory
       ok = __all_sync(0xffffffffu, mbar_wait(&tb.p_full, j & 1, &abort_flag, p.err));
       if (!ok) break;
@@ -665,6 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j1 = j + 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[j1 % kStagesKV], (j1 / kStagesKV) & 1, &abort_flag, p.err));
         if (!ok) break;
+        if constexpr (kK4) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar_wk_full[j1 & 1], (j1 >> 1) & 1, &abort_flag, p.err));
+          if (!ok) break;
+        }
         tc_fence_after();
         issue_s(j1);
       }
@@ -700,31 +790,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 3) {
     regs_dec<kRegsLow>();
-    if constexpr (kV4) {
-      // ------------------------------------------------------------ INT4 V widening
-      // Packed V tile j (stage j % 3, D/2 bytes per key row) -> INT8 codes in
-      // sW[j & 1], laid out as a TMA load of INT8 codes with the same swizzle
-      // would leave them (16-byte chunk c of row t at chunk c ^ swz(t)).
-      constexpr int kPC = D / 32;                      // packed 16-byte chunks per row
-      for (int j = 0; j < nt_max; ++j) {
-        const int st = j % kStagesKV;
-        bool ok = mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err);
-        if (ok && j >= 2) ok = mbar_wait(&bar_wv_empty[j & 1], ((j >> 1) - 1) & 1, &abort_flag, p.err);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        const uint4* src = reinterpret_cast<const uint4*>(sV + st * L::kVTileBytes);
-        uint8_t* dst = sW + (j & 1) * L::kTileBytes;
-#pragma unroll 4
-        for (int q = lane; q < kTileN * kPC; q += 32) {
-          const int t = q / kPC, c = q % kPC;
-          uint4 lo16, hi16;
-          widen_int4x32_biased(src[q], lo16, hi16);
-          const int swz = D == 128 ? (t & 7) : ((t >> 1) & 3);
-          *reinterpret_cast<uint4*>(dst + t * D + (((2 * c) ^ swz) << 4)) = lo16;
-          *reinterpret_cast<uint4*>(dst + t * D + (((2 * c + 1) ^ swz) << 4)) = hi16;
+    if constexpr (kK4 || kV4) {
+      // ------------------------------------------------------------ INT4 widening
+      // Packed tiles -> 8-bit codes laid out as TMA loads of 8-bit codes
+      // would leave them: the two Q tiles once (signed), then per key tile j
+      // K(j) into sKw[j & 1] and V(j) into sW[j & 1] (code + 8, unsigned).
+      bool ok = true;
+      if constexpr (kK4) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar_q_full, 0, &abort_flag, p.err));
+        if (ok) {
+          for (int x = 0; x < 2; ++x)
+            if (qt2[x] >= 0) widen_tile<D, false>(sQp + x * L::kQTileBytes, sQ + x * L::kTileBytes, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_q_wide);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_wv_full[j & 1]);
+      }
+      for (int j = 0; ok && j < nt_max; ++j) {
+        const int st = j % kStagesKV;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err));
+        if (!ok) break;
+        if constexpr (kK4) {
+          if (j >= 2)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_wk_empty[j & 1], ((j >> 1) - 1) & 1, &abort_flag, p.err));
+          if (!ok) break;
+          widen_tile<D, true>(sK + st * L::kKTileBytes, sKw + (j & 1) * L::kTileBytes, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_wk_full[j & 1]);
+        }
+        if constexpr (kV4) {
+          if (j >= 2)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_wv_empty[j & 1], ((j >> 1) - 1) & 1, &abort_flag, p.err));
+          if (!ok) break;
+          widen_tile<D, true>(sV + st * L::kVTileBytes, sW + (j & 1) * L::kTileBytes, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_wv_full[j & 1]);
+        }
       }
     }
   } else {
@@ -741,8 +844,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 256);
     if (qt2[x] >= 0)
-      tile_rows<D, kSInt8, kPInt8, kV4>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
-                          sKsc, sVsc, qt2[x], nt2[x], x, nt2[1 - x], bh, b, h, warp & 3, lane, &abort_flag);
+      tile_rows<D, kSInt8, kPInt8, kV4, kK4>(p, bars[x], bars[1 - x], tmem + x * 256, tmem + x * 256 + 128, sP + x * kTileM * kTileN,
+                          sKsc, sVsc, qt2[x], nt2[x], x, nt2[1 - x], bh, b, h, warp & 3, lane, &abort_flag,
+                          &bar_q_wide, sQ + x * L::kTileBytes);
   }
 
   tc_fence_before();
@@ -796,14 +900,16 @@ bool make_map_v4(CUtensorMap* m, const void* base, int layout, int B, int H, int
   return encode_map_u8(m, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <int D, bool kSInt8, int kVCode>
+template <int D, int kQKCode, int kVCode>
 cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   CUtensorMap mq, mk, mv;
   const bool v_ok = kVCode == 2 ? make_map_v4(&mv, a.v, a.layout, a.B, a.H, a.Nkv, D)
                                 : make_map(&mv, a.v, a.layout, a.B, a.H, a.Nkv, D);
-  if (!make_map(&mq, a.q, a.layout, a.B, a.H, a.Nq, D) || !make_map(&mk, a.k, a.layout, a.B, a.H, a.Nkv, D) ||
-      !v_ok)
-    return cudaErrorInvalidValue;
+  const bool qk_ok = kQKCode == 2 ? make_map_v4(&mq, a.q, a.layout, a.B, a.H, a.Nq, D) &&
+                                        make_map_v4(&mk, a.k, a.layout, a.B, a.H, a.Nkv, D)
+                                  : make_map(&mq, a.q, a.layout, a.B, a.H, a.Nq, D) &&
+                                        make_map(&mk, a.k, a.layout, a.B, a.H, a.Nkv, D);
+  if (!qk_ok || !v_ok) return cudaErrorInvalidValue;
   PrefillParams p;
   p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
   p.out = static_cast<__nv_bfloat16*>(a.out);
@@ -817,8 +923,8 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   p.layout = a.layout;
   p.scale_log2 = a.scale_log2;
   p.err = err;
-  auto k = prefill_kernel<D, kSInt8, kVCode>;
-  constexpr int kSmem = Smem<D, kVCode>::kBytes;
+  auto k = prefill_kernel<D, kQKCode, kVCode>;
+  constexpr int kSmem = Smem<D, kQKCode, kVCode>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   // The register split inside the kernel needs at least kRegsNeeded
@@ -834,12 +940,14 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
 
 template <int D>
 cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int* err) {
-  if (a.int8) {
-    if (a.v_code == 1) return launch_t<D, true, 1>(a, st, err);
-    if (a.v_code == 0) return launch_t<D, true, 0>(a, st, err);
-    if (a.v_code == 2) return launch_t<D, true, 2>(a, st, err);
-  } else if (a.v_code == 0) {
-    return launch_t<D, false, 0>(a, st, err);
+  if (a.qk_code == 1) {
+    if (a.v_code == 1) return launch_t<D, 1, 1>(a, st, err);
+    if (a.v_code == 0) return launch_t<D, 1, 0>(a, st, err);
+    if (a.v_code == 2) return launch_t<D, 1, 2>(a, st, err);
+  } else if (a.qk_code == 0 && a.v_code == 0) {
+    return launch_t<D, 0, 0>(a, st, err);
+  } else if (a.qk_code == 2 && a.v_code == 2) {
+    return launch_t<D, 2, 2>(a, st, err);
   }
   return cudaErrorInvalidValue;
 }
@@ -848,12 +956,16 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int* err) {
 
 bool prefill_supported(int D) { return D == 64 || D == 128; }
 
-// Q/K INT8 with V e4m3, INT8 or packed INT4; Q/K e4m3 with V e4m3.
-bool prefill_codes_supported(int qk_int8, int v_code) { return qk_int8 ? (v_code >= 0 && v_code <= 2) : v_code == 0; }
+// Q/K INT8 with V e4m3, INT8 or packed INT4; Q/K e4m3 with V e4m3; Q/K/V
+// packed INT4.
+bool prefill_codes_supported(int qk_code, int v_code) {
+  if (qk_code == 1) return v_code >= 0 && v_code <= 2;
+  return qk_code == v_code && (qk_code == 0 || qk_code == 2);
+}
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st, int num_sms, int* err) {
   (void)num_sms;
-  if (!prefill_codes_supported(a.int8, a.v_code)) return cudaErrorInvalidValue;
+  if (!prefill_codes_supported(a.qk_code, a.v_code)) return cudaErrorInvalidValue;
   if (a.D == 128) return launch_d<128>(a, st, err);
   if (a.D == 64) return launch_d<64>(a, st, err);
   return cudaErrorInvalidValue;

@@ -159,7 +159,6 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype, qa
     return QATTN_ERR_INVALID_ARG;
   if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
   if (!rotate_block_quant_supported(D, block_tokens)) return QATTN_ERR_UNSUPPORTED;
-  if (code_dtype == QATTN_INT4_PACKED && rot) return QATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * N == 0) return QATTN_OK;
   if (!x || !codes || !scales) return QATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes) || (rot && !aligned16(rot))) return QATTN_ERR_ALIGNMENT;
@@ -185,13 +184,15 @@ qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, c
                                    int H, int N_q, int N_kv, int D, int q_block, int kv_block, int causal,
                                    float softmax_scale, void* out, float* lse, qattn_stream_t stream) {
   if (B < 0 || H < 0 || N_q < 0 || N_kv < 0 || D <= 0) return QATTN_ERR_INVALID_ARG;
-  if (qk_dtype != QATTN_INT8 && qk_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (qk_dtype != QATTN_INT8 && qk_dtype != QATTN_FP8_E4M3 && qk_dtype != QATTN_INT4_PACKED)
+    return QATTN_ERR_INVALID_ARG;
   if (v_dtype != QATTN_INT8 && v_dtype != QATTN_FP8_E4M3 && v_dtype != QATTN_INT4_PACKED)
     return QATTN_ERR_INVALID_ARG;
   if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return QATTN_ERR_INVALID_ARG;
   const int v_code = v_dtype == QATTN_FP8_E4M3 ? 0 : v_dtype == QATTN_INT8 ? 1 : 2;
-  if (!prefill_codes_supported(qk_dtype == QATTN_INT8, v_code)) return QATTN_ERR_UNSUPPORTED;
+  const int qk_code = qk_dtype == QATTN_FP8_E4M3 ? 0 : qk_dtype == QATTN_INT8 ? 1 : 2;
+  if (!prefill_codes_supported(qk_code, v_code)) return QATTN_ERR_UNSUPPORTED;
   if (causal && N_q != N_kv) return QATTN_ERR_UNSUPPORTED;
   if (q_block != 128 || kv_block != 256) return QATTN_ERR_UNSUPPORTED;
   if (!prefill_supported(D)) return QATTN_ERR_UNSUPPORTED;
@@ -209,7 +210,7 @@ qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, c
   a.q = q_codes; a.qs = q_scales;
   a.k = k_codes; a.ks = k_scales;
   a.v = v_codes; a.vs = v_scales;
-  a.int8 = qk_dtype == QATTN_INT8;
+  a.qk_code = qk_code;
   a.v_code = v_code;
   a.layout = layout;
   a.B = B; a.H = H; a.Nq = N_q; a.Nkv = N_kv; a.D = D;

@@ -25,7 +25,7 @@ struct RotQuantArgs {
   int B, H, N, D, T;  // T = block tokens
   const float* rot;   // D x D or nullptr
   int int8;           // 1: INT8 codes, 0: e4m3
-  int int4;           // 1: packed INT4 codes (with int8 = 1; no rotation)
+  int int4;           // 1: packed INT4 codes (with int8 = 1)
   void* codes;
   float* scales;
 };
@@ -41,8 +41,8 @@ struct PrefillArgs {
   const float* ks;
   const void* v;
   const float* vs;
-  int int8;           // Q/K codes: 1 INT8, 0 e4m3
-  int v_code;         // V codes: 0 e4m3, 1 INT8, 2 packed INT4 (two per byte)
+  int qk_code;        // Q/K codes: 0 e4m3, 1 INT8, 2 packed INT4 (two per byte)
+  int v_code;         // V codes: 0 e4m3, 1 INT8, 2 packed INT4
   int layout;
   int B, H, Nq, Nkv, D;
   int causal;
@@ -52,7 +52,7 @@ struct PrefillArgs {
 };
 
 bool prefill_supported(int D);
-bool prefill_codes_supported(int qk_int8, int v_code);
+bool prefill_codes_supported(int qk_code, int v_code);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st, int num_sms, int* err);
 
 struct DecodeArgs {

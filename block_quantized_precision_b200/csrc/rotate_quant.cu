@@ -158,8 +158,13 @@ __device__ __forceinline__ bool codes8_fast(const float (&f)[8], float rcp, uint
       ok = ok && fabsf(v0 - (m - 12582912.0f)) <= 0.4999f;
       t[e] = __float_as_uint(m);
     }
-    lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-    hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    if constexpr (kInt4) {
+      lo = pack_nibbles8(t);
+      hi = 0;
+    } else {
+      lo = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+      hi = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
+    }
     return ok;
   } else if constexpr (kInt8) {
     const float2 rc = make_float2(rcp, rcp);
@@ -263,8 +268,14 @@ struct F8 {
 
 // Codes of 8 values with the IEEE quotient for every value, packed like
 // codes8_fast.
-template <bool kInt8>
+template <bool kInt8, bool kInt4 = false>
 __device__ __noinline__ uint2 codes8_exact_f(F8 f, float scale) {
+  if constexpr (kInt4) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w |= code_exact<true, true>(f.v[e], scale) << (4 * e);
+    return make_uint2(w, 0);
+  }
   uint32_t lo = 0, hi = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) lo |= code_of<kInt8>(f.v[j], scale, 0.0f, true) << (8 * j);
@@ -281,7 +292,8 @@ __device__ __noinline__ uint2 codes8_exact_f(F8 f, float scale) {
 // owns columns 4cg..4cg+3 and D/2+4cg..D/2+4cg+3 (two float4 of each R row,
 // consecutive across the warp, so the R reads are free of bank conflicts);
 // row group rg = tid / (D/8) owns rows rg*kRPT .. rg*kRPT + kRPT - 1.
-template <int D, int T, bool kInt8>
+// kInt4 (with kInt8): INT4 codes (scale absmax / 7), two per byte.
+template <int D, int T, bool kInt8, bool kInt4>
 __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
     rotq_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
                 const float* __restrict__ rot, uint8_t* __restrict__ codes,
@@ -305,7 +317,7 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
   const int64_t total = static_cast<int64_t>(B) * H * nblk;
   const int cg = tid % kCG, rg = tid / kCG;
   const int c0 = 4 * cg, c1 = D / 2 + 4 * cg;   // this thread's two column quads
-  const float qmax = kInt8 ? 127.0f : 448.0f;
+  const float qmax = kInt4 ? 7.0f : kInt8 ? 127.0f : 448.0f;
 
   // Raw 16-byte input vectors of the next block, loaded into registers while
   // the current block is being computed (thread t: token row idx % T and
@@ -404,7 +416,7 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
     for (int i = 0; i < kRPT; ++i) {
       const float f[8] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
                           acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y};
-      fix |= codes8_fast<kInt8, false>(f, rcp, w[i].x, w[i].y) ? 0u : 1u << i;
+      fix |= codes8_fast<kInt8, false, kInt4>(f, rcp, w[i].x, w[i].y) ? 0u : 1u << i;
     }
     if (scale == 0.0f) {                              // all-zero block: zero codes
       fix = 0;
@@ -413,13 +425,23 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
     } else if (slow) {
       fix = (1u << kRPT) - 1;
     }
-    uint8_t* crow0 = codes + row_offset(layout, H, N, D, b, h, n0 + rg * kRPT);
-    const int64_t rstride = layout == 0 ? D : static_cast<int64_t>(H) * D;   // between token rows
+    // (INT4: byte offsets halved; columns c0.. and c1.. are 2 bytes each)
+    constexpr int kDiv = kInt4 ? 2 : 1;
+    uint8_t* crow0 = codes + row_offset(layout, H, N, D, b, h, n0 + rg * kRPT) / kDiv;
+    const int64_t rstride = (layout == 0 ? D : static_cast<int64_t>(H) * D) / kDiv;   // between token rows
+    auto store = [&](int i, uint2 w2) {
+      if constexpr (kInt4) {
+        *reinterpret_cast<uint16_t*>(crow0 + i * rstride + c0 / 2) = static_cast<uint16_t>(w2.x & 0xFFFFu);
+        *reinterpret_cast<uint16_t*>(crow0 + i * rstride + c1 / 2) = static_cast<uint16_t>(w2.x >> 16);
+      } else {
+        *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c0) = w2.x;
+        *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c1) = w2.y;
+      }
+    };
 #pragma unroll
     for (int i = 0; i < kRPT; ++i) {
       if (((fix >> i) & 1u) || rg * kRPT + i >= rows) continue;
-      *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c0) = w[i].x;
-      *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c1) = w[i].y;
+      store(i, w[i]);
     }
     if (fix != 0) {
 #pragma unroll
@@ -427,9 +449,7 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
         if (!((fix >> i) & 1u) || rg * kRPT + i >= rows) continue;
         const F8 f = {{acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
                        acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y}};
-        const uint2 we = codes8_exact_f<kInt8>(f, scale);
-        *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c0) = we.x;
-        *reinterpret_cast<uint32_t*>(crow0 + i * rstride + c1) = we.y;
+        store(i, codes8_exact_f<kInt8, kInt4>(f, scale));
       }
     }
   }
@@ -613,10 +633,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
   }
 }
 
-template <int D, int T, bool kInt8>
+template <int D, int T, bool kInt8, bool kInt4 = false>
 cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
   constexpr size_t smem = sizeof(float) * (D * D + D * (T + 4));
-  auto k = rotq_kernel<D, T, kInt8>;
+  auto k = rotq_kernel<D, T, kInt8, kInt4>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
@@ -663,7 +683,10 @@ cudaError_t launch_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, in
 
 template <int D, int T>
 cudaError_t dispatch_t(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err) {
-  if (a.rot) return a.int8 ? launch_rotq<D, T, true>(a, st, num_sms) : launch_rotq<D, T, false>(a, st, num_sms);
+  if (a.rot) {
+    if (a.int4) return launch_rotq<D, T, true, true>(a, st, num_sms);
+    return a.int8 ? launch_rotq<D, T, true>(a, st, num_sms) : launch_rotq<D, T, false>(a, st, num_sms);
+  }
   return a.int8 ? launch_quant<D, T, true>(a, st, num_sms, err) : launch_quant<D, T, false>(a, st, num_sms, err);
 }
 

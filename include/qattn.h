@@ -105,8 +105,7 @@ const char* qattn_status_string(qattn_status_t status);
  *               [B,H,N,D] or [B,N,H,D].
  * rot:          D x D float32 row-major (rot[k*D + j] = R[k][j]), or NULL.
  * block_tokens: tokens per block: 128 (Q) or 256 (K/V).
- * code_dtype:   QATTN_INT8, QATTN_FP8_E4M3, or QATTN_INT4_PACKED (no
- *               rotation: rot must be NULL, else QATTN_ERR_UNSUPPORTED):
+ * code_dtype:   QATTN_INT8, QATTN_FP8_E4M3, or QATTN_INT4_PACKED:
  *               scale = max|x| / 7, codes RNE(x / scale) clamped to [-7, 7]
  *               ("FlashAttention 的 INT8/INT4 量化", 第二层, with the block
  *               scales above), two per byte, element 2i in the low nibble
@@ -166,11 +165,14 @@ qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const v
  * 第二层 (INT4 codes widened to INT8 for the matmul).
  *
  * Same computation and arguments as qattn_prefill, with:
- *   qk_dtype: QATTN_INT8 or QATTN_FP8_E4M3 (Q and K codes);
- *   v_dtype:  QATTN_INT8, QATTN_FP8_E4M3 or QATTN_INT4_PACKED (V codes,
- *             [B,H,N_kv,D/2] or [B,N_kv,H,D/2] bytes for INT4, as written by
- *             qattn_rotate_block_quant). Supported pairs: INT8 Q/K with any V;
- *             e4m3 Q/K with e4m3 V (else QATTN_ERR_UNSUPPORTED).
+ *   qk_dtype: QATTN_INT8, QATTN_FP8_E4M3 or QATTN_INT4_PACKED (Q and K);
+ *   v_dtype:  QATTN_INT8, QATTN_FP8_E4M3 or QATTN_INT4_PACKED (V codes;
+ *             packed INT4 tensors are [B,H,N,D/2] or [B,N,H,D/2] bytes, as
+ *             written by qattn_rotate_block_quant). Supported pairs: INT8 Q/K
+ *             with any V; e4m3 Q/K with e4m3 V; INT4 Q/K with INT4 V
+ *             ("FlashAttention 的 INT8/INT4 量化", 第二层: every INT4 operand
+ *             widened to INT8 for the matmul; the scores are exact integers).
+ *             Other pairs: QATTN_ERR_UNSUPPORTED.
  *   P is rounded to INT8 codes (round(127 p) / 127) when V is INT8 or INT4
  *   (INT4 V is widened to INT8 on chip) and to e4m3 when V is e4m3.
  * v_scales: float32 [B, H, ceil(N_kv / kv_block)] for every V type.

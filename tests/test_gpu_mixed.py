@@ -117,3 +117,82 @@ def test_mixed_int4_full_size(orc):
     heads = [(0, int(h)) for h in rng.choice(p.H, 3, replace=False)]
     rows = sorted(set(rng.choice(p.N, 96, replace=False).tolist()) | {0, 127, 128, p.N - 1})
     _mixed(orc, p, d, synth.INT4_PACKED, {hd: rows for hd in heads})
+
+
+@pytest.mark.parametrize("layout", [synth.BNSD, synth.BSND])
+@pytest.mark.parametrize("D,block", [(64, 128), (128, 128), (128, 256)])
+def test_int4_rotated_block_quant_bit_exact(orc, layout, D, block):
+    """Rotation + INT4 codes (the float32 FMA chain of the rotation decides
+    the codes as for INT8)."""
+    N = 300
+    rng = np.random.default_rng(D + block + 11 * layout)
+    shape = (1, 3, N, D) if layout == synth.BNSD else (1, N, 3, D)
+    bits = synth.f32_to_bf16_bits(rng.standard_normal(shape))
+    R = synth.haar_orthogonal(3, 1, D)
+    codes, scales = qa.qattn_rotate_block_quant(dev_bits(bits, synth.BF16), layout, dev(R), block,
+                                                qa.QATTN_INT4_PACKED)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    oc, osc = orc.rotate_block_quant(bits, synth.BF16, layout, R, block, synth.INT4_PACKED)
+    assert np.array_equal(codes.cpu().numpy(), oc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), osc.view(np.uint32))
+
+
+def _int4_all(orc, p, d, rows_by_head, check_codes=True):
+    rot = dev(d["rot"])
+    c = {}
+    for nm, blk, r in (("q", 128, rot), ("k", 256, rot), ("v", 256, None)):
+        c[nm] = qa.qattn_rotate_block_quant(dev_bits(d[nm], p.in_dtype), p.layout, r, blk, qa.QATTN_INT4_PACKED)
+    lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device="cuda")
+    out = qa.qattn_prefill_mixed(*c["q"], *c["k"], *c["v"], qa.QATTN_INT4_PACKED, qa.QATTN_INT4_PACKED, p.layout,
+                                 p.causal, lse=lse)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    assert out.shape == tuple(p.shape())
+    heads = sorted(rows_by_head)
+    o = {nm: orc.rotate_block_quant(d[nm], p.in_dtype, p.layout, d["rot"] if nm != "v" else None,
+                                    128 if nm == "q" else 256, synth.INT4_PACKED, heads=heads) for nm in "qkv"}
+    if check_codes:
+        for nm in "qkv":
+            gcodes, gsc = c[nm][0].cpu().numpy(), c[nm][1].cpu().numpy()
+            for (b, h) in heads:
+                assert np.array_equal(head_rows(gcodes, p.layout, b, h), head_rows(o[nm][0], p.layout, b, h))
+                assert np.array_equal(gsc[b, h], o[nm][1][b, h])
+    ref = orc.prefill_rows(*o["q"], *o["k"], *o["v"], synth.INT4_PACKED, p.layout, p.causal, rows_by_head,
+                           want_lse=True)
+    out_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    lse_np = lse.cpu().numpy()
+    for (b, h), rows in rows_by_head.items():
+        got = bf16_to_f64(head_rows(out_bits, p.layout, b, h)[rows])
+        vmax = dequant_v_max(o["v"][0], o["v"][1], synth.INT4_PACKED, p.layout, b, h, orc)
+        assert_close(got, bf16_to_f64(ref[(b, h)][0]), vmax, "head (%d,%d)" % (b, h))
+        assert np.abs(lse_np[b, h, rows] - ref[(b, h)][2]).max() < 1e-2
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("layout", [synth.BNSD, synth.BSND])
+@pytest.mark.parametrize("causal", [False, True])
+def test_int4_qkv_small_shapes(orc, D, layout, causal):
+    p = synth.PrefillProblem("int4", 2, 3, 300, D, synth.BF16, synth.INT8, layout, causal=causal, rotate=True,
+                             seed=600 + D + 3 * layout + 5 * causal)
+    d = synth.make_prefill(p)
+    _int4_all(orc, p, d, {(b, h): list(range(p.N)) for b in range(p.B) for h in range(p.H)})
+
+
+@pytest.mark.parametrize("N", [1, 129, 640])
+def test_int4_qkv_sequence_lengths(orc, N):
+    p = synth.PrefillProblem("len4", 1, 2, N, 128, synth.BF16, synth.INT8, synth.BNSD, causal=True, rotate=True,
+                             seed=700 + N, outlier_frac=0.01)
+    d = synth.make_prefill(p)
+    _int4_all(orc, p, d, {(0, h): list(range(N)) for h in range(2)})
+
+
+def test_int4_qkv_full_size(orc):
+    """The INT8 causal problem (B1 H32 N4096 D128) with Q, K and V in packed
+    INT4; sampled rows of sampled heads."""
+    p = synth.INT8_CAUSAL
+    d = synth.make_prefill(p)
+    rng = np.random.default_rng(1)
+    heads = [(0, int(h)) for h in rng.choice(p.H, 3, replace=False)]
+    rows = sorted(set(rng.choice(p.N, 96, replace=False).tolist()) | {0, 127, 128, p.N - 1})
+    _int4_all(orc, p, d, {hd: rows for hd in heads})
