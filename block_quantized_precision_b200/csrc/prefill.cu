@@ -661,19 +661,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int x = 0; x < 2; ++x)
         if (qt2[x] >= 0) tma_load_4d(qdst + x * L::kQTileBytes, &tmQ, &bar_q_full, 0, qt2[x] * kTileM, h, b);
     }
-    int j = 0;
-    for (; j < nt_max; ++j) {
-      const int st = j % kStagesKV;
-      if (j >= kStagesKV) {
-        const bool ok = mbar_wait(&bar_kv_empty[st], ((j / kStagesKV) - 1) & 1, &abort_flag, p.err);
-        if (!__all_sync(0xffffffffu, ok)) break;
+    // K/V tile j into stage j % 3 (after both tiles' P.V(j - 3) released it).
+    auto load = [&](int jj) -> bool {
+      const int st = jj % kStagesKV;
+      if (jj >= kStagesKV) {
+        const bool ok = mbar_wait(&bar_kv_empty[st], ((jj / kStagesKV) - 1) & 1, &abort_flag, p.err);
+        if (!__all_sync(0xffffffffu, ok)) return false;
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar_kv_full[st], L::kKTileBytes + L::kVTileBytes);
-        tma_load_4d(sK + st * L::kKTileBytes, &tmK, &bar_kv_full[st], 0, j * kTileN, h, b);
-        tma_load_4d(sV + st * L::kVTileBytes, &tmV, &bar_kv_full[st], 0, j * kTileN, h, b);
+        tma_load_4d(sK + st * L::kKTileBytes, &tmK, &bar_kv_full[st], 0, jj * kTileN, h, b);
+        tma_load_4d(sV + st * L::kVTileBytes, &tmV, &bar_kv_full[st], 0, jj * kTileN, h, b);
       }
       __syncwarp();
+      return true;
+    };
+    // INT4 K: this warp also widens each K tile (warp 3 has Q and V), K(jj)
+    // into sKw[jj & 1] once it has landed and both tiles' S(jj - 2) read the
+    // buffer. K(j + 1) is widened before the wait that frees stage j, so the
+    // scores never wait on a P.V product.
+    auto widen_k = [&](int jj) -> bool {
+      bool ok = mbar_wait(&bar_kv_full[jj % kStagesKV], (jj / kStagesKV) & 1, &abort_flag, p.err);
+      if (ok && jj >= 2) ok = mbar_wait(&bar_wk_empty[jj & 1], ((jj >> 1) - 1) & 1, &abort_flag, p.err);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      widen_tile<D, true>(sK + (jj % kStagesKV) * L::kKTileBytes, sKw + (jj & 1) * L::kTileBytes, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_wk_full[jj & 1]);
+      return true;
+    };
+    int j = 0;                                         // K/V tiles loaded so far
+    if constexpr (kK4) {
+      bool ok = true;
+      for (; ok && j < min(nt_max, kStagesKV); ++j) ok = load(j);
+      if (ok && nt_max > 0) ok = widen_k(0);
+      for (int jw = 0; ok && jw < nt_max; ++jw) {
+        if (jw + 1 < nt_max) ok = widen_k(jw + 1);
+        if (ok && j < nt_max) {
+          ok = load(j);
+          if (ok) ++j;
+        }
+      }
+    } else {
+      // (this form of the loop measured faster than calling load())
+      for (; j < nt_max; ++j) {
+        const int st = j % kStagesKV;
+        if (j >= kStagesKV) {
+          const bool ok = mbar_wait(&bar_kv_empty[st], ((j / kStagesKV) - 1) & 1, &abort_flag, p.err);
+          if (!__all_sync(0xffffffffu, ok)) break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar_kv_full[st], L::kKTileBytes + L::kVTileBytes);
+          tma_load_4d(sK + st * L::kKTileBytes, &tmK, &bar_kv_full[st], 0, j * kTileN, h, b);
+          tma_load_4d(sV + st * L::kVTileBytes, &tmV, &bar_kv_full[st], 0, j * kTileN, h, b);
+        }
+        __syncwarp();
+      }
     }
     if (abort_flag && lane == 0) {
       // Let issued copies land before the CTA can exit (bounded).
@@ -794,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ INT4 widening
       // Packed tiles -> 8-bit codes laid out as TMA loads of 8-bit codes
       // would leave them: the two Q tiles once (signed), then per key tile j
-      // K(j) into sKw[j & 1] and V(j) into sW[j & 1] (code + 8, unsigned).
+      // V(j) into sW[j & 1] (code + 8, unsigned). (Warp 0 widens K.)
       bool ok = true;
       if constexpr (kK4) {
         ok = __all_sync(0xffffffffu, mbar_wait(&bar_q_full, 0, &abort_flag, p.err));
@@ -810,15 +853,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = j % kStagesKV;
         ok = __all_sync(0xffffffffu, mbar_wait(&bar_kv_full[st], (j / kStagesKV) & 1, &abort_flag, p.err));
         if (!ok) break;
-        if constexpr (kK4) {
-          if (j >= 2)
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar_wk_empty[j & 1], ((j >> 1) - 1) & 1, &abort_flag, p.err));
-          if (!ok) break;
-          widen_tile<D, true>(sK + st * L::kKTileBytes, sKw + (j & 1) * L::kTileBytes, lane);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar_wk_full[j & 1]);
-        }
         if constexpr (kV4) {
           if (j >= 2)
             ok = __all_sync(0xffffffffu, mbar_wait(&bar_wv_empty[j & 1], ((j >> 1) - 1) & 1, &abort_flag, p.err));
