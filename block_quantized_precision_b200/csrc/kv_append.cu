@@ -15,7 +15,7 @@
 //     each code as the IEEE quotient decides it (code_fast), clamped to
 //     [-127, 127].
 // Packed INT4 cache, one fp16 scale per token per group:
-//   kv_append_int4_kernel: one warp per 4 new tokens; lane l owns channels
+//   kv_append_int4_kernel: one warp per 4 new tokens of one (b, h_kv); lane l owns channels
 //     4l..4l+3. s16 = fp16(absmax_group / 7), codes RNE(x / s16) clamped to
 //     [-7, 7], packed two per byte.
 // Both are small, memory-bound kernels (the new rows are read once, the
@@ -66,14 +66,23 @@ __global__ void __launch_bounds__(kAppendThreads)
   const int64_t total = static_cast<int64_t>(t1 - t0) * vecs;
   const uint16_t* xb = x + (head * n + (t0 - L)) * D;
 
-  float m = 0.0f;
-  for (int64_t i = threadIdx.x; i < total; i += kAppendThreads) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xb + i * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // Four vectors per thread in flight at a time; |x| of bf16 values orders
+  // like the bits with the sign cleared.
+  uint32_t mb = 0;
+  for (int64_t i0 = threadIdx.x; i0 < total; i0 += 4 * kAppendThreads) {
+    uint4 v[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[k] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[k] >> 16))));
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * kAppendThreads;
+      v[u] = i < total ? *reinterpret_cast<const uint4*>(xb + i * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      mb = __vmaxu2(mb, __vmaxu2(v[u].x & 0x7FFF7FFFu, v[u].y & 0x7FFF7FFFu));
+      mb = __vmaxu2(mb, __vmaxu2(v[u].z & 0x7FFF7FFFu, v[u].w & 0x7FFF7FFFu));
+    }
   }
+  float m = bf16_bits_to_f32(max(mb & 0xFFFFu, mb >> 16));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -106,21 +115,31 @@ __global__ void __launch_bounds__(kAppendThreads)
       *reinterpret_cast<uint2*>(cb + i * 8) = make_uint2(o[0], o[1]);
     }
   }
-  // new tokens
+  // new tokens (four vectors in flight at a time)
   int8_t* cn = cache + (head * Lmax + t0) * D;
-  for (int64_t i = threadIdx.x; i < total; i += kAppendThreads) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xb + i * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[2] = {0, 0};
-    if (s != 0.0f) {
+  for (int64_t i0 = threadIdx.x; i0 < total; i0 += 4 * kAppendThreads) {
+    uint4 vv[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] & 0xFFFFu), s, rcp, slow, 127)) & 0xFFu;
-        const uint32_t hi = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] >> 16), s, rcp, slow, 127)) & 0xFFu;
-        o[k >> 1] |= (lo | (hi << 8)) << (16 * (k & 1));
-      }
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * kAppendThreads;
+      vv[u] = i < total ? *reinterpret_cast<const uint4*>(xb + i * 8) : make_uint4(0, 0, 0, 0);
     }
-    *reinterpret_cast<uint2*>(cn + i * 8) = make_uint2(o[0], o[1]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * kAppendThreads;
+      if (i >= total) break;
+      const uint32_t w[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+      uint32_t o[2] = {0, 0};
+      if (s != 0.0f) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t lo = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] & 0xFFFFu), s, rcp, slow, 127)) & 0xFFu;
+          const uint32_t hi = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] >> 16), s, rcp, slow, 127)) & 0xFFu;
+          o[k >> 1] |= (lo | (hi << 8)) << (16 * (k & 1));
+        }
+      }
+      *reinterpret_cast<uint2*>(cn + i * 8) = make_uint2(o[0], o[1]);
+    }
   }
   if (threadIdx.x == 0) scales[head * nblk + blk] = s;
 }
@@ -130,24 +149,25 @@ __global__ void __launch_bounds__(kAppendThreads)
 // 64 (all lanes or one half-warp per group).
 constexpr int kInt4RowsPerWarp = 4;
 
+// Grid (ceil(n / rows per CTA), B * H_kv): blockIdx.y is the (b, h_kv) head.
 __global__ void __launch_bounds__(kAppendThreads)
-    kv_append_int4_kernel(const uint16_t* __restrict__ x, int B, int Hkv, int n, int L, int Lmax, int group,
+    kv_append_int4_kernel(const uint16_t* __restrict__ x, int n, int L, int Lmax, int group,
                           uint8_t* __restrict__ cache, uint16_t* __restrict__ scales) {
   constexpr int D = 128;
   const int lane = threadIdx.x & 31;
-  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * (kAppendThreads / 32) + (threadIdx.x >> 5)) * kInt4RowsPerWarp;
-  const int64_t rows = static_cast<int64_t>(B) * Hkv * n;
+  const int64_t head = blockIdx.y;
+  const int r0 = (static_cast<int>(blockIdx.x) * (kAppendThreads / 32) + (threadIdx.x >> 5)) * kInt4RowsPerWarp;
+  const uint16_t* xh = x + head * n * D;
   // the warp's rows are loaded first (in flight together), then coded
   uint2 raw[kInt4RowsPerWarp];
 #pragma unroll
   for (int i = 0; i < kInt4RowsPerWarp; ++i)
-    raw[i] = row0 + i < rows ? *reinterpret_cast<const uint2*>(x + (row0 + i) * D + lane * 4) : make_uint2(0, 0);
+    raw[i] = r0 + i < n ? *reinterpret_cast<const uint2*>(xh + static_cast<int64_t>(r0 + i) * D + lane * 4)
+                        : make_uint2(0, 0);
 #pragma unroll
   for (int i = 0; i < kInt4RowsPerWarp; ++i) {
-    const int64_t row = row0 + i;
-    if (row >= rows) break;                             // (uniform per warp)
-    const int64_t head = row / n;
-    const int t = L + static_cast<int>(row % n);
+    if (r0 + i >= n) break;                             // (uniform per warp)
+    const int t = L + r0 + i;
     const float f[4] = {bf16_bits_to_f32(raw[i].x & 0xFFFFu), bf16_bits_to_f32(raw[i].x >> 16),
                         bf16_bits_to_f32(raw[i].y & 0xFFFFu), bf16_bits_to_f32(raw[i].y >> 16)};
     float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
@@ -189,12 +209,11 @@ cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st) {
                                                             a.Lmax, a.kv_block, static_cast<int8_t*>(a.cache),
                                                             static_cast<float*>(a.scales));
   } else {
-    const int64_t rows = static_cast<int64_t>(a.B) * a.Hkv * a.n;
-    const int64_t per_cta = static_cast<int64_t>(kAppendThreads / 32) * kInt4RowsPerWarp;
-    const int64_t ctas = (rows + per_cta - 1) / per_cta;
-    kv_append_int4_kernel<<<static_cast<unsigned>(ctas), kAppendThreads, 0, st>>>(
-        static_cast<const uint16_t*>(a.x), a.B, a.Hkv, a.n, a.L, a.Lmax, a.group, static_cast<uint8_t*>(a.cache),
-        static_cast<uint16_t*>(a.scales));
+    const int per_cta = (kAppendThreads / 32) * kInt4RowsPerWarp;
+    const dim3 grid(static_cast<unsigned>((a.n + per_cta - 1) / per_cta), static_cast<unsigned>(a.B * a.Hkv));
+    kv_append_int4_kernel<<<grid, kAppendThreads, 0, st>>>(static_cast<const uint16_t*>(a.x), a.n, a.L, a.Lmax,
+                                                           a.group, static_cast<uint8_t*>(a.cache),
+                                                           static_cast<uint16_t*>(a.scales));
   }
   return cudaGetLastError();
 }

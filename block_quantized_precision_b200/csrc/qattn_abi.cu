@@ -292,6 +292,7 @@ qattn_status_t qattn_kv_append(const void* x_new, int B, int H_kv, int n, int D,
   if (!x_new || !cache || !scales) return QATTN_ERR_INVALID_ARG;
   if (!aligned16(x_new) || !aligned16(cache)) return QATTN_ERR_ALIGNMENT;
   if (static_cast<int64_t>(B) * H_kv * n >= (1LL << 31) * 8) return QATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || H_kv > 65535 || (int4 && static_cast<int64_t>(B) * H_kv > 65535)) return QATTN_ERR_UNSUPPORTED;
   DeviceState* ds = nullptr;
   qattn_status_t s = device_state(&ds);
   if (s != QATTN_OK) return s;

@@ -286,7 +286,8 @@ qattn_status_t qattn_decode_kvq_noalloc(const void* q, const void* k_cache, cons
  * cache and scales are updated in place on `stream`; rows outside
  * [L, L + n) are not written except the earlier rows of a growing INT8
  * block. Errors: QATTN_ERR_INVALID_ARG (ranges, null pointers),
- * QATTN_ERR_UNSUPPORTED (D, kv_block, group), QATTN_ERR_ALIGNMENT; nothing
+ * QATTN_ERR_UNSUPPORTED (D, kv_block, group; B or H_kv above 65535, or
+ * B * H_kv above 65535 for INT4), QATTN_ERR_ALIGNMENT; nothing
  * is launched on error. n == 0 returns QATTN_OK without a launch.
  */
 qattn_status_t qattn_kv_append(const void* x_new, int B, int H_kv, int n, int D,
