@@ -64,7 +64,7 @@ constexpr int kStep = 16;             // tokens per consumer step
 constexpr int kWsStride = kD + 4;     // floats per (b, h_q, split) partial: O[D], m, l, pad
 constexpr int kPStride = 20;          // floats per head row of the per-warp P' buffer
 constexpr uint32_t kOnesF16x2 = 0x3C003C00u;
-constexpr int kCtasPerSm = 2;         // resident CTAs per SM (registers)
+constexpr int kCtasPerSm = 3;         // resident CTAs per SM (registers)
 
 template <bool kInt4>
 struct Cfg {
@@ -379,9 +379,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const int ra = r0 + gq, rb = r0 + gq + 8;             // this lane's score rows (tokens)
       const bool va = chunk_t0 + ra < t_end, vb = chunk_t0 + rb < t_end;
       // ---------------- scores: S^T = K Q^T ----------------
-      int sc[kNAcc][4];
+      // one accumulator per 32-channel slice, so that the four MMAs do not
+      // wait on one another; the slices are then added (exact in INT32)
+      int sck[4][4];
 #pragma unroll
-      for (int a = 0; a < kNAcc; ++a) sc[a][0] = sc[a][1] = sc[a][2] = sc[a][3] = 0;
+      for (int a = 0; a < 4; ++a) sck[a][0] = sck[a][1] = sck[a][2] = sck[a][3] = 0;
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
         if constexpr (!kInt4) {
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const int off = ((ch ^ gq) << 4) + (cq & 1) * 8;
           const uint2 xa = *reinterpret_cast<const uint2*>(cK + ra * 128 + off);
           const uint2 xb = *reinterpret_cast<const uint2*>(cK + rb * 128 + off);
-          mma_s8(sc[0], xa.x, xb.x, xa.y, xb.y, qb0[kb], qb1[kb]);
+          mma_s8(sck[kb], xa.x, xb.x, xa.y, xb.y, qb0[kb], qb1[kb]);
         } else {
           // 4 bytes (8 nibbles) of rows ra / rb at channel kb*32 + 8*cq:
           // 16-byte chunk kb, stored at kb ^ ((row / 2) % 4)
@@ -401,7 +403,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           // nibble c -> byte c + 8 (even channels, odd channels)
           const uint32_t ea = (wa & 0x0F0F0F0Fu) ^ 0x08080808u, oa = ((wa >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
           const uint32_t eb = (wb & 0x0F0F0F0Fu) ^ 0x08080808u, ob = ((wb >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-          mma_s8(sc[kNAcc == 2 ? (kb >> 1) : 0], ea, eb, oa, ob, qb0[kb], qb1[kb]);
+          mma_s8(sck[kb], ea, eb, oa, ob, qb0[kb], qb1[kb]);
+        }
+      }
+      int sc[kNAcc][4];                                    // per INT4 group (else all 128 channels)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if constexpr (kNAcc == 2) {
+          sc[0][e] = sck[0][e] + sck[1][e];
+          sc[kNAcc - 1][e] = sck[2][e] + sck[3][e];
+        } else {
+          sc[0][e] = (sck[0][e] + sck[1][e]) + (sck[2][e] + sck[3][e]);
         }
       }
       // accumulator layout: [0] = (ra, h0), [1] = (ra, h1), [2] = (rb, h0), [3] = (rb, h1)
