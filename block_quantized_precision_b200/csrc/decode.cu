@@ -124,6 +124,10 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
 }
 
 // Two fp16 parts of (x, y): high = RN_f16(x, y), low = RN_f16((x, y) - high).
+// Exact int -> float for |x| < 2^22 on the integer pipe: the float with
+// bits 0x4B400000 + x is 1.5 * 2^23 + x, and the subtraction is exact.
+__device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(x + 0x4B400000) - 12582912.0f; }
+
 __device__ __forceinline__ void split_f16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
   const __half2 h = __floats2half2_rn(x, y);
   const float2 f = __half22float2(h);
@@ -158,8 +162,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // warp on distinct banks
   __shared__ __align__(16) float sPw[kConsumers][kGroups][8][kPStride];
   __shared__ float sKsc[kStages], sVsc[kStages], sVmax[kStages];
-  __shared__ uint16_t sKs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
-  __shared__ uint16_t sVs16[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
+  // INT4 group scales of the chunk as float [token][group]: K as stored, V
+  // already divided by the running max V scale (sVmax)
+  __shared__ __align__(8) float sKsf[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
+  __shared__ __align__(8) float sVsf[kInt4 ? kStages : 1][kInt4 ? C::kChunk * kGroups : 1];
   __shared__ float sWm[kConsumers][8], sWl[kConsumers][8];
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
   __shared__ int abort_flag;
@@ -241,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
     };
     if (nchunks > 0) load_scales(0);
+    float vrun = 0.0f;                 // running max V scale over the chunks staged so far
     int c = 0;
     for (; c < nchunks; ++c) {
       const int s = c % kStages;
@@ -254,24 +261,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tma_load_3d(sK + s * kTile, &tmK, &full[s], 0, t0, static_cast<int>(head));
         tma_load_3d(sV + s * kTile, &tmV, &full[s], 0, t0, static_cast<int>(head));
       }
+      // The consumers weight P by v scale / running max v scale; the running
+      // max (sVmax) and the weights are formed here, once per chunk.
       if constexpr (!kInt4) {
+        vrun = fmaxf(vrun, fabsf(vsc));
+        const float inv = vrun > 0.0f ? 1.0f / vrun : 0.0f;
         if (lane == 0) {
           sKsc[s] = ksc;
-          sVsc[s] = vsc;
-          sVmax[s] = fabsf(vsc);
+          sVsc[s] = vsc * inv;
+          sVmax[s] = vrun;
         }
       } else {
         // largest V scale of the chunk (non-negative fp16 values order as
         // their bit patterns; the sign bit is cleared)
         uint32_t vm = 0;
 #pragma unroll
-        for (int j = 0; j < kScalePerLane; ++j) {
-          sKs16[s][lane + 32 * j] = ksv[j];
-          sVs16[s][lane + 32 * j] = vsv[j];
-          vm = max(vm, static_cast<uint32_t>(vsv[j] & 0x7FFFu));
-        }
+        for (int j = 0; j < kScalePerLane; ++j) vm = max(vm, static_cast<uint32_t>(vsv[j] & 0x7FFFu));
         vm = __reduce_max_sync(0xffffffffu, vm);
-        if (lane == 0) sVmax[s] = __half2float(__ushort_as_half(static_cast<unsigned short>(vm)));
+        vrun = fmaxf(vrun, __half2float(__ushort_as_half(static_cast<unsigned short>(vm))));
+        const float inv = vrun > 0.0f ? 1.0f / vrun : 0.0f;
+#pragma unroll
+        for (int j = 0; j < kScalePerLane; ++j) {
+          sKsf[s][lane + 32 * j] = __half2float(__ushort_as_half(ksv[j]));
+          sVsf[s][lane + 32 * j] = __half2float(__ushort_as_half(vsv[j])) * inv;
+        }
+        if (lane == 0) sVmax[s] = vrun;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
@@ -292,9 +306,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // supplies head gq, channels kb*32 + 8*cq + {0..3} (b0) and {4..7} (b1);
   // INT4: the even channels of those 8 (b0) and the odd ones (b1). Any
   // channel order works as long as the key fragments use the same one.
+  // With G <= 4 the 8 MMA columns hold each head twice (column n: head
+  // n % 4): the score columns 4-7 repeat 0-3, and in P.V columns 0-3 take
+  // the fp16 high part of P', columns 4-7 its remainder, so that one MMA
+  // does both (the two halves are added at the end).
+  constexpr bool kHiLo = G <= 4;
+  const int qh = kHiLo ? (gq & 3) : gq;     // head of MMA column gq
+  const bool qok = qh < G;
   uint32_t qb0[4], qb1[4];
   {
-    const uint8_t* qbytes = reinterpret_cast<const uint8_t*>(&sQw[gq < G ? gq : 0][0]);
+    const uint8_t* qbytes = reinterpret_cast<const uint8_t*>(&sQw[qok ? qh : 0][0]);
 #pragma unroll
     for (int kb = 0; kb < 4; ++kb) {
       const int d0 = kb * 32 + 8 * cq;
@@ -308,13 +329,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         x0 = __byte_perm(w0, w1, 0x6420);
         x1 = __byte_perm(w0, w1, 0x7531);
       }
-      qb0[kb] = gq < G ? x0 : 0u;
-      qb1[kb] = gq < G ? x1 : 0u;
+      qb0[kb] = qok ? x0 : 0u;
+      qb1[kb] = qok ? x1 : 0u;
     }
   }
-  // Heads of this lane's score columns: 2*cq and 2*cq + 1.
-  const int h0 = 2 * cq, h1 = 2 * cq + 1;
+  // Heads of this lane's score columns 2*cq and 2*cq + 1.
+  // (with kHiLo, lanes cq >= 2 hold copies of heads 2(cq-2), 2(cq-2) + 1)
+  const int h0 = kHiLo ? (2 * cq) & 3 : 2 * cq, h1 = h0 + 1;
   const bool h0ok = h0 < G, h1ok = h1 < G;
+  const bool own = !kHiLo || cq < 2;        // this lane writes its heads' P' and state
   const float qf0 = h0ok ? sQf[h0] : 0.0f, qf1 = h1ok ? sQf[h1] : 0.0f;
   int qs0[2] = {0, 0}, qs1[2] = {0, 0};          // INT4: 8 * query code sums per group
   if constexpr (kInt4) {
@@ -361,7 +384,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // running V-scale reference: P' = p * vscale / vref stays in [0, 1]
     const float vref_new = fmaxf(vref, sVmax[s]);
     const float vratio = vref_new > 0.0f ? vref / vref_new : 1.0f;
-    const float inv_vref = vref_new > 0.0f ? 1.0f / vref_new : 0.0f;
     vref = vref_new;
     if (vratio != 1.0f) {                     // the same on every lane
 #pragma unroll
@@ -420,20 +442,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       float s_a0, s_a1, s_b0, s_b1;
       if constexpr (!kInt4) {
         const float kq0 = qf0 * sKsc[s], kq1 = qf1 * sKsc[s];
-        s_a0 = static_cast<float>(sc[0][0]) * kq0;
-        s_a1 = static_cast<float>(sc[0][1]) * kq1;
-        s_b0 = static_cast<float>(sc[0][2]) * kq0;
-        s_b1 = static_cast<float>(sc[0][3]) * kq1;
+        s_a0 = i2f_exact(sc[0][0]) * kq0;
+        s_a1 = i2f_exact(sc[0][1]) * kq1;
+        s_b0 = i2f_exact(sc[0][2]) * kq0;
+        s_b1 = i2f_exact(sc[0][3]) * kq1;
       } else {
         float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
 #pragma unroll
         for (int gg = 0; gg < kNAcc; ++gg) {
-          const float ka = __half2float(__ushort_as_half(sKs16[s][ra * kGroups + gg]));
-          const float kb2 = __half2float(__ushort_as_half(sKs16[s][rb * kGroups + gg]));
-          t0 += static_cast<float>(sc[gg][0] - qs0[gg]) * ka;
-          t1 += static_cast<float>(sc[gg][1] - qs1[gg]) * ka;
-          t2 += static_cast<float>(sc[gg][2] - qs0[gg]) * kb2;
-          t3 += static_cast<float>(sc[gg][3] - qs1[gg]) * kb2;
+          const float ka = sKsf[s][ra * kGroups + gg];
+          const float kb2 = sKsf[s][rb * kGroups + gg];
+          t0 = fmaf(i2f_exact(sc[gg][0] - qs0[gg]), ka, t0);
+          t1 = fmaf(i2f_exact(sc[gg][1] - qs1[gg]), ka, t1);
+          t2 = fmaf(i2f_exact(sc[gg][2] - qs0[gg]), kb2, t2);
+          t3 = fmaf(i2f_exact(sc[gg][3] - qs1[gg]), kb2, t3);
         }
         s_a0 = t0 * qf0; s_a1 = t1 * qf1; s_b0 = t2 * qf0; s_b1 = t3 * qf1;
       }
@@ -457,16 +479,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       l_run1 = l_run1 * al1 + (pa1 + pb1);
       // P' = p * vscale / vref -> per-warp buffer [group][head][token]
       if constexpr (!kInt4) {
-        const float f = sVsc[s] * inv_vref;
-        if (h0ok) { myP[0][h0][gq] = pa0 * f; myP[0][h0][gq + 8] = pb0 * f; }
-        if (h1ok) { myP[0][h1][gq] = pa1 * f; myP[0][h1][gq + 8] = pb1 * f; }
+        const float f = sVsc[s];
+        if (own && h0ok) { myP[0][h0][gq] = pa0 * f; myP[0][h0][gq + 8] = pb0 * f; }
+        if (own && h1ok) { myP[0][h1][gq] = pa1 * f; myP[0][h1][gq + 8] = pb1 * f; }
       } else {
 #pragma unroll
         for (int gg = 0; gg < kGroups; ++gg) {
-          const float fa = __half2float(__ushort_as_half(sVs16[s][ra * kGroups + gg])) * inv_vref;
-          const float fb = __half2float(__ushort_as_half(sVs16[s][rb * kGroups + gg])) * inv_vref;
-          if (h0ok) { myP[gg][h0][gq] = pa0 * fa; myP[gg][h0][gq + 8] = pb0 * fb; }
-          if (h1ok) { myP[gg][h1][gq] = pa1 * fa; myP[gg][h1][gq + 8] = pb1 * fb; }
+          const float fa = sVsf[s][ra * kGroups + gg];
+          const float fb = sVsf[s][rb * kGroups + gg];
+          if (own && h0ok) { myP[gg][h0][gq] = pa0 * fa; myP[gg][h0][gq + 8] = pb0 * fb; }
+          if (own && h1ok) { myP[gg][h1][gq] = pa1 * fa; myP[gg][h1][gq + 8] = pb1 * fb; }
         }
       }
       __syncwarp();
@@ -481,18 +503,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           sacc[gg][0] *= al0; sacc[gg][1] *= al1; sacc[gg][2] *= al0; sacc[gg][3] *= al1;
         }
       }
-      // P'^T fragments (B): head gq, tokens 2cq, 2cq+1 (b0) and 2cq+8, 2cq+9
-      // (b1), as fp16 high and low parts
+      // P'^T fragments (B): column gq = head qh, tokens 2cq, 2cq+1 (b0) and
+      // 2cq+8, 2cq+9 (b1), as fp16 high and low parts; with kHiLo column gq
+      // carries the high part (gq < 4) or the remainder (gq >= 4) alone, in
+      // the *_hi registers
       uint32_t p0_hi[kGroups], p0_lo[kGroups], p1_hi[kGroups], p1_lo[kGroups];
 #pragma unroll
       for (int gg = 0; gg < kGroups; ++gg) {
         float2 x01 = make_float2(0.0f, 0.0f), x89 = make_float2(0.0f, 0.0f);
-        if (gq < G) {
-          x01 = *reinterpret_cast<const float2*>(&myP[gg][gq][2 * cq]);
-          x89 = *reinterpret_cast<const float2*>(&myP[gg][gq][2 * cq + 8]);
+        if (qok) {
+          x01 = *reinterpret_cast<const float2*>(&myP[gg][qh][2 * cq]);
+          x89 = *reinterpret_cast<const float2*>(&myP[gg][qh][2 * cq + 8]);
         }
         split_f16x2(x01.x, x01.y, p0_hi[gg], p0_lo[gg]);
         split_f16x2(x89.x, x89.y, p1_hi[gg], p1_lo[gg]);
+        if constexpr (kHiLo) {
+          if (gq >= 4) { p0_hi[gg] = p0_lo[gg]; p1_hi[gg] = p1_lo[gg]; }
+        }
       }
       // ---------------- O^T += V'^T P'^T, sum(P') against a tile of ones ----------------
       {
@@ -514,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               const uint32_t a2 = __byte_perm(xh, 0x64646464u, 0x4240), a3 = __byte_perm(xh, 0x64646464u, 0x4341);
               const int mt = 2 * cp + h;
               mma_f16x4(acc[mt], a0, a1, a2, a3, p0_hi[0], p1_hi[0]);
-              mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[0], p1_lo[0]);
+              if constexpr (!kHiLo) mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[0], p1_lo[0]);
             }
           } else {
             // chunk 2cp + h (32 channels) -> m-tiles 4cp + 2h + u: row g =
@@ -531,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int mt = 4 * cp + 2 * h + u;
                 const int gg = (kGroups == 2 && mt >= 4) ? 1 : 0;
                 mma_f16x4(acc[mt], a0, a1, a2, a3, p0_hi[gg], p1_hi[gg]);
-                mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[gg], p1_lo[gg]);
+                if constexpr (!kHiLo) mma_f16x4(acc[mt], a0, a1, a2, a3, p0_lo[gg], p1_lo[gg]);
               }
             }
           }
@@ -540,7 +567,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
       for (int gg = 0; gg < kGroups; ++gg) {
         mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_hi[gg], p1_hi[gg]);
-        mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_lo[gg], p1_lo[gg]);
+        if constexpr (!kHiLo)
+          mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_lo[gg], p1_lo[gg]);
       }
       __syncwarp();                  // buffers reused by the next step
     }
@@ -558,9 +586,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // every issued copy was consumed (or waited for on a timeout): the ring can
   // be reused for the reduction once all consumer warps are past their loops
   named_bar_sync(1, 32 * kConsumers);
-  if (gq == 0) {
+  if (gq == 0 && own) {
     if (h0ok) { sWm[warp][h0] = m_run0; sWl[warp][h0] = l_run0; }
     if (h1ok) { sWm[warp][h1] = m_run1; sWl[warp][h1] = l_run1; }
+  }
+  if constexpr (kHiLo) {
+    // columns 2cq, 2cq+1 (cq < 2) gathered the high parts of P', columns
+    // 2cq+4, 2cq+5 (lane ^ 2) the remainders of the same heads
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][e] += __shfl_xor_sync(0xffffffffu, acc[mt][e], 2);
+#pragma unroll
+    for (int gg = 0; gg < kGroups; ++gg)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[gg][e] += __shfl_xor_sync(0xffffffffu, sacc[gg][e], 2);
   }
   // O = (acc - offset * sum(P')) * vref; INT4 odd channels also / 16.
   // Row g of m-tile mt holds channel 16mt + 2g (INT8) or 32(mt/4)... see the
@@ -572,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int hh = 2 * cq + (e & 1);
-      if (hh >= G) continue;
+      if (hh >= G || !own) continue;
       const bool odd = (e >> 1) != 0;                        // row g+8
       const float sp = sacc[gg][e & 1];
       float o;
