@@ -32,12 +32,27 @@ namespace qattn {
 
 namespace {
 
-// 8 x 8 thread tiles: 256 threads for 128-token blocks (and D = 64), 512 for
-// 256-token blocks at D = 128.
+// Threads per team (one team computes one block at a time): at D = 128,
+// 16 x 8 thread tiles for 128-token blocks (128 threads; two teams per CTA
+// share R, so one team's staging and coding overlap the other's FMA loop)
+// and 8 x 8 tiles for 256-token blocks (512 threads, one team); at D = 64,
+// 4 x 8 tiles (256 threads).
 template <int D, int T>
 struct RotqThreads {
-  static constexpr int value = D == 128 && T == 256 ? 512 : 256;
+  static constexpr int value = D == 128 ? (T == 256 ? 512 : 128) : 256;
 };
+template <int D, int T>
+struct RotqTeams {
+  static constexpr int value = D == 128 && T == 128 ? 2 : 1;
+};
+
+// Barrier of one team: the whole CTA when it is the only team, else the
+// team's named barrier (1 + team).
+template <int kNT, int kTeams>
+__device__ __forceinline__ void team_sync(int team) {
+  if constexpr (kTeams == 1) __syncthreads();
+  else named_bar_sync(1 + team, kNT);
+}
 
 __device__ __forceinline__ void unpack8(uint4 v, bool is_bf16, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -98,17 +113,19 @@ __device__ __forceinline__ uint32_t code_of(float y, float scale, float rcp, boo
   }
 }
 
-template <int kNT>
-__device__ __forceinline__ float block_max(float v, float* red) {
+// Maximum of v over the kNT threads of a team (ttid: thread within the team;
+// red: kNT / 32 floats of the team).
+template <int kNT, int kTeams = 1>
+__device__ __forceinline__ float block_max(float v, float* red, int ttid = threadIdx.x, int team = 0) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[w] = v;
-  __syncthreads();
+  const int w = ttid >> 5;
+  if ((ttid & 31) == 0) red[w] = v;
+  team_sync<kNT, kTeams>(team);
   float m = 0.0f;
 #pragma unroll
   for (int i = 0; i < kNT / 32; ++i) m = fmaxf(m, red[i]);
-  __syncthreads();  // red[] may be reused
+  team_sync<kNT, kTeams>(team);  // red[] may be reused
   return m;
 }
 
@@ -294,24 +311,28 @@ __device__ __noinline__ uint2 codes8_exact_f(F8 f, float scale) {
 // row group rg = tid / (D/8) owns rows rg*kRPT .. rg*kRPT + kRPT - 1.
 // kInt4 (with kInt8): INT4 codes (scale absmax / 7), two per byte.
 template <int D, int T, bool kInt8, bool kInt4>
-__global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
+__global__ void __launch_bounds__(RotqThreads<D, T>::value * RotqTeams<D, T>::value, 1)
     rotq_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
                 const float* __restrict__ rot, uint8_t* __restrict__ codes,
                 float* __restrict__ scales) {
   constexpr int kNT = RotqThreads<D, T>::value;
+  constexpr int kTeams = RotqTeams<D, T>::value;
   constexpr int kCG = D / 8;               // column groups
   constexpr int kRG = kNT / kCG;           // row groups
   constexpr int kRPT = T / kRG;            // rows per thread
   constexpr int kXS = T + 4;               // padded row stride of the transposed x tile
   static_assert(kRPT % 4 == 0 && kRPT >= 4, "row tile");
   extern __shared__ __align__(16) float smem[];
+  const int team = threadIdx.x / kNT;
+  const int tid = threadIdx.x % kNT;       // thread within the team
   float* sR = smem;                        // [D][D]
-  float* sX = smem + D * D;                // [D][kXS]: sX[k * kXS + r] = x[r][k]
-  __shared__ float red[kNT / 32];
+  float* sX = smem + D * D + team * D * kXS;   // this team's [D][kXS]: sX[k * kXS + r] = x[r][k]
+  __shared__ float red_all[kTeams][kNT / 32];
+  float* red = red_all[team];
 
-  const int tid = threadIdx.x;
-  for (int i = tid; i < D * D / 4; i += kNT)
+  for (int i = threadIdx.x; i < D * D / 4; i += kNT * kTeams)
     reinterpret_cast<float4*>(sR)[i] = reinterpret_cast<const float4*>(rot)[i];
+  if constexpr (kTeams > 1) __syncthreads();   // sR ready
 
   const int nblk = (N + T - 1) / T;
   const int64_t total = static_cast<int64_t>(B) * H * nblk;
@@ -342,9 +363,20 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
   // Only where the registers allow it (the larger row tiles of 256-token
   // blocks already use them all): otherwise the block is loaded on the spot.
   constexpr bool kPrefetch = kLd <= 4;
-  if (kPrefetch && blockIdx.x < total) load_block(blockIdx.x);
+  // Team t of CTA c takes the blocks c + (t + kTeams i) * gridDim.x.
+  const int64_t first = blockIdx.x + static_cast<int64_t>(team) * gridDim.x;
+  const int64_t step = static_cast<int64_t>(kTeams) * gridDim.x;
+  if (kPrefetch && first < total) load_block(first);
+  // The second team starts once the first has finished the FMA loop of its
+  // first block, so that the teams' loops are out of phase (one team's
+  // loading, staging and coding run under the other's loop). Team 0 arrives
+  // exactly once, whether or not it has a block.
+  if constexpr (kTeams > 1) {
+    if (team == 1) named_bar_sync(3, 2 * kNT);
+    else if (first >= total) named_bar_arrive(3, 2 * kNT);
+  }
 
-  for (int64_t blk_id = blockIdx.x; blk_id < total; blk_id += gridDim.x) {
+  for (int64_t blk_id = first; blk_id < total; blk_id += step) {
     const int blk = static_cast<int>(blk_id % nblk);
     const int bh = static_cast<int>(blk_id / nblk);
     const int b = bh / H, h = bh % H;
@@ -352,7 +384,7 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
     const int rows = min(T, N - n0);
 
     if (!kPrefetch) load_block(blk_id);
-    __syncthreads();  // sR ready (first pass); previous block's sX reads done
+    team_sync<kNT, kTeams>(team);  // sR ready (first pass); previous block's sX reads done
     // Stage x transposed: consecutive threads write consecutive words.
 #pragma unroll
     for (int i = 0; i < kLd; ++i) {
@@ -365,42 +397,51 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
         for (int e = 0; e < 8; ++e) sX[(c * 8 + e) * kXS + r] = f[e];
       }
     }
-    __syncthreads();
-    if (kPrefetch && blk_id + gridDim.x < total) load_block(blk_id + gridDim.x);
+    team_sync<kNT, kTeams>(team);
+    if (kPrefetch && blk_id + step < total) load_block(blk_id + step);
 
-    // acc[i][j]: row rg*kRPT + i, column (j < 4 ? c0 + j : c1 + j - 4); each
-    // is the float32 FMA chain over k ascending, two lanes per f32x2 FMA.
-    float2 acc[kRPT][4];
+    // acc[p][j]: rows rg*kRPT + 2p (.x) and + 2p + 1 (.y), column (j < 4 ?
+    // c0 + j : c1 + j - 4); each is the float32 FMA chain over k ascending,
+    // two rows per f32x2 FMA (x pairs straight from the transposed tile, the
+    // R value duplicated).
+    float2 acc[kRPT / 2][8];
 #pragma unroll
-    for (int i = 0; i < kRPT; ++i)
+    for (int i = 0; i < kRPT / 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+      for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
 #pragma unroll 2
     for (int k = 0; k < D; ++k) {
       const float4 r0 = *reinterpret_cast<const float4*>(sR + k * D + c0);
       const float4 r1 = *reinterpret_cast<const float4*>(sR + k * D + c1);
-      const float2 rv[4] = {make_float2(r0.x, r0.y), make_float2(r0.z, r0.w), make_float2(r1.x, r1.y),
-                            make_float2(r1.z, r1.w)};
+      const float rs[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+      float2 r2[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) r2[j] = make_float2(rs[j], rs[j]);
 #pragma unroll
       for (int i4 = 0; i4 < kRPT / 4; ++i4) {
         const float4 xv = *reinterpret_cast<const float4*>(sX + k * kXS + rg * kRPT + i4 * 4);
-        const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float2 xa = make_float2(xv.x, xv.y), xb = make_float2(xv.z, xv.w);
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          const float2 x2 = make_float2(xs[ii], xs[ii]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i4 * 4 + ii][j] = ffma2(x2, rv[j], acc[i4 * 4 + ii][j]);
+        for (int j = 0; j < 8; ++j) {
+          acc[2 * i4][j] = ffma2(xa, r2[j], acc[2 * i4][j]);
+          acc[2 * i4 + 1][j] = ffma2(xb, r2[j], acc[2 * i4 + 1][j]);
         }
       }
     }
+    if (kTeams > 1 && team == 0 && blk_id == first) named_bar_arrive(3, 2 * kNT);
+    // the 8 values of row i (columns c0..c0+3, c1..c1+3)
+    auto row8 = [&](int i, float (&f)[8]) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = (i & 1) ? acc[i >> 1][j].y : acc[i >> 1][j].x;
+    };
 
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kRPT; ++i)
+    for (int i = 0; i < kRPT / 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(acc[i][j].x), fabsf(acc[i][j].y)));  // padded rows are +0
-    const float amax = block_max<kNT>(m, red);
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fmaxf(fabsf(acc[i][j].x), fabsf(acc[i][j].y)));  // padded rows are +0
+    const float amax = block_max<kNT, kTeams>(m, red, tid, team);
     const float scale = __fdiv_rn(amax, qmax);
     const float rcp = __frcp_rn(scale);
     const bool slow = scale < 1.17549435e-38f;
@@ -414,8 +455,8 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
     uint32_t fix = 0;
 #pragma unroll
     for (int i = 0; i < kRPT; ++i) {
-      const float f[8] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
-                          acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y};
+      float f[8];
+      row8(i, f);
       fix |= codes8_fast<kInt8, false, kInt4>(f, rcp, w[i].x, w[i].y) ? 0u : 1u << i;
     }
     if (scale == 0.0f) {                              // all-zero block: zero codes
@@ -447,8 +488,8 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value, 1)
 #pragma unroll
       for (int i = 0; i < kRPT; ++i) {
         if (!((fix >> i) & 1u) || rg * kRPT + i >= rows) continue;
-        const F8 f = {{acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y,
-                       acc[i][2].x, acc[i][2].y, acc[i][3].x, acc[i][3].y}};
+        F8 f;
+        row8(i, f.v);
         store(i, codes8_exact_f<kInt8, kInt4>(f, scale));
       }
     }
@@ -635,13 +676,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
 template <int D, int T, bool kInt8, bool kInt4 = false>
 cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
-  constexpr size_t smem = sizeof(float) * (D * D + D * (T + 4));
+  constexpr int kTeams = RotqTeams<D, T>::value;
+  constexpr size_t smem = sizeof(float) * (D * D + kTeams * D * (T + 4));
   auto k = rotq_kernel<D, T, kInt8, kInt4>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
   const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
-  k<<<grid, RotqThreads<D, T>::value, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B,
+  k<<<grid, RotqThreads<D, T>::value * kTeams, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B,
                                                 a.H, a.N, a.rot, static_cast<uint8_t*>(a.codes), a.scales);
   return cudaGetLastError();
 }
