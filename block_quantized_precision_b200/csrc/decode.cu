@@ -18,7 +18,9 @@
 //               multicast); it also stages each chunk's scales and the
 //               largest V scale of the chunk.
 //   warps 0-3   consumers, each on its own quarter of every chunk with its
-//               own running softmax, 16 tokens per step, on the warp-level
+//               own running softmax, one step per chunk (16 tokens INT8, 32
+//               INT4: two 16-token halves whose score MMAs are independent
+//               and which share one max reduction), on the warp-level
 //               tensor-core instructions:
 //                 scores  S^T[16 tokens x 8 heads] = K Q^T by
 //                         mma.m16n8k32 s8 x s8 -> s32: key rows straight from
@@ -62,17 +64,22 @@ constexpr int kConsumers = 4;         // consumer warps
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStep = 16;             // tokens per consumer step
 constexpr int kWsStride = kD + 4;     // floats per (b, h_q, split) partial: O[D], m, l, pad
-constexpr int kPStride = 20;          // floats per head row of the per-warp P' buffer
 constexpr uint32_t kOnesF16x2 = 0x3C003C00u;
-constexpr int kCtasPerSm = 3;         // resident CTAs per SM (registers)
 
 template <bool kInt4>
 struct Cfg {
   static constexpr int kRowBytes = kInt4 ? kD / 2 : kD;
   static constexpr int kChunk = kInt4 ? 128 : 64;             // tokens per stage
-  static constexpr int kStages = kInt4 ? 3 : 4;
+  static constexpr int kStages = 3;
+  // resident CTAs per SM: 4 (<= 96 registers) for INT8; the 32-token steps
+  // of INT4 need more registers: 3 (<= 136)
+  static constexpr int kCtasPerSm = kInt4 ? 3 : 4;
   static constexpr int kTileBytes = kChunk * kRowBytes;       // one tensor, one stage (8 KB)
   static constexpr int kPerWarp = kChunk / kConsumers;        // tokens per warp per chunk
+  static constexpr int kHalves = kInt4 ? 2 : 1;               // 16-token halves per consumer step
+  // floats per head row of the per-warp P' buffer (the step's tokens + pad:
+  // the rows' float2 reads of one warp fall on distinct banks)
+  static constexpr int kPStride = kInt4 ? 40 : 20;
   static constexpr int kSmemBytes = 2 * kStages * kTileBytes + 1024;
 };
 
@@ -137,7 +144,7 @@ __device__ __forceinline__ void split_f16x2(float x, float y, uint32_t& hi, uint
 }
 
 template <int G, bool kInt4, int kGroups>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
   static_assert(G >= 1 && G <= 8, "query heads per kv head");
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __shared__ float sQf[G];                             // sq * softmax scale * log2(e)
   // P'[head][token] per warp; rows of kPStride floats keep the stores of a
   // warp on distinct banks
-  __shared__ __align__(16) float sPw[kConsumers][kGroups][8][kPStride];
+  __shared__ __align__(16) float sPw[kConsumers][kGroups][8][C::kPStride];
   __shared__ float sKsc[kStages], sVsc[kStages], sVmax[kStages];
   // INT4 group scales of the chunk as float [token][group]: K as stored, V
   // already divided by the running max V scale (sVmax)
@@ -349,7 +356,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       qs0[0] = 8 * (s00 + s01); qs1[0] = 8 * (s10 + s11);
     }
   }
-  float (*myP)[8][kPStride] = sPw[warp];
+  float (*myP)[8][C::kPStride] = sPw[warp];
+  constexpr int kH = C::kHalves;
   // P.V is computed transposed, O^T[channels x heads] += V'^T P'^T, with
   // A = V'^T taken straight from the swizzled V tile: ldmatrix.trans on
   // 2-byte elements gives each lane, for tokens (2cq, 2cq+1) of a 16-token
@@ -396,73 +404,82 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int e = 0; e < 4; ++e) sacc[gg][e] *= vratio;
     }
 #pragma unroll 1
-    for (int sub = 0; sub < C::kPerWarp / kStep; ++sub) {
-      const int r0 = warp * C::kPerWarp + sub * kStep;      // first row of this step in the chunk
-      const int ra = r0 + gq, rb = r0 + gq + 8;             // this lane's score rows (tokens)
-      const bool va = chunk_t0 + ra < t_end, vb = chunk_t0 + rb < t_end;
-      // ---------------- scores: S^T = K Q^T ----------------
-      // one accumulator per 32-channel slice, so that the four MMAs do not
-      // wait on one another; the slices are then added (exact in INT32)
-      int sck[4][4];
+    for (int sub = 0; sub < C::kPerWarp / (kStep * kH); ++sub) {
+      const int r0 = warp * C::kPerWarp + sub * kStep * kH;  // first row of this step in the chunk
+      // ---------------- scores: S^T = K Q^T, per 16-token half ----------------
+      // sv[hf]: (row ra, head h0), (ra, h1), (rb, h0), (rb, h1) with ra =
+      // r0 + 16 hf + gq, rb = ra + 8 (the accumulator layout)
+      float sv[kH][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) sck[a][0] = sck[a][1] = sck[a][2] = sck[a][3] = 0;
+      for (int hf = 0; hf < kH; ++hf) {
+        const int ra = r0 + kStep * hf + gq, rb = ra + 8;   // this lane's score rows (tokens)
+        const bool va = chunk_t0 + ra < t_end, vb = chunk_t0 + rb < t_end;
+        // one accumulator per 32-channel slice, so that the four MMAs do not
+        // wait on one another; the slices are then added (exact in INT32)
+        int sck[4][4];
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
+        for (int a = 0; a < 4; ++a) sck[a][0] = sck[a][1] = sck[a][2] = sck[a][3] = 0;
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          if constexpr (!kInt4) {
+            // 8 bytes of rows ra / rb at channel kb*32 + 8*cq: 16-byte chunk
+            // 2kb + cq/2, stored at chunk ^ (row % 8)
+            const int ch = 2 * kb + (cq >> 1);
+            const int off = ((ch ^ gq) << 4) + (cq & 1) * 8;
+            const uint2 xa = *reinterpret_cast<const uint2*>(cK + ra * 128 + off);
+            const uint2 xb = *reinterpret_cast<const uint2*>(cK + rb * 128 + off);
+            mma_s8(sck[kb], xa.x, xb.x, xa.y, xb.y, qb0[kb], qb1[kb]);
+          } else {
+            // 4 bytes (8 nibbles) of rows ra / rb at channel kb*32 + 8*cq:
+            // 16-byte chunk kb, stored at kb ^ ((row / 2) % 4)
+            const int off = ((kb ^ ((gq >> 1) & 3)) << 4) + 4 * cq;
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(cK + ra * 64 + off);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(cK + rb * 64 + off);
+            // nibble c -> byte c + 8 (even channels, odd channels)
+            const uint32_t ea = (wa & 0x0F0F0F0Fu) ^ 0x08080808u, oa = ((wa >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t eb = (wb & 0x0F0F0F0Fu) ^ 0x08080808u, ob = ((wb >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            mma_s8(sck[kb], ea, eb, oa, ob, qb0[kb], qb1[kb]);
+          }
+        }
+        int sc[kNAcc][4];                                  // per INT4 group (else all 128 channels)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (kNAcc == 2) {
+            sc[0][e] = sck[0][e] + sck[1][e];
+            sc[kNAcc - 1][e] = sck[2][e] + sck[3][e];
+          } else {
+            sc[0][e] = (sck[0][e] + sck[1][e]) + (sck[2][e] + sck[3][e]);
+          }
+        }
         if constexpr (!kInt4) {
-          // 8 bytes of rows ra / rb at channel kb*32 + 8*cq: 16-byte chunk
-          // 2kb + cq/2, stored at chunk ^ (row % 8)
-          const int ch = 2 * kb + (cq >> 1);
-          const int off = ((ch ^ gq) << 4) + (cq & 1) * 8;
-          const uint2 xa = *reinterpret_cast<const uint2*>(cK + ra * 128 + off);
-          const uint2 xb = *reinterpret_cast<const uint2*>(cK + rb * 128 + off);
-          mma_s8(sck[kb], xa.x, xb.x, xa.y, xb.y, qb0[kb], qb1[kb]);
+          const float kq0 = qf0 * sKsc[s], kq1 = qf1 * sKsc[s];
+          sv[hf][0] = i2f_exact(sc[0][0]) * kq0;
+          sv[hf][1] = i2f_exact(sc[0][1]) * kq1;
+          sv[hf][2] = i2f_exact(sc[0][2]) * kq0;
+          sv[hf][3] = i2f_exact(sc[0][3]) * kq1;
         } else {
-          // 4 bytes (8 nibbles) of rows ra / rb at channel kb*32 + 8*cq:
-          // 16-byte chunk kb, stored at kb ^ ((row / 2) % 4)
-          const int off = ((kb ^ ((gq >> 1) & 3)) << 4) + 4 * cq;
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>(cK + ra * 64 + off);
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>(cK + rb * 64 + off);
-          // nibble c -> byte c + 8 (even channels, odd channels)
-          const uint32_t ea = (wa & 0x0F0F0F0Fu) ^ 0x08080808u, oa = ((wa >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-          const uint32_t eb = (wb & 0x0F0F0F0Fu) ^ 0x08080808u, ob = ((wb >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-          mma_s8(sck[kb], ea, eb, oa, ob, qb0[kb], qb1[kb]);
-        }
-      }
-      int sc[kNAcc][4];                                    // per INT4 group (else all 128 channels)
+          float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if constexpr (kNAcc == 2) {
-          sc[0][e] = sck[0][e] + sck[1][e];
-          sc[kNAcc - 1][e] = sck[2][e] + sck[3][e];
-        } else {
-          sc[0][e] = (sck[0][e] + sck[1][e]) + (sck[2][e] + sck[3][e]);
+          for (int gg = 0; gg < kNAcc; ++gg) {
+            const float ka = sKsf[s][ra * kGroups + gg];
+            const float kb2 = sKsf[s][rb * kGroups + gg];
+            t0 = fmaf(i2f_exact(sc[gg][0] - qs0[gg]), ka, t0);
+            t1 = fmaf(i2f_exact(sc[gg][1] - qs1[gg]), ka, t1);
+            t2 = fmaf(i2f_exact(sc[gg][2] - qs0[gg]), kb2, t2);
+            t3 = fmaf(i2f_exact(sc[gg][3] - qs1[gg]), kb2, t3);
+          }
+          sv[hf][0] = t0 * qf0; sv[hf][1] = t1 * qf1; sv[hf][2] = t2 * qf0; sv[hf][3] = t3 * qf1;
         }
+        if (!va) { sv[hf][0] = -CUDART_INF_F; sv[hf][1] = -CUDART_INF_F; }
+        if (!vb) { sv[hf][2] = -CUDART_INF_F; sv[hf][3] = -CUDART_INF_F; }
       }
-      // accumulator layout: [0] = (ra, h0), [1] = (ra, h1), [2] = (rb, h0), [3] = (rb, h1)
-      float s_a0, s_a1, s_b0, s_b1;
-      if constexpr (!kInt4) {
-        const float kq0 = qf0 * sKsc[s], kq1 = qf1 * sKsc[s];
-        s_a0 = i2f_exact(sc[0][0]) * kq0;
-        s_a1 = i2f_exact(sc[0][1]) * kq1;
-        s_b0 = i2f_exact(sc[0][2]) * kq0;
-        s_b1 = i2f_exact(sc[0][3]) * kq1;
-      } else {
-        float t0 = 0.0f, t1 = 0.0f, t2 = 0.0f, t3 = 0.0f;
+      // ---------------- running softmax per head over the step's tokens ----------------
+      float mx0 = fmaxf(sv[0][0], sv[0][2]), mx1 = fmaxf(sv[0][1], sv[0][3]);
 #pragma unroll
-        for (int gg = 0; gg < kNAcc; ++gg) {
-          const float ka = sKsf[s][ra * kGroups + gg];
-          const float kb2 = sKsf[s][rb * kGroups + gg];
-          t0 = fmaf(i2f_exact(sc[gg][0] - qs0[gg]), ka, t0);
-          t1 = fmaf(i2f_exact(sc[gg][1] - qs1[gg]), ka, t1);
-          t2 = fmaf(i2f_exact(sc[gg][2] - qs0[gg]), kb2, t2);
-          t3 = fmaf(i2f_exact(sc[gg][3] - qs1[gg]), kb2, t3);
-        }
-        s_a0 = t0 * qf0; s_a1 = t1 * qf1; s_b0 = t2 * qf0; s_b1 = t3 * qf1;
+      for (int hf = 1; hf < kH; ++hf) {
+        mx0 = fmaxf(mx0, fmaxf(sv[hf][0], sv[hf][2]));
+        mx1 = fmaxf(mx1, fmaxf(sv[hf][1], sv[hf][3]));
       }
-      if (!va) { s_a0 = -CUDART_INF_F; s_a1 = -CUDART_INF_F; }
-      if (!vb) { s_b0 = -CUDART_INF_F; s_b1 = -CUDART_INF_F; }
-      // ---------------- running softmax per head over the 16 tokens ----------------
-      float mx0 = fmaxf(s_a0, s_b0), mx1 = fmaxf(s_a1, s_b1);
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
@@ -473,22 +490,36 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const float al0 = ex2(m_run0 - mn0), al1 = ex2(m_run1 - mn1);
       m_run0 = mn0;
       m_run1 = mn1;
-      const float pa0 = ex2(s_a0 - mn0), pa1 = ex2(s_a1 - mn1);
-      const float pb0 = ex2(s_b0 - mn0), pb1 = ex2(s_b1 - mn1);
-      l_run0 = l_run0 * al0 + (pa0 + pb0);
-      l_run1 = l_run1 * al1 + (pa1 + pb1);
-      // P' = p * vscale / vref -> per-warp buffer [group][head][token]
-      if constexpr (!kInt4) {
-        const float f = sVsc[s];
-        if (own && h0ok) { myP[0][h0][gq] = pa0 * f; myP[0][h0][gq + 8] = pb0 * f; }
-        if (own && h1ok) { myP[0][h1][gq] = pa1 * f; myP[0][h1][gq + 8] = pb1 * f; }
-      } else {
+      float pr[kH][4];
+      float ls0 = 0.0f, ls1 = 0.0f;
 #pragma unroll
-        for (int gg = 0; gg < kGroups; ++gg) {
-          const float fa = sVsf[s][ra * kGroups + gg];
-          const float fb = sVsf[s][rb * kGroups + gg];
-          if (own && h0ok) { myP[gg][h0][gq] = pa0 * fa; myP[gg][h0][gq + 8] = pb0 * fb; }
-          if (own && h1ok) { myP[gg][h1][gq] = pa1 * fa; myP[gg][h1][gq + 8] = pb1 * fb; }
+      for (int hf = 0; hf < kH; ++hf) {
+        pr[hf][0] = ex2(sv[hf][0] - mn0);
+        pr[hf][1] = ex2(sv[hf][1] - mn1);
+        pr[hf][2] = ex2(sv[hf][2] - mn0);
+        pr[hf][3] = ex2(sv[hf][3] - mn1);
+        ls0 += pr[hf][0] + pr[hf][2];
+        ls1 += pr[hf][1] + pr[hf][3];
+      }
+      l_run0 = l_run0 * al0 + ls0;
+      l_run1 = l_run1 * al1 + ls1;
+      // P' = p * vscale / vref -> per-warp buffer [group][head][token of the step]
+#pragma unroll
+      for (int hf = 0; hf < kH; ++hf) {
+        const int ta = kStep * hf + gq;                    // token of row ra within the step
+        if constexpr (!kInt4) {
+          const float f = sVsc[s];
+          if (own && h0ok) { myP[0][h0][ta] = pr[hf][0] * f; myP[0][h0][ta + 8] = pr[hf][2] * f; }
+          if (own && h1ok) { myP[0][h1][ta] = pr[hf][1] * f; myP[0][h1][ta + 8] = pr[hf][3] * f; }
+        } else {
+          const int ra = r0 + ta, rb = ra + 8;
+#pragma unroll
+          for (int gg = 0; gg < kGroups; ++gg) {
+            const float fa = sVsf[s][ra * kGroups + gg];
+            const float fb = sVsf[s][rb * kGroups + gg];
+            if (own && h0ok) { myP[gg][h0][ta] = pr[hf][0] * fa; myP[gg][h0][ta + 8] = pr[hf][2] * fb; }
+            if (own && h1ok) { myP[gg][h1][ta] = pr[hf][1] * fa; myP[gg][h1][ta + 8] = pr[hf][3] * fb; }
+          }
         }
       }
       __syncwarp();
@@ -503,27 +534,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           sacc[gg][0] *= al0; sacc[gg][1] *= al1; sacc[gg][2] *= al0; sacc[gg][3] *= al1;
         }
       }
-      // P'^T fragments (B): column gq = head qh, tokens 2cq, 2cq+1 (b0) and
-      // 2cq+8, 2cq+9 (b1), as fp16 high and low parts; with kHiLo column gq
-      // carries the high part (gq < 4) or the remainder (gq >= 4) alone, in
-      // the *_hi registers
-      uint32_t p0_hi[kGroups], p0_lo[kGroups], p1_hi[kGroups], p1_lo[kGroups];
 #pragma unroll
-      for (int gg = 0; gg < kGroups; ++gg) {
-        float2 x01 = make_float2(0.0f, 0.0f), x89 = make_float2(0.0f, 0.0f);
-        if (qok) {
-          x01 = *reinterpret_cast<const float2*>(&myP[gg][qh][2 * cq]);
-          x89 = *reinterpret_cast<const float2*>(&myP[gg][qh][2 * cq + 8]);
+      for (int hf = 0; hf < kH; ++hf) {
+        // P'^T fragments (B): column gq = head qh, tokens 2cq, 2cq+1 (b0) and
+        // 2cq+8, 2cq+9 (b1) of this half, as fp16 high and low parts; with
+        // kHiLo column gq carries the high part (gq < 4) or the remainder
+        // (gq >= 4) alone, in the *_hi registers
+        uint32_t p0_hi[kGroups], p0_lo[kGroups], p1_hi[kGroups], p1_lo[kGroups];
+#pragma unroll
+        for (int gg = 0; gg < kGroups; ++gg) {
+          float2 x01 = make_float2(0.0f, 0.0f), x89 = make_float2(0.0f, 0.0f);
+          if (qok) {
+            x01 = *reinterpret_cast<const float2*>(&myP[gg][qh][kStep * hf + 2 * cq]);
+            x89 = *reinterpret_cast<const float2*>(&myP[gg][qh][kStep * hf + 2 * cq + 8]);
+          }
+          split_f16x2(x01.x, x01.y, p0_hi[gg], p0_lo[gg]);
+          split_f16x2(x89.x, x89.y, p1_hi[gg], p1_lo[gg]);
+          if constexpr (kHiLo) {
+            if (gq >= 4) { p0_hi[gg] = p0_lo[gg]; p1_hi[gg] = p1_lo[gg]; }
+          }
         }
-        split_f16x2(x01.x, x01.y, p0_hi[gg], p0_lo[gg]);
-        split_f16x2(x89.x, x89.y, p1_hi[gg], p1_lo[gg]);
-        if constexpr (kHiLo) {
-          if (gq >= 4) { p0_hi[gg] = p0_lo[gg]; p1_hi[gg] = p1_lo[gg]; }
-        }
-      }
-      // ---------------- O^T += V'^T P'^T, sum(P') against a tile of ones ----------------
-      {
-        const int vt = r0 + ldsm_tok;                        // this lane's ldmatrix row (token)
+        // ---------------- O^T += V'^T P'^T, sum(P') against a tile of ones ----------------
+        const int vt = r0 + kStep * hf + ldsm_tok;            // this lane's ldmatrix row (token)
         const uint32_t vrow = smem_u32(cV + vt * C::kRowBytes);
 #pragma unroll
         for (int cp = 0; cp < (kInt4 ? 2 : 4); ++cp) {        // pairs of 16-byte chunks
@@ -546,13 +578,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           } else {
             // chunk 2cp + h (32 channels) -> m-tiles 4cp + 2h + u: row g =
             // channel 4g + 2u (low nibble, 1032 + code), row g+8 = channel
-            // 4g + 2u + 1 (high nibble, 1152 + 16 code)
+            // 4g + 2u + 1 (high nibble, 1152 + 16 code); byte 0 of each
+            // 16-bit half is already in place (u = 0), byte 1 is moved down
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
-                const uint32_t yl = __byte_perm(r[2 * h], 0u, u ? 0x4341 : 0x4240);
-                const uint32_t yh = __byte_perm(r[2 * h + 1], 0u, u ? 0x4341 : 0x4240);
+                const uint32_t yl = u ? __byte_perm(r[2 * h], 0u, 0x4341) : r[2 * h];
+                const uint32_t yh = u ? __byte_perm(r[2 * h + 1], 0u, 0x4341) : r[2 * h + 1];
                 const uint32_t a0 = (yl & 0x000F000Fu) ^ 0x64086408u, a1 = (yl & 0x00F000F0u) ^ 0x64806480u;
                 const uint32_t a2 = (yh & 0x000F000Fu) ^ 0x64086408u, a3 = (yh & 0x00F000F0u) ^ 0x64806480u;
                 const int mt = 4 * cp + 2 * h + u;
@@ -563,12 +596,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
           }
         }
-      }
 #pragma unroll
-      for (int gg = 0; gg < kGroups; ++gg) {
-        mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_hi[gg], p1_hi[gg]);
-        if constexpr (!kHiLo)
-          mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_lo[gg], p1_lo[gg]);
+        for (int gg = 0; gg < kGroups; ++gg) {
+          mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_hi[gg], p1_hi[gg]);
+          if constexpr (!kHiLo)
+            mma_f16x4(sacc[gg], kOnesF16x2, kOnesF16x2, kOnesF16x2, kOnesF16x2, p0_lo[gg], p1_lo[gg]);
+        }
       }
       __syncwarp();                  // buffers reused by the next step
     }
@@ -718,13 +751,13 @@ bool decode_supported(int D, int group_ratio) { return D == kD && (group_ratio =
 // Split count: each split is a whole number of chunks (at least 4, to keep
 // the ring busy); among the counts that give at least two waves of resident
 // CTAs, take the smallest whose last wave is at least 90% full (else the
-// fullest). kCtasPerSm CTAs per SM are resident.
+// fullest). Cfg::kCtasPerSm CTAs per SM are resident.
 static int splits_for(int B, int Hkv, int L, int num_sms, bool int4) {
   const int ck = chunk_tokens(int4);
   const int chunks = (L + ck - 1) / ck;
   if (chunks == 0) return 1;
   const int64_t pairs = static_cast<int64_t>(B) * Hkv;
-  const int64_t slots = static_cast<int64_t>(num_sms) * kCtasPerSm;
+  const int64_t slots = static_cast<int64_t>(num_sms) * (int4 ? Cfg<true>::kCtasPerSm : Cfg<false>::kCtasPerSm);
   const int max_splits = max(1, min(64, chunks / 4));
   int best = 1;
   double best_fill = -1.0;
