@@ -35,6 +35,7 @@ QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 
 EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
             "qattn_prefill_mixed",
             "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc", "qattn_kv_append",
+            "qattn_attention_path_host_workspace_size", "qattn_attention_path_host",
             "qattn_device_error", "qattn_selftest_wait_timeout")
 
 # Fixed scratch of qattn_decode_kvq_noalloc (bytes).
@@ -72,6 +73,10 @@ def lib() -> C.CDLL:
         L.qattn_decode_kvq_noalloc.restype = i
         L.qattn_kv_append.argtypes = [P, i, i, i, i, i, i, i, P, P, i, i, P]
         L.qattn_kv_append.restype = i
+        L.qattn_attention_path_host_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.qattn_attention_path_host_workspace_size.restype = z
+        L.qattn_attention_path_host.argtypes = [P, P, P, i, i, i, i, i, i, P, i, i, f, P, i, P, z, P]
+        L.qattn_attention_path_host.restype = i
         L.qattn_device_error.argtypes, L.qattn_device_error.restype = [P], i
         L.qattn_selftest_wait_timeout.argtypes, L.qattn_selftest_wait_timeout.restype = [i, P], i
         _lib = L
@@ -168,6 +173,36 @@ def qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales,
                                    kv_block, int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse),
                                    _stream(stream))
     _check(st, "qattn_prefill_mixed")
+    return out
+
+
+def qattn_attention_path_host_workspace_size(B: int, H: int, N: int, D: int, layout: int, groups: int = 0) -> int:
+    return int(lib().qattn_attention_path_host_workspace_size(B, H, N, D, layout, groups))
+
+
+def qattn_attention_path_host(q, k, v, rot, layout: int, code_dtype: int, causal: bool, softmax_scale: float = 0.0,
+                              out=None, groups: int = 0, workspace=None, stream=None):
+    """The whole prefill path (rotate + quantize Q/K, quantize V, attention)
+    from HOST tensors: q, k, v are CPU bfloat16/float16 tensors (pinned for
+    the copies to overlap the compute), rot a CUDA float32 [D, D] tensor or
+    None. Returns `out`, a CPU bfloat16 tensor in the layout of q, complete
+    once `stream` has reached the end of the call's work."""
+    import torch
+    B, H, N, D = _dims(q, layout)
+    x_dtype = {torch.bfloat16: QATTN_BF16, torch.float16: QATTN_F16}[q.dtype]
+    for t in (q, k, v):
+        if t.is_cuda or not t.is_contiguous() or t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must be contiguous CPU tensors of one shape and dtype")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    dev = rot.device if rot is not None else torch.device("cuda", torch.cuda.current_device())
+    need = qattn_attention_path_host_workspace_size(B, H, N, D, layout, groups)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = lib().qattn_attention_path_host(_ptr(q), _ptr(k), _ptr(v), x_dtype, layout, B, H, N, D, _ptr(rot),
+                                         code_dtype, int(bool(causal)), float(softmax_scale), _ptr(out),
+                                         int(groups), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "qattn_attention_path_host")
     return out
 
 

@@ -12,7 +12,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqattn.so")
-SOURCES = ["qattn_abi.cu", "rotate_quant.cu", "prefill.cu", "decode.cu", "decode_noalloc.cu", "kv_append.cu"]
+SOURCES = ["qattn_abi.cu", "rotate_quant.cu", "prefill.cu", "decode.cu", "decode_noalloc.cu", "kv_append.cu",
+           "path_host.cu"]
 HEADERS = ["qattn_device.cuh", "qattn_internal.h"]
 
 NVCC_FLAGS = [

@@ -23,7 +23,8 @@
  *      packing).
  *
  * Conventions for every entry point:
- *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *   - All tensor pointers are DEVICE pointers owned by the caller (except
+ *     the host inputs and output of qattn_attention_path_host); the
  *     library never frees or keeps them. The library allocates no device
  *     memory per call (scratch for decode is passed in as `workspace`).
  *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
@@ -293,6 +294,57 @@ qattn_status_t qattn_decode_kvq_noalloc(const void* q, const void* k_cache, cons
 qattn_status_t qattn_kv_append(const void* x_new, int B, int H_kv, int n, int D,
                                qattn_dtype_t kv_dtype, int L, int L_max, void* cache,
                                void* scales, int kv_block, int group, qattn_stream_t stream);
+
+/*
+ * The whole prefill path from HOST buffers: rotation and block quantization
+ * of Q and K (qattn_rotate_block_quant with R, blocks of 128 and 256
+ * tokens), quantization of V (no rotation, 256-token blocks) and
+ * qattn_prefill on the codes -- the path of "MindIE-SD quantization", FA量化
+ * (rotate, quantize per block, attention in the low-precision domain,
+ * output in the original precision). The results are those of the four
+ * device calls made one after another on the same inputs, bit for bit.
+ *
+ * No counterpart on the pages: it moves the inputs to the GPU and the
+ * output back with the copies overlapped with the compute. The (b, h) heads
+ * are split into `groups` consecutive groups; group g is copied in on one
+ * internal stream, computed on `stream`, and copied out on another, so the
+ * copy-in of group g + 1 and the copy-out of group g - 1 run while group g
+ * is computed. Two workspace slots alternate between the groups.
+ *
+ * q, k, v: HOST pointers, x_dtype (QATTN_BF16 or QATTN_F16) [B, H, N, D] or
+ *          [B, N, H, D] (layout). Page-locked memory (cudaHostAlloc or
+ *          cudaHostRegister) is needed for the copies to overlap; pageable
+ *          memory gives the same results, slower.
+ * rot:     DEVICE pointer, float32 [D, D] row-major (y = x R), 16-byte
+ *          aligned; NULL quantizes Q and K without rotation.
+ * code_dtype: QATTN_INT8 or QATTN_FP8_E4M3 (Q, K and V alike).
+ * causal, softmax_scale: as for qattn_prefill (N_q = N_kv = N).
+ * out:     HOST pointer, bfloat16, same layout as q.
+ * groups:  number of head groups, 1..64; 0 selects 8. With layout BSND and
+ *          groups > B every group lies within one b (ceil(groups / B) head
+ *          ranges per b).
+ * workspace: DEVICE memory of at least
+ *          qattn_attention_path_host_workspace_size(B, H, N, D, layout,
+ *          groups) bytes, 256-byte aligned; contents need no initialisation.
+ *          Calls that share a workspace must not overlap.
+ * stream:  the compute stream; the call returns once everything is
+ *          enqueued, and `out` is complete when `stream` reaches the end of
+ *          this call's work. The library keeps two copy streams per device
+ *          (created on first use, never destroyed) and serialises the
+ *          enqueueing of concurrent calls.
+ * Errors: as the device calls (checked for the whole problem before
+ * anything is enqueued), QATTN_ERR_WORKSPACE for a missing or small
+ * workspace; QATTN_ERR_CUDA if a copy or launch fails to enqueue, in which
+ * case `out` is unspecified.
+ */
+size_t qattn_attention_path_host_workspace_size(int B, int H, int N, int D, qattn_layout_t layout,
+                                                int groups);
+qattn_status_t qattn_attention_path_host(const void* q, const void* k, const void* v,
+                                         qattn_dtype_t x_dtype, qattn_layout_t layout, int B, int H,
+                                         int N, int D, const float* rot, qattn_dtype_t code_dtype,
+                                         int causal, float softmax_scale, void* out, int groups,
+                                         void* workspace, size_t workspace_bytes,
+                                         qattn_stream_t stream);
 
 /*
  * Waits for `stream`, then reads and clears the per-device error word that
