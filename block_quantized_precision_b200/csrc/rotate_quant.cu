@@ -33,13 +33,14 @@ namespace qattn {
 namespace {
 
 // Threads per team (one team computes one block at a time): at D = 128,
-// 16 x 8 thread tiles for 128-token blocks (128 threads; two teams per CTA
-// share R, so one team's staging and coding overlap the other's FMA loop)
-// and 8 x 8 tiles for 256-token blocks (512 threads, one team); at D = 64,
-// 4 x 8 tiles (256 threads).
+// 8 x 8 thread tiles, 256 threads for 128-token blocks (two teams per CTA
+// share R, so one team's staging and coding overlap the other's FMA loop;
+// 256 threads keep the FMA pipe near 88 % busy while a team computes alone)
+// and 512 for 256-token blocks (one team); at D = 64, 4 x 8 tiles (256
+// threads).
 template <int D, int T>
 struct RotqThreads {
-  static constexpr int value = D == 128 ? (T == 256 ? 512 : 128) : 256;
+  static constexpr int value = D == 128 ? (T == 256 ? 512 : 256) : 256;
 };
 template <int D, int T>
 struct RotqTeams {
