@@ -114,6 +114,22 @@ __device__ __forceinline__ uint32_t code_of(float y, float scale, float rcp, boo
   }
 }
 
+// True on every thread of the team iff v is true on every thread of it
+// (a barrier with an AND reduction: the whole CTA for one team, else the
+// team's named barrier 1 + team).
+template <int kNT, int kTeams>
+__device__ __forceinline__ bool team_all(bool v, int team) {
+  if constexpr (kTeams == 1) return __syncthreads_and(v) != 0;
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.b32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<int>(v)), "r"(1 + team), "r"(kNT)
+      : "memory");
+  return r != 0;
+}
+
 // Maximum of v over the kNT threads of a team (ttid: thread within the team;
 // red: kNT / 32 floats of the team).
 template <int kNT, int kTeams = 1>
@@ -315,7 +331,7 @@ template <int D, int T, bool kInt8, bool kInt4>
 __global__ void __launch_bounds__(RotqThreads<D, T>::value * RotqTeams<D, T>::value, 1)
     rotq_kernel(const uint16_t* __restrict__ x, int is_bf16, int layout, int B, int H, int N,
                 const float* __restrict__ rot, uint8_t* __restrict__ codes,
-                float* __restrict__ scales) {
+                float* __restrict__ scales, int* err) {
   constexpr int kNT = RotqThreads<D, T>::value;
   constexpr int kTeams = RotqTeams<D, T>::value;
   constexpr int kCG = D / 8;               // column groups
@@ -330,6 +346,12 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value * RotqTeams<D, T>::va
   float* sX = smem + D * D + team * D * kXS;   // this team's [D][kXS]: sX[k * kXS + r] = x[r][k]
   __shared__ float red_all[kTeams][kNT / 32];
   float* red = red_all[team];
+  // start1: completes when team 0 has finished its first FMA loop (two teams)
+  __shared__ __align__(8) uint64_t start1;
+  if (kTeams > 1 && threadIdx.x == 0) {
+    mbar_init(&start1, kNT);
+    mbar_fence_init();
+  }
 
   for (int i = threadIdx.x; i < D * D / 4; i += kNT * kTeams)
     reinterpret_cast<float4*>(sR)[i] = reinterpret_cast<const float4*>(rot)[i];
@@ -368,16 +390,16 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value * RotqTeams<D, T>::va
   const int64_t first = blockIdx.x + static_cast<int64_t>(team) * gridDim.x;
   const int64_t step = static_cast<int64_t>(kTeams) * gridDim.x;
   if (kPrefetch && first < total) load_block(first);
-  // The second team starts once the first has finished the FMA loop of its
-  // first block, so that the teams' loops are out of phase (one team's
-  // loading, staging and coding run under the other's loop). Team 0 arrives
-  // exactly once, whether or not it has a block.
-  if constexpr (kTeams > 1) {
-    if (team == 1) named_bar_sync(3, 2 * kNT);
-    else if (first >= total) named_bar_arrive(3, 2 * kNT);
-  }
+  // With two teams, team 1 starts its first FMA loop once team 0 has
+  // finished its own, so that the teams' loops run out of phase and one
+  // team's loading, staging and coding overlap the other's loop. (Strict
+  // turn-taking of every loop measured slower.) Team 0 arrives only if team
+  // 1 has a block; the wait is bounded (QATTN_ERR_TIMEOUT, and the team
+  // stops).
+  const bool team1_has_work = blockIdx.x + static_cast<int64_t>(gridDim.x) < total;
+  int64_t it = 0;
 
-  for (int64_t blk_id = first; blk_id < total; blk_id += step) {
+  for (int64_t blk_id = first; blk_id < total; blk_id += step, ++it) {
     const int blk = static_cast<int>(blk_id % nblk);
     const int bh = static_cast<int>(blk_id / nblk);
     const int b = bh / H, h = bh % H;
@@ -400,6 +422,12 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value * RotqTeams<D, T>::va
     }
     team_sync<kNT, kTeams>(team);
     if (kPrefetch && blk_id + step < total) load_block(blk_id + step);
+    if constexpr (kTeams > 1) {
+      if (team == 1 && it == 0) {
+        const bool ok = mbar_wait(&start1, 0, nullptr, err);
+        if (!team_all<kNT, kTeams>(ok, team)) break;
+      }
+    }
 
     // acc[p][j]: rows rg*kRPT + 2p (.x) and + 2p + 1 (.y), column (j < 4 ?
     // c0 + j : c1 + j - 4); each is the float32 FMA chain over k ascending,
@@ -430,7 +458,9 @@ __global__ void __launch_bounds__(RotqThreads<D, T>::value * RotqTeams<D, T>::va
         }
       }
     }
-    if (kTeams > 1 && team == 0 && blk_id == first) named_bar_arrive(3, 2 * kNT);
+    if constexpr (kTeams > 1) {
+      if (team == 0 && it == 0 && team1_has_work) mbar_arrive(&start1);
+    }
     // the 8 values of row i (columns c0..c0+3, c1..c1+3)
     auto row8 = [&](int i, float (&f)[8]) {
 #pragma unroll
@@ -676,7 +706,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 }
 
 template <int D, int T, bool kInt8, bool kInt4 = false>
-cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
+cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err) {
   constexpr int kTeams = RotqTeams<D, T>::value;
   constexpr size_t smem = sizeof(float) * (D * D + kTeams * D * (T + 4));
   auto k = rotq_kernel<D, T, kInt8, kInt4>;
@@ -685,7 +715,7 @@ cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms) {
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
   const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
   k<<<grid, RotqThreads<D, T>::value * kTeams, smem, st>>>(static_cast<const uint16_t*>(a.x), a.is_bf16, a.layout, a.B,
-                                                a.H, a.N, a.rot, static_cast<uint8_t*>(a.codes), a.scales);
+                                                a.H, a.N, a.rot, static_cast<uint8_t*>(a.codes), a.scales, err);
   return cudaGetLastError();
 }
 
@@ -727,8 +757,8 @@ cudaError_t launch_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, in
 template <int D, int T>
 cudaError_t dispatch_t(const RotQuantArgs& a, cudaStream_t st, int num_sms, int* err) {
   if (a.rot) {
-    if (a.int4) return launch_rotq<D, T, true, true>(a, st, num_sms);
-    return a.int8 ? launch_rotq<D, T, true>(a, st, num_sms) : launch_rotq<D, T, false>(a, st, num_sms);
+    if (a.int4) return launch_rotq<D, T, true, true>(a, st, num_sms, err);
+    return a.int8 ? launch_rotq<D, T, true>(a, st, num_sms, err) : launch_rotq<D, T, false>(a, st, num_sms, err);
   }
   return a.int8 ? launch_quant<D, T, true>(a, st, num_sms, err) : launch_quant<D, T, false>(a, st, num_sms, err);
 }
