@@ -101,6 +101,38 @@ def test_cross_attention_lengths(orc):
         assert_close(bf16_to_f64(got_bits[b, h]), bf16_to_f64(ref[(b, h)][0]), vmax, "cross")
 
 
+@pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
+def test_key_scales_beyond_the_shared_memory_cache(orc, code_dtype):
+    """More than 512 K/V blocks (131072 keys): the block scales past the
+    first 512 come from global memory. Per-token log-normal magnitudes give
+    every block its own scale, and the last block is ragged."""
+    nkv = 513 * 256 + 100
+    p = synth.PrefillProblem("x", 1, 1, 200, 128, synth.BF16, code_dtype, synth.BNSD, causal=False,
+                             rotate=True, seed=310)
+    d = synth.make_prefill(p)
+    pk = synth.PrefillProblem("x", 1, 1, nkv, 128, synth.BF16, code_dtype, synth.BNSD, causal=False,
+                              rotate=True, seed=311, lognormal_sigma=0.7)
+    dk = synth.make_prefill(pk)
+    R = d["rot"]
+    r = torch.from_numpy(R).cuda()
+    qc, qs = qa.qattn_rotate_block_quant(dev_bits(d["q"], p.in_dtype), p.layout, r, 128, code_dtype)
+    kc, ks = qa.qattn_rotate_block_quant(dev_bits(dk["k"], p.in_dtype), p.layout, r, 256, code_dtype)
+    vc, vs = qa.qattn_rotate_block_quant(dev_bits(dk["v"], p.in_dtype), p.layout, None, 256, code_dtype)
+    assert ks.shape[-1] == 514
+    out = qa.qattn_prefill(qc, qs, kc, ks, vc, vs, code_dtype, p.layout, False)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    oq = orc.rotate_block_quant(d["q"], p.in_dtype, p.layout, R, 128, code_dtype)
+    ok_ = orc.rotate_block_quant(dk["k"], p.in_dtype, p.layout, R, 256, code_dtype)
+    ov = orc.rotate_block_quant(dk["v"], p.in_dtype, p.layout, None, 256, code_dtype)
+    assert np.array_equal(ks.cpu().numpy(), ok_[1]) and np.array_equal(vs.cpu().numpy(), ov[1])
+    rows = {(0, 0): [0, 57, 128, 199]}
+    ref = orc.prefill_rows(*oq, *ok_, *ov, code_dtype, p.layout, False, rows, want_f64=True)
+    got_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    vmax = dequant_v_max(ov[0], ov[1], code_dtype, p.layout, 0, 0, orc)
+    assert_close(bf16_to_f64(got_bits[0, 0][rows[(0, 0)]]), bf16_to_f64(ref[(0, 0)][0]), vmax, "long kv")
+
+
 @pytest.mark.parametrize("prob", ["tiny_fp8_b1h2n256d64", "int8_causal_b1h32n4096d128", "fp8_bsnd_b1h24n16384d128"])
 def test_full_size(orc, prob):
     """The stated problems at full size, in the benchmark's launch
