@@ -281,7 +281,11 @@ def gpu_arm(args):
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "ms_percentiles": {"p10": round(float(np.percentile(step_ms, 10)), 4),
+                           "p50": round(float(np.percentile(step_ms, 50)), 4),
+                           "p90": round(float(np.percentile(step_ms, 90)), 4)},
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; shapes and distributions of the stated problem)",
         "config": {"workload": p.name, "B": p.B, "H": p.H, "N": p.N, "D": p.D, "layout": "BNSD", "causal": True,
                    "codes": "int8", "rotation": "seeded orthogonal 128x128 on Q and K",
