@@ -217,11 +217,8 @@ def gpu_arm(args):
     step_launches = launches[0]
     per = np.array([[evs[i][k].elapsed_time(evs[i][k + 1]) for k in range(4)] for i in range(args.steps)])
     step_ms = per.sum(axis=1)
-    t = torch.tensor([float(step_ms.mean())], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    value = world * ops / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(float(step_ms.mean()), world, dev)
+    value = job_rate(ops, world, ms)
     kern_ms = per.mean(axis=0)
     qk_rows = p.B * p.H * p.N
     kernels = {
@@ -264,11 +261,9 @@ def gpu_arm(args):
     assert qa.qattn_device_error() == qa.QATTN_OK
     h2d = sum(host[n].numel() * 2 for n in host)
     d2h = out_host.numel() * 2
-    te = torch.tensor([float(np.mean(e2e_ms))], device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e = {"value": round(world * ops / (float(te.item()) * 1e-3) / 1e12, 3), "unit": "TOPS",
-           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(float(te.item()), 4),
+    te = max_over_ranks(float(np.mean(e2e_ms)), world, dev)
+    e2e = {"value": round(job_rate(ops, world, te), 3), "unit": "TOPS",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(te, 4),
            "api": "qattn_attention_path_host (host buffers, 8 head groups, copies overlapped with compute)"}
 
     extra = {}
@@ -304,6 +299,24 @@ def gpu_arm(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values of x (x itself on one rank): the
+    job's time is its slowest rank's. `device` holds the reduction tensor
+    (the GPU with NCCL, the CPU with gloo)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(ops_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput in TOPS: every rank processes ops_per_rank in
+    the (max-over-ranks) time ms."""
+    return world * ops_per_rank / (ms * 1e-3) / 1e12
 
 
 def load_traffic(kernel):
