@@ -338,11 +338,6 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Arrives on named barrier `id` (of `count` threads) without waiting.
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // Packed float32 pairs (sm_100): one instruction, two IEEE float32 results
 // ---------------------------------------------------------------------------
