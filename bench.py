@@ -356,6 +356,20 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
             ts.append(a.elapsed_time(b))
         return float(np.mean(ts))
 
+    def timeit_back_to_back(fn, reps):
+        # reps calls between two events: the host's per-call work overlaps the
+        # GPU's, so this is the launches' average device duration
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+
     # decode, INT8 and packed INT4 caches (inputs far larger than L2)
     for key, p in (("decode_int8kv", synth.INT8_KV_DECODE), ("decode_int4kv", synth.INT4_KV_DECODE)):
         dd = synth.make_decode(p)
@@ -371,10 +385,13 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         out = torch.empty((p.B, p.Hq, 1, p.D), dtype=torch.bfloat16, device=dev)
         ws = torch.empty(max(16, qa.qattn_decode_workspace_size(p.B, p.Hq, p.Hkv, p.L, p.D)), dtype=torch.uint8, device=dev)
         fn = lambda: qa.qattn_decode_kvq(q, k, v, ks, vs, kvt, kv_block=p.kv_block, group=p.group, out=out, workspace=ws)
-        ms = timeit(fn, n)
+        ms_single = timeit(fn, n)
+        ms = timeit_back_to_back(fn, 10)
         by = decode_bytes(p)
         gbs = by / (ms * 1e-3) / 1e9
         res[key] = {"workload": p.name, "ms": round(ms, 4), "GB/s": round(gbs, 1), "bytes": by,
+                    "timing": "10 calls back to back between two events (cache far larger than L2)",
+                    "ms_single_call": round(ms_single, 4),
                     "roofline": {"bound": "hbm", "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
         del k, v, dd
         torch.cuda.empty_cache()

@@ -724,7 +724,7 @@ cudaError_t launch_g(const DecodeArgs& a, const DecodeParams& p, cudaStream_t st
   if (!make_cache_map<kInt4>(&mk, a.k, a.B, a.Hkv, a.L) || !make_cache_map<kInt4>(&mv, a.v, a.B, a.Hkv, a.L))
     return cudaErrorInvalidValue;
   auto k = decode_kernel<G, kInt4, kGroups>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<kInt4>::kSmemBytes);
+  cudaError_t e = set_max_dyn_smem(reinterpret_cast<const void*>(k), Cfg<kInt4>::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.splits, p.Hkv, p.B);
   k<<<grid, kThreads, Cfg<kInt4>::kSmemBytes, st>>>(mk, mv, p);

@@ -38,6 +38,7 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include <atomic>
 #include <climits>
 
 #include "qattn_device.cuh"
@@ -959,14 +960,19 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t st, int* err) {
   p.err = err;
   auto k = prefill_kernel<D, kQKCode, kVCode>;
   constexpr int kSmem = Smem<D, kQKCode, kVCode>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  cudaError_t e = set_max_dyn_smem(reinterpret_cast<const void*>(k), kSmem);
   if (e != cudaSuccess) return e;
   // The register split inside the kernel needs at least kRegsNeeded
-  // registers per thread at launch; never launch with fewer.
-  cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, k);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs < kRegsNeeded) return cudaErrorInvalidConfiguration;
+  // registers per thread at launch; never launch with fewer. (The count is
+  // a property of the compiled kernel: looked up once.)
+  static std::atomic<int> regs{-1};
+  if (regs.load() < 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, k);
+    if (e != cudaSuccess) return e;
+    regs.store(fa.numRegs);
+  }
+  if (regs.load() < kRegsNeeded) return cudaErrorInvalidConfiguration;
   const int64_t grid = static_cast<int64_t>(p.npairs) * a.B * a.H;
   k<<<static_cast<unsigned>(grid), kThreads, kSmem, st>>>(mq, mk, mv, p);
   return cudaGetLastError();

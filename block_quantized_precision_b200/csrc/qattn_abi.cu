@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/qattn.h"
 #include "qattn_device.cuh"
@@ -121,6 +122,21 @@ bool encode_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t*
 bool encode_map_u16(CUtensorMap* map, int rank, const void* base, const uint64_t* dims, const uint64_t* strides,
                     const uint32_t* box, CUtensorMapSwizzle swizzle) {
   return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, rank, base, dims, strides, box, swizzle);
+}
+
+cudaError_t set_max_dyn_smem(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;   // kernel -> devices (bit per id < 64) already set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  std::lock_guard<std::mutex> lock(mu);
+  uint64_t& mask = done[func];
+  if (bit != 0 && (mask & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) mask |= bit;
+  return e;
 }
 
 cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err) {

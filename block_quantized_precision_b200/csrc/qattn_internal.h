@@ -88,4 +88,9 @@ cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err);
 
+// Sets kernel `func`'s dynamic shared-memory limit on the current device the
+// first time it is asked for there (the attribute stays set for the life of
+// the context), so that launches do not repeat the runtime call.
+cudaError_t set_max_dyn_smem(const void* func, int bytes);
+
 }  // namespace qattn

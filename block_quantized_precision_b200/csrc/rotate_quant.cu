@@ -710,7 +710,7 @@ cudaError_t launch_rotq(const RotQuantArgs& a, cudaStream_t st, int num_sms, int
   constexpr int kTeams = RotqTeams<D, T>::value;
   constexpr size_t smem = sizeof(float) * (D * D + kTeams * D * (T + 4));
   auto k = rotq_kernel<D, T, kInt8, kInt4>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = set_max_dyn_smem(reinterpret_cast<const void*>(k), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
   const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
@@ -745,7 +745,7 @@ cudaError_t launch_quant(const RotQuantArgs& a, cudaStream_t st, int num_sms, in
   using L = QuantSmem<D, T>;
   auto k = a.int4 ? (a.is_bf16 ? quant_kernel<D, T, true, true, true> : quant_kernel<D, T, true, false, true>)
                   : (a.is_bf16 ? quant_kernel<D, T, kInt8, true, false> : quant_kernel<D, T, kInt8, false, false>);
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+  cudaError_t e = set_max_dyn_smem(reinterpret_cast<const void*>(k), L::kBytes);
   if (e != cudaSuccess) return e;
   const int64_t nblocks = static_cast<int64_t>(a.B) * a.H * ((a.N + T - 1) / T);
   const int grid = static_cast<int>(nblocks < num_sms ? nblocks : num_sms);
