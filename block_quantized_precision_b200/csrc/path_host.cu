@@ -198,6 +198,14 @@ qattn_status_t qattn_attention_path_host(const void* q, const void* k, const voi
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(P->enqueue);
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // On a failure after the first copy was enqueued, the copies already on
+  // the internal streams finish before the error is returned, so none of
+  // them touches the caller's buffers afterwards.
+  auto fail = [&](qattn_status_t status) {
+    cudaStreamSynchronize(P->in);
+    cudaStreamSynchronize(P->out);
+    return status;
+  };
   // the copies start after the work already on `stream` (earlier users of
   // the workspace and of the host buffers)
   if (!ok(cudaEventRecord(P->start, st)) || !ok(cudaStreamWaitEvent(P->in, P->start, 0)) ||
@@ -210,16 +218,16 @@ qattn_status_t qattn_attention_path_host(const void* q, const void* k, const voi
     char* base = static_cast<char*>(workspace) + (gi % 2) * sl.bytes;
     if (gi >= 2) {
       const int e2 = static_cast<int>((gi - 2) % kMaxGroups);
-      if (!ok(cudaStreamWaitEvent(P->in, P->ev_comp[e2], 0))) return QATTN_ERR_CUDA;   // slot inputs consumed
+      if (!ok(cudaStreamWaitEvent(P->in, P->ev_comp[e2], 0))) return fail(QATTN_ERR_CUDA);   // slot inputs consumed
     }
     if (!ok(copy_group(g, N, H, D, es, base + sl.xq, q, true, P->in)) ||
         !ok(copy_group(g, N, H, D, es, base + sl.xk, k, true, P->in)) ||
         !ok(copy_group(g, N, H, D, es, base + sl.xv, v, true, P->in)) ||
         !ok(cudaEventRecord(P->ev_in[e], P->in)) || !ok(cudaStreamWaitEvent(st, P->ev_in[e], 0)))
-      return QATTN_ERR_CUDA;
+      return fail(QATTN_ERR_CUDA);
     if (gi >= 2) {
       const int e2 = static_cast<int>((gi - 2) % kMaxGroups);
-      if (!ok(cudaStreamWaitEvent(st, P->ev_out[e2], 0))) return QATTN_ERR_CUDA;       // slot output copied out
+      if (!ok(cudaStreamWaitEvent(st, P->ev_out[e2], 0))) return fail(QATTN_ERR_CUDA);       // slot output copied out
     }
     float* qs = reinterpret_cast<float*>(base + sl.qs);
     float* ks = reinterpret_cast<float*>(base + sl.ks);
@@ -235,14 +243,14 @@ qattn_status_t qattn_attention_path_host(const void* q, const void* k, const voi
     if (s == QATTN_OK)
       s = qattn_prefill(base + sl.qc, qs, base + sl.kc, ks, base + sl.vc, vs, code_dtype, layout, g.Bp, g.Hp, N, N,
                         D, 128, 256, causal, softmax_scale, base + sl.out, nullptr, stream);
-    if (s != QATTN_OK) return s;
+    if (s != QATTN_OK) return fail(s);
     if (!ok(cudaEventRecord(P->ev_comp[e], st)) || !ok(cudaStreamWaitEvent(P->out, P->ev_comp[e], 0)) ||
         !ok(copy_group(g, N, H, D, es, out, base + sl.out, false, P->out)) ||
         !ok(cudaEventRecord(P->ev_out[e], P->out)))
-      return QATTN_ERR_CUDA;
+      return fail(QATTN_ERR_CUDA);
   }
   const int last = static_cast<int>((gs.size() - 1) % kMaxGroups);
-  return ok(cudaStreamWaitEvent(st, P->ev_out[last], 0)) ? QATTN_OK : QATTN_ERR_CUDA;
+  return ok(cudaStreamWaitEvent(st, P->ev_out[last], 0)) ? QATTN_OK : fail(QATTN_ERR_CUDA);
 }
 
 }  // extern "C"

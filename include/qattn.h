@@ -335,7 +335,8 @@ qattn_status_t qattn_kv_append(const void* x_new, int B, int H_kv, int n, int D,
  * Errors: as the device calls (checked for the whole problem before
  * anything is enqueued), QATTN_ERR_WORKSPACE for a missing or small
  * workspace; QATTN_ERR_CUDA if a copy or launch fails to enqueue, in which
- * case `out` is unspecified.
+ * case `out` is unspecified and the copies already enqueued have finished
+ * when the call returns (none still reads or writes the caller's buffers).
  */
 size_t qattn_attention_path_host_workspace_size(int B, int H, int N, int D, qattn_layout_t layout,
                                                 int groups);
