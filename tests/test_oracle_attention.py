@@ -42,7 +42,8 @@ def _bf16_to_f64(bits):
 def test_running_softmax_equals_exact_softmax_without_quantization(orc, layout, causal):
     """float32 'codes', random per-block scales, probabilities not rounded:
     the tiled running softmax must equal the one-shot softmax (several key
-    tiles and a ragged tail)."""
+    tiles and a ragged tail), and its LSE the float64 log-sum-exp of the
+    scaled scores (natural log)."""
     B, H, N, D = 1, 2, 300, 64
     rng = np.random.default_rng(21)
     q = rng.standard_normal((B, H, N, D)).astype(np.float32)
@@ -54,7 +55,7 @@ def test_running_softmax_equals_exact_softmax_without_quantization(orc, layout, 
     rows = list(range(N))
     res = orc.prefill_rows(_store(q, layout), qs, _store(k, layout), ks, _store(v, layout), vs,
                            orc.F32, layout, causal, {(0, h): rows for h in range(H)},
-                           p_quant=False, want_f64=True)
+                           p_quant=False, want_f64=True, want_lse=True)
     tok = np.arange(N)
     for h in range(H):
         qd = q[0, h].astype(np.float64) * qs[0, h, tok // 128, None]
@@ -63,6 +64,12 @@ def test_running_softmax_equals_exact_softmax_without_quantization(orc, layout, 
         ref = _ref_attention(qd, kd, vd, causal, 1.0 / np.sqrt(D))
         got = res[(0, h)][1]
         assert np.abs(got - ref).max() <= 2e-5 * np.abs(vd).max()
+        sc = (qd @ kd.T) / np.sqrt(D)
+        if causal:
+            sc = np.where(np.tril(np.ones(sc.shape, bool)), sc, -np.inf)
+        mx = sc.max(axis=1)
+        ref_lse = mx + np.log(np.exp(sc - mx[:, None]).sum(axis=1))
+        assert np.abs(res[(0, h)][2] - ref_lse).max() <= 1e-4 * max(1.0, np.abs(ref_lse).max())
 
 
 @pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
