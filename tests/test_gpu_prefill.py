@@ -102,6 +102,28 @@ def test_cross_attention_lengths(orc):
 
 
 @pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
+def test_explicit_softmax_scale(orc, code_dtype):
+    """A softmax scale other than 1/sqrt(D), causal, ragged: CUDA path and
+    oracle given the same scale."""
+    p = synth.PrefillProblem("x", 1, 2, 300, 128, synth.BF16, code_dtype, synth.BNSD, causal=True,
+                             rotate=True, seed=320)
+    d = synth.make_prefill(p)
+    (qc, qs), (kc, ks), (vc, vs) = gpu_quant_all(d)
+    out = qa.qattn_prefill(qc, qs, kc, ks, vc, vs, code_dtype, p.layout, True, softmax_scale=0.37)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    oq = orc.rotate_block_quant(d["q"], p.in_dtype, p.layout, d["rot"], 128, code_dtype)
+    ok_ = orc.rotate_block_quant(d["k"], p.in_dtype, p.layout, d["rot"], 256, code_dtype)
+    ov = orc.rotate_block_quant(d["v"], p.in_dtype, p.layout, None, 256, code_dtype)
+    rows = {(0, h): list(range(p.N)) for h in range(p.H)}
+    ref = orc.prefill_rows(*oq, *ok_, *ov, code_dtype, p.layout, True, rows, softmax_scale=0.37, want_f64=True)
+    got_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    for (b, h) in rows:
+        vmax = dequant_v_max(ov[0], ov[1], code_dtype, p.layout, b, h, orc)
+        assert_close(bf16_to_f64(got_bits[b, h]), bf16_to_f64(ref[(b, h)][0]), vmax, "scale 0.37")
+
+
+@pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
 def test_key_scales_beyond_the_shared_memory_cache(orc, code_dtype):
     """More than 512 K/V blocks (131072 keys): the block scales past the
     first 512 come from global memory. Per-token log-normal magnitudes give

@@ -72,6 +72,24 @@ def test_running_softmax_equals_exact_softmax_without_quantization(orc, layout, 
         assert np.abs(res[(0, h)][2] - ref_lse).max() <= 1e-4 * max(1.0, np.abs(ref_lse).max())
 
 
+def test_explicit_softmax_scale(orc):
+    """A given softmax scale replaces 1/sqrt(D): float32 'codes', P not
+    rounded, against float64 softmax at that scale."""
+    B, H, N, D = 1, 1, 200, 64
+    rng = np.random.default_rng(23)
+    q = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    k = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    v = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    ones_q, ones_kv = np.ones((B, H, 2), np.float32), np.ones((B, H, 1), np.float32)
+    rows = {(0, 0): list(range(N))}
+    for scale in (0.37, 0.0):
+        res = orc.prefill_rows(q, ones_q, k, ones_kv, v, ones_kv, orc.F32, synth.BNSD, False, rows,
+                               softmax_scale=scale, p_quant=False, want_f64=True)
+        want = _ref_attention(q[0, 0].astype(np.float64), k[0, 0].astype(np.float64), v[0, 0].astype(np.float64),
+                              False, scale if scale > 0 else 1.0 / np.sqrt(D))
+        assert np.abs(res[(0, 0)][1] - want).max() <= 2e-5 * np.abs(v).max()
+
+
 @pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
 def test_constant_v_reproduces_v(orc, code_dtype):
     """Every value row equal: the output is that row whatever the weights,
