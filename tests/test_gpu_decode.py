@@ -25,7 +25,7 @@ def _vmax(d, p, b, hk):
     return float((m * sc).max())
 
 
-def _run(orc, p, d, heads):
+def _run(orc, p, d, heads, softmax_scale=0.0):
     q = dev(d["q"]).view(torch.bfloat16)
     k, v = dev(d["k"]), dev(d["v"])
     if p.kv_dtype == synth.INT8:
@@ -34,12 +34,13 @@ def _run(orc, p, d, heads):
     else:
         ks, vs = dev(d["k_scales"]).view(torch.float16), dev(d["v_scales"]).view(torch.float16)
         kv = qa.QATTN_INT4_PACKED
-    out = qa.qattn_decode_kvq(q, k, v, ks, vs, kv, kv_block=p.kv_block, group=p.group)
+    out = qa.qattn_decode_kvq(q, k, v, ks, vs, kv, kv_block=p.kv_block, group=p.group, softmax_scale=softmax_scale)
     torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
     got = out.view(torch.int16).cpu().numpy().view(np.uint16)
     ref_bits, ref = orc.decode(d["q"], d["k"], d["v"], d["k_scales"], d["v_scales"], p.kv_dtype, p.Hkv,
-                               heads=heads, kv_block=p.kv_block, group=p.group, want_f64=True)
+                               heads=heads, kv_block=p.kv_block, group=p.group, softmax_scale=softmax_scale,
+                               want_f64=True)
     g = p.Hq // p.Hkv
     for (b, h) in heads:
         # both sides round their output to bfloat16; compare those outputs
@@ -54,6 +55,15 @@ def test_lengths(orc, kv_dtype, L):
     p = synth.scaled(base, B=2, L=L, seed=40 + L)
     d = synth.make_decode(p)
     _run(orc, p, d, [(b, h) for b in range(2) for h in range(p.Hq)])
+
+
+@pytest.mark.parametrize("kv_dtype", [synth.INT8, synth.INT4_PACKED])
+def test_explicit_softmax_scale(orc, kv_dtype):
+    """A softmax scale other than 1/sqrt(D), given to both sides."""
+    base = synth.INT8_KV_DECODE if kv_dtype == synth.INT8 else synth.INT4_KV_DECODE
+    p = synth.scaled(base, B=2, Hq=8, Hkv=2, L=900, seed=61)
+    d = synth.make_decode(p)
+    _run(orc, p, d, [(b, h) for b in range(2) for h in range(p.Hq)], softmax_scale=0.21)
 
 
 @pytest.mark.parametrize("kv_dtype", [synth.INT8, synth.INT4_PACKED])

@@ -67,6 +67,23 @@ def test_pageable_host_memory_and_no_rotation():
     assert torch.equal(out.view(torch.int16), want.view(torch.int16))
 
 
+def test_f16_inputs():
+    """fp16 Q/K/V through the host path: the same bytes as the device calls."""
+    p = synth.PrefillProblem("host", 1, 4, 333, 128, synth.F16, synth.INT8, synth.BNSD, causal=True,
+                             rotate=True, seed=960)
+    d = synth.make_prefill(p)
+    rot = dev(d["rot"])
+    codes = [qa.qattn_rotate_block_quant(dev_bits(d[n], p.in_dtype), p.layout, r, blk, p.code_dtype)
+             for n, blk, r in (("q", 128, rot), ("k", 256, rot), ("v", 256, None))]
+    want = qa.qattn_prefill(*codes[0], *codes[1], *codes[2], p.code_dtype, p.layout, p.causal)
+    torch.cuda.synchronize()
+    host = [torch.from_numpy(np.ascontiguousarray(d[n]).view(np.int16)).view(torch.float16).pin_memory()
+            for n in ("q", "k", "v")]
+    out = qa.qattn_attention_path_host(*host, rot, p.layout, p.code_dtype, p.causal, groups=3)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), want.cpu().view(torch.int16))
+
+
 def test_small_workspace_is_rejected():
     q = torch.zeros((1, 2, 128, 128), dtype=torch.bfloat16).pin_memory()
     need = qa.qattn_attention_path_host_workspace_size(1, 2, 128, 128, qa.QATTN_BNSD, 2)
