@@ -75,8 +75,10 @@ def test_gqa_ratios(orc, kv_dtype, Hq, Hkv):
     _run(orc, p, d, [(b, h) for b in range(3) for h in range(Hq)])
 
 
-def test_int4_two_groups_per_row(orc):
-    p = synth.scaled(synth.INT4_KV_DECODE, B=2, L=500, group=64, seed=61)
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (8, 4), (16, 2)])
+def test_int4_two_groups_per_row(orc, Hq, Hkv):
+    """Scale groups of 64 channels (two per row) at every query-head ratio."""
+    p = synth.scaled(synth.INT4_KV_DECODE, B=2, Hq=Hq, Hkv=Hkv, L=500, group=64, seed=61 + Hq + Hkv)
     d = synth.make_decode(p)
     _run(orc, p, d, [(b, h) for b in range(2) for h in range(p.Hq)])
 
