@@ -266,13 +266,17 @@ def gpu_arm(args):
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(te, 4),
            "api": "qattn_attention_path_host (host buffers, 8 head groups, copies overlapped with compute)"}
 
+    keep = {"int8_causal": {"problem": p, "data": d,
+                            "out": bufs["out"].view(torch.int16).cpu().numpy().view(np.uint16)}}
     extra = {}
     if not args.no_extra:
-        extra = extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak, flush=l2_flush)
+        extra = extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak, flush=l2_flush,
+                                   keep=keep)
 
-    cpu = None
+    cpu, errors = None, None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(p, d, args.cpu_seconds)
+        errors = parity_errors(keep)
 
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -294,6 +298,8 @@ def gpu_arm(args):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if errors is not None:
+        line["errors"] = errors
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -336,9 +342,15 @@ def load_traffic(kernel):
         return None
 
 
-def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak, flush=None):
+def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_peak, flush=None, keep=None):
+    """Decode, KV append, the FP8 long prefill (first class: its own roofline
+    and its rotation/quantization reported apart), mixed and INT4 prefill.
+    `keep` (a dict) receives the outputs that the CPU leg samples for the
+    error figures."""
     import torch
     res = {}
+    keep = {} if keep is None else keep
+    pk_bf16 = int8_peak / 2.0
     n = max(5, args.steps // 2)
 
     def timeit(fn, reps, flush=None):
@@ -389,10 +401,15 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         ms = timeit_back_to_back(fn, 10)
         by = decode_bytes(p)
         gbs = by / (ms * 1e-3) / 1e9
+        gbs_single = by / (ms_single * 1e-3) / 1e9
         res[key] = {"workload": p.name, "ms": round(ms, 4), "GB/s": round(gbs, 1), "bytes": by,
                     "timing": "10 calls back to back between two events (cache far larger than L2)",
-                    "ms_single_call": round(ms_single, 4),
-                    "roofline": {"bound": "hbm", "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
+                    "ms_single_call": round(ms_single, 4), "GB/s_single_call": round(gbs_single, 1),
+                    "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": round(gbs / hbm_peak, 4), "frac_single_call": round(gbs_single / hbm_peak, 4),
+                                 "traffic": load_traffic(key)}}
+        keep[key] = {"problem": p, "data": {nm: dd[nm] for nm in ("q", "k_scales", "v_scales")},
+                     "k": dd["k"], "v": dd["v"], "out": out.view(torch.int16).cpu().numpy().view(np.uint16)}
         del k, v, dd
         torch.cuda.empty_cache()
 
@@ -420,6 +437,36 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                     "roofline": {"bound": "hbm", "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)}}
         del cache, scl, xn
 
+    # KV-cache append at bandwidth scale: a 4096-token prefill's K and V
+    # written into empty caches of the decode problems' shapes (block-aligned:
+    # no earlier codes to requantize); bytes = new rows read once + codes and
+    # scales written once
+    for key, p, kvt in (("kv_append_prefill_int8", synth.INT8_KV_DECODE, qa.QATTN_INT8),
+                        ("kv_append_prefill_int4", synth.INT4_KV_DECODE, qa.QATTN_INT4_PACKED)):
+        n_new = 4096
+        g = torch.Generator(device=dev).manual_seed(8)
+        xs = [torch.randn((p.B, p.Hkv, n_new, p.D), generator=g, device=dev).to(torch.bfloat16) for _ in range(2)]
+        if kvt == qa.QATTN_INT8:
+            caches = [torch.zeros((p.B, p.Hkv, n_new, p.D), dtype=torch.int8, device=dev) for _ in range(2)]
+            scls = [torch.zeros((p.B, p.Hkv, n_new // 256), dtype=torch.float32, device=dev) for _ in range(2)]
+        else:
+            caches = [torch.zeros((p.B, p.Hkv, n_new, p.D // 2), dtype=torch.uint8, device=dev) for _ in range(2)]
+            scls = [torch.zeros((p.B, p.Hkv, n_new, p.D // p.group), dtype=torch.float16, device=dev)
+                    for _ in range(2)]
+        by = sum(xs[i].numel() * 2 + caches[i].numel() + scls[i].numel() * scls[i].element_size() for i in range(2))
+
+        def fn(xs=xs, caches=caches, scls=scls, kvt=kvt, p=p):
+            for i in range(2):
+                qa.qattn_kv_append(xs[i], caches[i], scls[i], 0, kvt, group=p.group)
+        ms = timeit(fn, n, flush)
+        gbs = by / (ms * 1e-3) / 1e9
+        res[key] = {"workload": "%s shape, K and V of a %d-token prefill into empty caches" % (p.name, n_new),
+                    "ms": round(ms, 4), "GB/s": round(gbs, 1), "bytes": by,
+                    "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": round(gbs / hbm_peak, 4)}}
+        del xs, caches, scls
+        torch.cuda.empty_cache()
+
     # FP8 long-sequence prefill path (inputs larger than L2)
     p = synth.FP8_LONG
     d = synth.make_prefill(p)
@@ -431,6 +478,11 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
     pf = lambda: qa.qattn_prefill(codes["q"][0], codes["q"][1], codes["k"][0], codes["k"][1], codes["v"][0],
                                   codes["v"][1], p.code_dtype, p.layout, p.causal, out=out)
     ms_pf = timeit(pf, n)
+    k1_ms = {}
+    for nm in ("q", "k", "v"):
+        k1_ms[nm] = timeit(lambda nm=nm: qa.qattn_rotate_block_quant(
+            x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256, p.code_dtype, codes[nm][0],
+            codes[nm][1]), n)
 
     def full():
         for nm in ("q", "k", "v"):
@@ -439,12 +491,41 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         pf()
     ms_full = timeit(full, n)
     ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
+    tf = ops / (ms_pf * 1e-3) / 1e12
+    # K1 (rotate + quantize Q and K, quantize V): 3 bytes per element of each
+    # tensor (2 read, 1 written) and D FMAs per element of Q and K
+    elems = p.B * p.H * p.N * p.D
+    k1_bytes, k1_fma = 3 * 3 * elems, 2 * elems * p.D
+    k1_total = sum(k1_ms.values())
+    k1_floor_ms = max(k1_bytes / (hbm_peak * 1e9), 2 * k1_fma / (fp32_peak * 1e12)) * 1e3
     res["prefill_fp8_long"] = {"workload": p.name, "ms_prefill": round(ms_pf, 4), "ms_path": round(ms_full, 4),
-                               "TFLOPS_prefill": round(ops / (ms_pf * 1e-3) / 1e12, 1),
+                               "TFLOPS_prefill": round(tf, 1),
                                "TFLOPS_path": round(ops / (ms_full * 1e-3) / 1e12, 1),
-                               "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TFLOP/s",
-                                            "frac": round(ops / (ms_pf * 1e-3) / 1e12 / int8_peak, 4)}}
-    del x, codes, out, d
+                               "roofline": {"kernel": "prefill", "bound": "tensor", "achieved": round(tf, 1),
+                                            "peak": int8_peak, "unit": "TFLOP/s", "frac": round(tf / int8_peak, 4),
+                                            "traffic": load_traffic("prefill_fp8_long"),
+                                            "peak_source": "measured bf16 burst x 2 (FP8:bf16 nominal ratio)"},
+                               "k1": {"ms_rotq_q": round(k1_ms["q"], 4), "ms_rotq_k": round(k1_ms["k"], 4),
+                                      "ms_quant_v": round(k1_ms["v"], 4), "ms_total": round(k1_total, 4),
+                                      "bytes": k1_bytes, "fma": k1_fma,
+                                      "GB/s": round(k1_bytes / (k1_total * 1e-3) / 1e9, 1),
+                                      "TFLOP/s_rotation": round(2 * k1_fma / ((k1_ms["q"] + k1_ms["k"]) * 1e-3) / 1e12, 2),
+                                      "roofline": {"bound": "alu (FP32 FMA) / hbm, the larger time",
+                                                   "floor_ms": round(k1_floor_ms, 4),
+                                                   "frac": round(k1_floor_ms / k1_total, 4)}}}
+    keep["prefill_fp8_long"] = {"problem": p, "data": d, "out": out.view(torch.int16).cpu().numpy().view(np.uint16)}
+    del x, codes, out
+
+    # The tiny FP8 problem (parity only: launch-bound)
+    p = synth.TINY_FP8
+    d = synth.make_prefill(p)
+    x = {nm: torch.from_numpy(d[nm].view(np.int16)).to(dev).view(torch.float16) for nm in ("q", "k", "v")}
+    codes = {nm: qa.qattn_rotate_block_quant(x[nm], p.layout, None, 128 if nm == "q" else 256, p.code_dtype)
+             for nm in ("q", "k", "v")}
+    out = qa.qattn_prefill(*codes["q"], *codes["k"], *codes["v"], p.code_dtype, p.layout, p.causal)
+    torch.cuda.synchronize()
+    keep["tiny_fp8"] = {"problem": p, "data": d, "out": out.view(torch.int16).cpu().numpy().view(np.uint16)}
+    del x, codes, out
 
     # Mixed precision on the INT8 causal problem: Q/K INT8 (rotated), V in
     # packed INT4 or e4m3 (L2 flushed before every timed call)
@@ -469,6 +550,29 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                     "ms_prefill": round(ms_pf, 4), "TOPS_prefill": round(tops, 1),
                     "ms_quant_v": round(ms_qv, 4), "GB/s_quant_v": round(v_bytes / (ms_qv * 1e-3) / 1e9, 1),
                     "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TOPS", "frac": round(tops / int8_peak, 4)}}
+
+    # The dequantize-first comparison path on the same codes: bf16 = code x
+    # scale written to HBM, then attention on the 16-bit tensor-core path
+    # (P unquantized); timed beside the INT8 prefill
+    cq = {nm: qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
+                                          qa.QATTN_INT8) for nm in ("q", "k", "v")}
+    deq = {nm: torch.empty(p.shape(), dtype=torch.bfloat16, device=dev) for nm in ("q", "k", "v")}
+    dq = lambda: [qa.qattn_dequant_bf16(*cq[nm], qa.QATTN_INT8, p.layout, 128 if nm == "q" else 256, out=deq[nm])
+                  for nm in ("q", "k", "v")]
+    ab = lambda: qa.qattn_attention_bf16(deq["q"], deq["k"], deq["v"], p.layout, p.causal, out=out)
+    i8 = lambda: qa.qattn_prefill(*cq["q"], *cq["k"], *cq["v"], qa.QATTN_INT8, p.layout, p.causal, out=out)
+    ms_dq, ms_ab, ms_i8 = timeit(dq, n, flush), timeit(ab, n, flush), timeit(i8, n, flush)
+    dq_bytes = 3 * x["q"].numel() * 3
+    res["ablation_dequant_bf16"] = {
+        "workload": "%s: INT8 codes dequantized to bf16, then bf16 attention (P unquantized)" % p.name,
+        "ms_dequant": round(ms_dq, 4), "GB/s_dequant": round(dq_bytes / (ms_dq * 1e-3) / 1e9, 1),
+        "ms_attention_bf16": round(ms_ab, 4), "TFLOPS_attention_bf16": round(ops / (ms_ab * 1e-3) / 1e12, 1),
+        "ms_path": round(ms_dq + ms_ab, 4), "ms_int8_prefill": round(ms_i8, 4),
+        "int8_speedup_over_path": round((ms_dq + ms_ab) / ms_i8, 3),
+        "roofline": {"bound": "tensor", "peak": pk_bf16, "unit": "TFLOP/s",
+                     "frac": round(ops / (ms_ab * 1e-3) / 1e12 / pk_bf16, 4),
+                     "peak_source": "measured bf16 burst (cuBLAS)"}}
+    del cq, deq
 
     # INT4 Q/K/V on the same problem (Q/K rotated), widened to INT8 on chip
     c4 = {nm: qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
@@ -496,16 +600,17 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(p, d, heads):
+def oracle_sample(p, d, heads, row_chunk=128):
     """The oracle on `heads` of the workload: its own rotate+quantize of Q,
-    K, V and quantized attention for every row of those heads."""
+    K, V and quantized attention for every row of those heads (row_chunk
+    rows per parallel job; None: one job per head)."""
     import oracle
     hs = [(0, h) for h in range(heads)]
     oq = oracle.rotate_block_quant(d["q"], p.in_dtype, p.layout, d["rot"], 128, p.code_dtype, heads=hs)
     ok_ = oracle.rotate_block_quant(d["k"], p.in_dtype, p.layout, d["rot"], 256, p.code_dtype, heads=hs)
     ov = oracle.rotate_block_quant(d["v"], p.in_dtype, p.layout, None, 256, p.code_dtype, heads=hs)
     rows = {(b, h): list(range(p.N)) for (b, h) in hs}
-    oracle.prefill_rows(*oq, *ok_, *ov, p.code_dtype, p.layout, p.causal, rows, row_chunk=128)
+    oracle.prefill_rows(*oq, *ok_, *ov, p.code_dtype, p.layout, p.causal, rows, row_chunk=row_chunk)
 
 
 def cpu_baseline(p, d, target_s):
@@ -522,9 +627,128 @@ def cpu_baseline(p, d, target_s):
     oracle_sample(p, d, heads)
     dt = time.perf_counter() - t0
     ops = prefill_ops(1, heads, p.N, p.D, p.causal)
+    # one thread: one head as a single job (its rotation and all its rows in
+    # one call each), the same work per head as above
+    t0 = time.perf_counter()
+    oracle_sample(p, d, 1, row_chunk=None)
+    dt1 = time.perf_counter() - t0
+    ops1 = prefill_ops(1, 1, p.N, p.D, p.causal)
     return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
             "sample": "%d of %d heads of %s (all rows: rotate+quantize Q/K/V and quantized attention), %.1f s"
-                      % (heads, p.H, p.name, dt)}
+                      % (heads, p.H, p.name, dt),
+            "value_1thread": round(ops1 / dt1 / 1e12, 6), "cores_1thread": 1,
+            "sample_1thread": "1 head of %s on one thread, %.1f s" % (p.name, dt1)}
+
+
+def _v_absmax(vc, vs, p, b, h):
+    """max |dequantized V| of head (b, h) (the tolerance's scale)."""
+    import synth
+    codes = vc[b, h] if p.layout == synth.BNSD else vc[b, :, h]
+    if p.code_dtype == synth.INT8:
+        vals = np.abs(codes.view(np.int8).astype(np.float64))
+    else:
+        import oracle
+        vals = np.abs(oracle.e4m3_decode(codes).astype(np.float64))
+    blk = np.arange(codes.shape[0]) // p.kv_block
+    return float((vals.max(axis=1) * vs[b, h, blk].astype(np.float64)).max())
+
+
+def _bf16(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _prefill_errors(entry, heads, rows):
+    """Sampled rows of a GPU prefill output against the oracle (same codes,
+    same algorithm) and against float64 attention on the unquantized inputs;
+    errors relative to max |V| of the head (dequantized)."""
+    import oracle
+    import synth
+    p, d, out = entry["problem"], entry["data"], entry["out"]
+    hs = [(0, h) for h in heads]
+    oq = oracle.rotate_block_quant(d["q"], p.in_dtype, p.layout, d["rot"], 128, p.code_dtype, heads=hs)
+    ok_ = oracle.rotate_block_quant(d["k"], p.in_dtype, p.layout, d["rot"], 256, p.code_dtype, heads=hs)
+    ov = oracle.rotate_block_quant(d["v"], p.in_dtype, p.layout, None, 256, p.code_dtype, heads=hs)
+    rbh = {bh: list(rows) for bh in hs}
+    ref = oracle.prefill_rows(*oq, *ok_, *ov, p.code_dtype, p.layout, p.causal, rbh)
+    exact = oracle.exact_rows(d["q"], d["k"], d["v"], p.in_dtype, p.layout, p.causal, rbh)
+    e_or, e_ex = [], []
+    for (b, h) in hs:
+        got = _bf16(out[b, h] if p.layout == synth.BNSD else out[b, :, h])[list(rows)]
+        vmax = _v_absmax(ov[0], ov[1], p, b, h)
+        e_or.append(np.abs(got - _bf16(ref[(b, h)][0])) / vmax)
+        e_ex.append(np.abs(got - exact[(b, h)]) / vmax)
+    e_or, e_ex = np.concatenate(e_or), np.concatenate(e_ex)
+    return {"rows": "%d rows of heads %s" % (len(rows), heads), "max_abs_vs_oracle": float(e_or.max()),
+            "mean_abs_vs_oracle": float(e_or.mean()), "max_abs_vs_fp64": float(e_ex.max()),
+            "mean_abs_vs_fp64": float(e_ex.mean()), "within_tolerance": bool(e_or.max() <= 1e-2 and e_or.mean() <= 1e-3),
+            "scale": "max |dequantized V| of the head"}
+
+
+def _decode_dequant(p, k, scales, b, hk):
+    """float64 K or V rows [L, D] of cache head (b, hk), codes x scales."""
+    import synth
+    if p.kv_dtype == synth.INT8:
+        blk = np.arange(p.L) // p.kv_block
+        return k[b, hk].astype(np.float64) * scales[b, hk, blk].astype(np.float64)[:, None]
+    raw = k[b, hk]
+    lo = ((raw & 0xF).astype(np.int16) ^ 8) - 8
+    hi = ((raw >> 4).astype(np.int16) ^ 8) - 8
+    codes = np.empty((p.L, p.D), np.float64)
+    codes[:, 0::2], codes[:, 1::2] = lo, hi
+    sc = scales[b, hk].view(np.float16).astype(np.float64)            # [L, D / group]
+    return codes * np.repeat(sc, p.group, axis=1)
+
+
+def _decode_errors(entry, pairs):
+    """Sampled (b, h_q) outputs of a GPU decode against the oracle (query
+    quantized to INT8 per head, as the method reads it) and against float64
+    attention with the unquantized bf16 query over the dequantized cache (the
+    cost of that query quantization shows in the second figure)."""
+    import oracle
+    p, dd, out = entry["problem"], entry["data"], entry["out"]
+    ref, _ = oracle.decode(dd["q"], entry["k"], entry["v"], dd["k_scales"], dd["v_scales"], p.kv_dtype, p.Hkv,
+                           heads=pairs, kv_block=p.kv_block, group=p.group)
+    e_or, e_ex = [], []
+    for (b, h) in pairs:
+        hk = h // (p.Hq // p.Hkv)
+        K = _decode_dequant(p, entry["k"], dd["k_scales"], b, hk)
+        V = _decode_dequant(p, entry["v"], dd["v_scales"], b, hk)
+        q = _bf16(dd["q"][b, h, 0])
+        s = K @ q / np.sqrt(p.D)
+        w = np.exp(s - s.max())
+        exact = (w @ V) / w.sum()
+        got = _bf16(out[b, h, 0])
+        vmax = float(np.abs(V).max())
+        e_or.append(np.abs(got - _bf16(ref[b, h, 0])) / vmax)
+        e_ex.append(np.abs(got - exact) / vmax)
+    e_or, e_ex = np.concatenate(e_or), np.concatenate(e_ex)
+    return {"rows": "(b, h_q) pairs %s" % (pairs,), "max_abs_vs_oracle": float(e_or.max()),
+            "mean_abs_vs_oracle": float(e_or.mean()), "max_abs_vs_fp64_unquantized_query": float(e_ex.max()),
+            "mean_abs_vs_fp64_unquantized_query": float(e_ex.mean()),
+            "within_tolerance": bool(e_or.max() <= 1e-2 and e_or.mean() <= 1e-3),
+            "scale": "max |dequantized V| of the head"}
+
+
+def parity_errors(keep):
+    """Error figures of this run's GPU outputs, one entry per stated problem
+    (computed on the host after the timed regions)."""
+    res = {}
+    try:
+        if "tiny_fp8" in keep:
+            res["tiny_fp8"] = _prefill_errors(keep["tiny_fp8"], [0, 1], range(256))
+        if "int8_causal" in keep:
+            res["int8_causal"] = _prefill_errors(keep["int8_causal"], [0, 31],
+                                                 list(range(64)) + list(range(4032, 4096)))
+        if "prefill_fp8_long" in keep:
+            res["fp8_long"] = _prefill_errors(keep["prefill_fp8_long"], [0, 23],
+                                              list(range(64)) + list(range(16320, 16384)))
+        if "decode_int8kv" in keep:
+            res["int8kv_decode"] = _decode_errors(keep["decode_int8kv"], [(0, 0), (17, 5), (33, 31), (63, 12)])
+        if "decode_int4kv" in keep:
+            res["int4kv_decode"] = _decode_errors(keep["decode_int4kv"], [(0, 0), (5, 9), (11, 30), (15, 17)])
+    except Exception as e:      # a report, never a reason to lose the bench line
+        res["error"] = repr(e)
+    return res
 
 
 def reference_arm(args):
@@ -571,7 +795,35 @@ def profile_case(args):
     import synth
     dev = torch.device("cuda", 0)
     c = args.case
-    if c.startswith("decode"):
+    if c.startswith("kv_append"):
+        # the bandwidth-scale append: K of a 4096-token prefill into an empty
+        # cache of the decode problem's shape
+        p = synth.INT8_KV_DECODE if c == "kv_append_int8" else synth.INT4_KV_DECODE
+        kvt = qa.QATTN_INT8 if c == "kv_append_int8" else qa.QATTN_INT4_PACKED
+        g = torch.Generator(device=dev).manual_seed(8)
+        xn = torch.randn((p.B, p.Hkv, 4096, p.D), generator=g, device=dev).to(torch.bfloat16)
+        if kvt == qa.QATTN_INT8:
+            cache = torch.zeros((p.B, p.Hkv, 4096, p.D), dtype=torch.int8, device=dev)
+            scl = torch.zeros((p.B, p.Hkv, 16), dtype=torch.float32, device=dev)
+        else:
+            cache = torch.zeros((p.B, p.Hkv, 4096, p.D // 2), dtype=torch.uint8, device=dev)
+            scl = torch.zeros((p.B, p.Hkv, 4096, p.D // p.group), dtype=torch.float16, device=dev)
+        for _ in range(args.warmup + args.steps):
+            qa.qattn_kv_append(xn, cache, scl, 0, kvt, group=p.group)
+    elif c == "ablation_bf16":
+        # the dequantize-first comparison path on the INT8 causal problem
+        p = synth.INT8_CAUSAL
+        d = synth.make_prefill(p)
+        x = {n: torch.from_numpy(d[n].view(np.int16)).to(dev).view(torch.bfloat16) for n in ("q", "k", "v")}
+        rot = torch.from_numpy(d["rot"]).to(dev)
+        for _ in range(args.warmup + args.steps):
+            deq = []
+            for n in ("q", "k", "v"):
+                cs = qa.qattn_rotate_block_quant(x[n], p.layout, rot if n != "v" else None, 128 if n == "q" else 256,
+                                                 qa.QATTN_INT8)
+                deq.append(qa.qattn_dequant_bf16(*cs, qa.QATTN_INT8, p.layout, 128 if n == "q" else 256))
+            qa.qattn_attention_bf16(*deq, p.layout, p.causal)
+    elif c.startswith("decode"):
         p = synth.INT8_KV_DECODE if c == "decode_int8kv" else synth.INT4_KV_DECODE
         dd = synth.make_decode(p)
         q = torch.from_numpy(dd["q"].view(np.int16)).to(dev).view(torch.bfloat16)
@@ -614,7 +866,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-heads", type=int, default=4, help="heads per reference-arm step")
     ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "prefill_int4v", "prefill_int4", "decode_int8kv",
-                                                           "decode_int4kv"],
+                                                           "decode_int4kv", "kv_append_int8", "kv_append_int4",
+                                                           "ablation_bf16"],
                     help="run one workload only (for profiler captures); prints no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

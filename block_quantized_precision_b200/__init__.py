@@ -6,7 +6,8 @@ memory and streams. There is no fallback: if libqattn.so is missing or a call
 fails, an exception is raised.
 
 Function names follow the C ABI:
-    qattn_rotate_block_quant, qattn_prefill, qattn_prefill_mixed, qattn_decode_workspace_size,
+    qattn_rotate_block_quant, qattn_prefill, qattn_prefill_mixed, qattn_dequant_bf16,
+    qattn_attention_bf16, qattn_decode_workspace_size,
     qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_kv_append, qattn_device_error,
     qattn_selftest_wait_timeout,
     qattn_abi_version, qattn_status_string.
@@ -33,13 +34,13 @@ QATTN_BNSD, QATTN_BSND = 0, 1
 QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 3, 4
 
 EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
-            "qattn_prefill_mixed",
+            "qattn_prefill_mixed", "qattn_dequant_bf16", "qattn_attention_bf16",
             "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc", "qattn_kv_append",
             "qattn_attention_path_host_workspace_size", "qattn_attention_path_host",
             "qattn_device_error", "qattn_selftest_wait_timeout")
 
 # Fixed scratch of qattn_decode_kvq_noalloc (bytes).
-NOALLOC_SCRATCH_BYTES = 4 << 20
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _lib = None
 
@@ -66,6 +67,10 @@ def lib() -> C.CDLL:
         L.qattn_prefill.restype = i
         L.qattn_prefill_mixed.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
         L.qattn_prefill_mixed.restype = i
+        L.qattn_dequant_bf16.argtypes = [P, P, i, i, i, i, i, i, i, P, P]
+        L.qattn_dequant_bf16.restype = i
+        L.qattn_attention_bf16.argtypes = [P, P, P, i, i, i, i, i, i, i, f, P, P, P]
+        L.qattn_attention_bf16.restype = i
         L.qattn_decode_workspace_size.argtypes, L.qattn_decode_workspace_size.restype = [i, i, i, i, i], z
         L.qattn_decode_kvq.argtypes = [P, P, P, P, P, i, i, i, i, i, i, i, i, f, P, P, z, P]
         L.qattn_decode_kvq.restype = i
@@ -176,6 +181,34 @@ def qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales,
     return out
 
 
+def qattn_dequant_bf16(codes, scales, code_dtype: int, layout: int, block_tokens: int, out=None, stream=None):
+    """The dequantize pass of the comparison path: bfloat16 code * block
+    scale, same layout as the codes (INT8 or e4m3)."""
+    import torch
+    B, H, N, D = _dims(codes, layout)
+    if out is None:
+        out = torch.empty(codes.shape, dtype=torch.bfloat16, device=codes.device)
+    st = lib().qattn_dequant_bf16(_ptr(codes), _ptr(scales), code_dtype, layout, B, H, N, D, block_tokens, _ptr(out),
+                                  _stream(stream))
+    _check(st, "qattn_dequant_bf16")
+    return out
+
+
+def qattn_attention_bf16(q, k, v, layout: int, causal: bool, softmax_scale: float = 0.0, out=None, lse=None,
+                         stream=None):
+    """Attention over bfloat16 Q/K/V on the 16-bit tensor-core path (the
+    comparison path's second step); returns the bfloat16 output."""
+    import torch
+    B, H, Nq, D = _dims(q, layout)
+    Nkv = _dims(k, layout)[2]
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    st = lib().qattn_attention_bf16(_ptr(q), _ptr(k), _ptr(v), layout, B, H, Nq, Nkv, D, int(bool(causal)),
+                                    float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "qattn_attention_bf16")
+    return out
+
+
 def qattn_attention_path_host_workspace_size(B: int, H: int, N: int, D: int, layout: int, groups: int = 0) -> int:
     return int(lib().qattn_attention_path_host_workspace_size(B, H, N, D, layout, groups))
 
@@ -233,11 +266,11 @@ def qattn_decode_kvq(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: int, kv_
 
 def qattn_decode_kvq_noalloc(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: int, kv_block: int = 256,
                              group: int = 128, softmax_scale: float = 0.0, out=None, stream=None):
-    """qattn_decode_kvq with the split partials in the library's fixed 4 MiB
+    """qattn_decode_kvq with the split partials in the library's fixed 16 MiB
     device array instead of a caller workspace: for callers that cannot
     allocate device memory on their decode path. Calls must not overlap on
     the GPU (they share the array); make the first call on a device before
-    any stream capture. The output tensor is the caller's: pass `out` to
+    any stream capture, and none after a cudaDeviceReset() on it. The output tensor is the caller's: pass `out` to
     avoid allocating it here."""
     import torch
     B, Hq, _, D = q.shape

@@ -24,9 +24,10 @@
 //               tensor-core instructions:
 //                 scores  S^T[16 tokens x 8 heads] = K Q^T by
 //                         mma.m16n8k32 s8 x s8 -> s32: key rows straight from
-//                         the swizzled tile (INT4 nibbles widened to bytes,
-//                         biased by +8 and corrected with the query code
-//                         sums); the query codes live in 8 registers
+//                         the swizzled tile (INT4 nibbles read as signed
+//                         bytes times 16 by one mask each, the 16 folded
+//                         into the group scales); the query codes live in 8
+//                         registers
 //                 softmax per head over the 16 tokens (shuffles), running
 //                         max / sum in the log2 domain
 //                 P.V     O^T[128 x heads] += V'^T P'^T by mma.m16n8k16
@@ -163,7 +164,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
   float* sRed = reinterpret_cast<float*>(smem);   // after the loop: [warps][G][D]
 
   __shared__ __align__(16) uint32_t sQw[G][kD / 4];    // query codes, 4 per word (natural order)
-  __shared__ int sQsum[G][2];                          // sum of query codes per 64-channel half
   __shared__ float sQf[G];                             // sq * softmax scale * log2(e)
   // P'[head][token] per warp; rows of kPStride floats keep the stores of a
   // warp on distinct banks
@@ -204,23 +204,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       const float sq = __fdiv_rn(m, 127.0f);
       uint32_t w = 0;
-      int csum = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         int c = 0;
         if (sq != 0.0f) c = max(-127, min(127, __float2int_rn(__fdiv_rn(f[e], sq))));
-        csum += c;
         w |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * e);
       }
       sQw[hh][lane] = w;
-      // lanes 0..15 hold channels 0..63, lanes 16..31 channels 64..127
-      const int half_sum0 = __reduce_add_sync(0xffffffffu, lane < 16 ? csum : 0);
-      const int half_sum1 = __reduce_add_sync(0xffffffffu, lane >= 16 ? csum : 0);
-      if (lane == 0) {
-        sQf[hh] = sq * p.scale_log2;
-        sQsum[hh][0] = half_sum0;
-        sQsum[hh][1] = half_sum1;
-      }
+      if (lane == 0) sQf[hh] = sq * p.scale_log2;
     }
   }
   __syncthreads();
@@ -289,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
         const float inv = vrun > 0.0f ? 1.0f / vrun : 0.0f;
 #pragma unroll
         for (int j = 0; j < kScalePerLane; ++j) {
-          sKsf[s][lane + 32 * j] = __half2float(__ushort_as_half(ksv[j]));
+          sKsf[s][lane + 32 * j] = __half2float(__ushort_as_half(ksv[j])) * 0.0625f;   // keys arrive x16
           sVsf[s][lane + 32 * j] = __half2float(__ushort_as_half(vsv[j])) * inv;
         }
         if (lane == 0) sVmax[s] = vrun;
@@ -346,16 +337,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
   const bool h0ok = h0 < G, h1ok = h1 < G;
   const bool own = !kHiLo || cq < 2;        // this lane writes its heads' P' and state
   const float qf0 = h0ok ? sQf[h0] : 0.0f, qf1 = h1ok ? sQf[h1] : 0.0f;
-  int qs0[2] = {0, 0}, qs1[2] = {0, 0};          // INT4: 8 * query code sums per group
-  if constexpr (kInt4) {
-    const int s00 = h0ok ? sQsum[h0][0] : 0, s01 = h0ok ? sQsum[h0][1] : 0;
-    const int s10 = h1ok ? sQsum[h1][0] : 0, s11 = h1ok ? sQsum[h1][1] : 0;
-    if constexpr (kGroups == 2) {
-      qs0[0] = 8 * s00; qs0[1] = 8 * s01; qs1[0] = 8 * s10; qs1[1] = 8 * s11;
-    } else {
-      qs0[0] = 8 * (s00 + s01); qs1[0] = 8 * (s10 + s11);
-    }
-  }
   float (*myP)[8][C::kPStride] = sPw[warp];
   constexpr int kH = C::kHalves;
   // P.V is computed transposed, O^T[channels x heads] += V'^T P'^T, with
@@ -414,11 +395,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
       for (int hf = 0; hf < kH; ++hf) {
         const int ra = r0 + kStep * hf + gq, rb = ra + 8;   // this lane's score rows (tokens)
         const bool va = chunk_t0 + ra < t_end, vb = chunk_t0 + rb < t_end;
-        // one accumulator per 32-channel slice, so that the four MMAs do not
-        // wait on one another; the slices are then added (exact in INT32)
-        int sck[4][4];
+        // INT8: one accumulator per 32-channel slice so that the four MMAs do
+        // not wait on one another; INT4: one per 64-channel half (the two
+        // 16-token halves of a step supply the independent chains); the
+        // accumulators are then added (exact in INT32)
+        constexpr int kAcc = kInt4 ? 2 : 4;
+        int sck[kAcc][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) sck[a][0] = sck[a][1] = sck[a][2] = sck[a][3] = 0;
+        for (int a = 0; a < kAcc; ++a) sck[a][0] = sck[a][1] = sck[a][2] = sck[a][3] = 0;
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           if constexpr (!kInt4) {
@@ -435,20 +419,24 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
             const int off = ((kb ^ ((gq >> 1) & 3)) << 4) + 4 * cq;
             const uint32_t wa = *reinterpret_cast<const uint32_t*>(cK + ra * 64 + off);
             const uint32_t wb = *reinterpret_cast<const uint32_t*>(cK + rb * 64 + off);
-            // nibble c -> byte c + 8 (even channels, odd channels)
-            const uint32_t ea = (wa & 0x0F0F0F0Fu) ^ 0x08080808u, oa = ((wa >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-            const uint32_t eb = (wb & 0x0F0F0F0Fu) ^ 0x08080808u, ob = ((wb >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-            mma_s8(sck[kb], ea, eb, oa, ob, qb0[kb], qb1[kb]);
+            // the nibbles as signed bytes times 16 (exact two's complement):
+            // high nibble w & 0xF0 (odd channels), low nibble (w << 4) & 0xF0
+            // (even channels); the factor 16 is in the group scales
+            const uint32_t ea = (wa << 4) & 0xF0F0F0F0u, oa = wa & 0xF0F0F0F0u;
+            const uint32_t eb = (wb << 4) & 0xF0F0F0F0u, ob = wb & 0xF0F0F0F0u;
+            mma_s8(sck[kb >> 1], ea, eb, oa, ob, qb0[kb], qb1[kb]);
           }
         }
         int sc[kNAcc][4];                                  // per INT4 group (else all 128 channels)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           if constexpr (kNAcc == 2) {
-            sc[0][e] = sck[0][e] + sck[1][e];
-            sc[kNAcc - 1][e] = sck[2][e] + sck[3][e];
+            sc[0][e] = sck[0][e];
+            sc[kNAcc - 1][e] = sck[kAcc - 1][e];
+          } else if constexpr (kInt4) {
+            sc[0][e] = sck[0][e] + sck[kAcc - 1][e];
           } else {
-            sc[0][e] = (sck[0][e] + sck[1][e]) + (sck[2][e] + sck[3][e]);
+            sc[0][e] = (sck[0][e] + sck[1][e]) + (sck[kAcc - 2][e] + sck[kAcc - 1][e]);
           }
         }
         if constexpr (!kInt4) {
@@ -463,10 +451,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<kInt4>::kCtasPerSm)
           for (int gg = 0; gg < kNAcc; ++gg) {
             const float ka = sKsf[s][ra * kGroups + gg];
             const float kb2 = sKsf[s][rb * kGroups + gg];
-            t0 = fmaf(i2f_exact(sc[gg][0] - qs0[gg]), ka, t0);
-            t1 = fmaf(i2f_exact(sc[gg][1] - qs1[gg]), ka, t1);
-            t2 = fmaf(i2f_exact(sc[gg][2] - qs0[gg]), kb2, t2);
-            t3 = fmaf(i2f_exact(sc[gg][3] - qs1[gg]), kb2, t3);
+            t0 = fmaf(i2f_exact(sc[gg][0]), ka, t0);
+            t1 = fmaf(i2f_exact(sc[gg][1]), ka, t1);
+            t2 = fmaf(i2f_exact(sc[gg][2]), kb2, t2);
+            t3 = fmaf(i2f_exact(sc[gg][3]), kb2, t3);
           }
           sv[hf][0] = t0 * qf0; sv[hf][1] = t1 * qf1; sv[hf][2] = t2 * qf0; sv[hf][3] = t3 * qf1;
         }
@@ -784,6 +772,11 @@ int decode_splits(int B, int Hkv, int L, int num_sms) {
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int D, int num_sms) {
   (void)D;
   const int splits = decode_splits(B, Hkv, L, num_sms);
+  return static_cast<size_t>(B) * Hq * splits * kWsStride * sizeof(float);
+}
+
+size_t decode_workspace_bytes_for(int B, int Hq, int Hkv, int L, bool int4, int num_sms) {
+  const int splits = splits_for(B, Hkv, L, num_sms, int4);
   return static_cast<size_t>(B) * Hq * splits * kWsStride * sizeof(float);
 }
 

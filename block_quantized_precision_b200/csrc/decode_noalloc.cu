@@ -14,7 +14,8 @@
 // bytes; every GPU that loads the library keeps it until the process exits.
 // In host code the array's name only stands for it, so its device address is
 // looked up once per device (with that device current) and passed to the
-// kernels as an ordinary pointer.
+// kernels as an ordinary pointer. The address is kept for the life of the
+// process: a cudaDeviceReset() on that device would leave it stale.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,7 +25,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -58,11 +59,9 @@ qattn_status_t qattn_decode_kvq_noalloc(const void* q, const void* k_cache, cons
   void* scratch = nullptr;
   const qattn_status_t s = scratch_address(&scratch);
   if (s != QATTN_OK) return s;
-  if (B > 0 && H_q > 0 && H_kv > 0 && L >= 0 && D > 0 && H_q % H_kv == 0) {
-    const size_t need = qattn_decode_workspace_size(B, H_q, H_kv, L, D);
-    if (need > kNoAllocScratchBytes) return QATTN_ERR_WORKSPACE;  // sizes beyond the fixed scratch
-  }
-  // Same validation and kernels as qattn_decode_kvq; the partials of every
+  // Same validation and kernels as qattn_decode_kvq; a call whose own
+  // partials do not fit the fixed array is refused there with
+  // QATTN_ERR_WORKSPACE before anything is launched. The partials of every
   // split are written before they are read, so nothing needs clearing.
   return qattn_decode_kvq(q, k_cache, v_cache, k_scales, v_scales, kv_dtype, B, H_q, H_kv, L, D, kv_block, group,
                           softmax_scale, out, scratch, kNoAllocScratchBytes, stream);

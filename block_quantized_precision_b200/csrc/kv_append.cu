@@ -15,9 +15,10 @@
 //     each code as the IEEE quotient decides it (code_fast), clamped to
 //     [-127, 127].
 // Packed INT4 cache, one fp16 scale per token per group:
-//   kv_append_int4_kernel: one warp per 4 new tokens of one (b, h_kv); lane l owns channels
-//     4l..4l+3. s16 = fp16(absmax_group / 7), codes RNE(x / s16) clamped to
-//     [-7, 7], packed two per byte.
+//   kv_append_int4_kernel: eight lanes per new token of one (b, h_kv), 16
+//     channels each; s16 = fp16(absmax_group / 7), codes RNE(x / s16)
+//     clamped to [-7, 7] (the product with RN(1/s16) unless it is within
+//     1e-4 of a half-integer), packed two per byte.
 // Both are small, memory-bound kernels (the new rows are read once, the
 // codes written once; a growing INT8 block also rewrites its earlier codes).
 #include <cuda_bf16.h>
@@ -144,53 +145,97 @@ __global__ void __launch_bounds__(kAppendThreads)
   if (threadIdx.x == 0) scales[head * nblk + blk] = s;
 }
 
-// x: bf16 [B, H_kv, n, D], D = 128 (lane l: channels 4l..4l+3); cache bytes
-// [B, H_kv, L_max, D/2]; scales fp16 [B, H_kv, L_max, D/group], group 128 or
-// 64 (all lanes or one half-warp per group).
-constexpr int kInt4RowsPerWarp = 4;
+// x: bf16 [B, H_kv, n, D], D = 128; cache bytes [B, H_kv, L_max, D/2]; scales
+// fp16 [B, H_kv, L_max, D/group], group 128 or 64. Eight lanes per row (lane
+// q of the row's octet owns channels 16q .. 16q + 15: two 16-byte loads, one
+// 8-byte store), so one warp instruction serves four rows and the per-row
+// work (group maximum, scale, reciprocal) is shared by them.
+constexpr int kInt4RowsPerCta = 64;                 // 32 rows per pass of 256 threads, two passes
 
-// Grid (ceil(n / rows per CTA), B * H_kv): blockIdx.y is the (b, h_kv) head.
+// Codes RNE(y / s) clamped to [-7, 7] of 16 values, packed two per byte
+// (element 2i in the low nibble of byte i) into 8 bytes. The product with
+// rcp = RN(1/s) decides unless it lies within 1e-4 of a half-integer, or
+// `wide` says a product may exceed 7.5 in magnitude (an fp16 scale in the
+// subnormal range can round well below absmax / 7); those take the IEEE
+// quotient, clamped.
+__device__ __forceinline__ uint2 int4_codes16(const float (&f)[16], float s, float rcp, bool wide) {
+  const float2 rc = make_float2(rcp, rcp);
+  const float2 mg = make_float2(12582912.0f, 12582912.0f);
+  uint32_t t[16];
+  float dmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 y = make_float2(f[2 * i], f[2 * i + 1]);
+    const float2 m = ffma2(y, rc, mg);                               // RNE(y * rcp) in the low bits
+    const float2 d = ffma2(y, rc, ffma2(m, make_float2(-1.0f, -1.0f), mg));   // y * rcp - that integer
+    dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+    t[2 * i] = __float_as_uint(m.x);
+    t[2 * i + 1] = __float_as_uint(m.y);
+  }
+  if (wide || dmax > 0.4999f) {                                      // rare: decide exactly
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      t[e] = static_cast<uint32_t>(max(-7, min(7, __float2int_rn(__fdiv_rn(f[e], s)))));
+  }
+  uint32_t w[2] = {0, 0};
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e >> 3] |= (t[e] & 0xFu) << (4 * (e & 7));
+  return make_uint2(w[0], w[1]);
+}
+
+// Grid (ceil(n / kInt4RowsPerCta), B * H_kv): blockIdx.y is the (b, h_kv) head.
 __global__ void __launch_bounds__(kAppendThreads)
     kv_append_int4_kernel(const uint16_t* __restrict__ x, int n, int L, int Lmax, int group,
                           uint8_t* __restrict__ cache, uint16_t* __restrict__ scales) {
   constexpr int D = 128;
-  const int lane = threadIdx.x & 31;
+  constexpr int kPasses = kInt4RowsPerCta / (kAppendThreads / 8);
+  const int q = threadIdx.x & 7;                      // lane within the row's octet
   const int64_t head = blockIdx.y;
-  const int r0 = (static_cast<int>(blockIdx.x) * (kAppendThreads / 32) + (threadIdx.x >> 5)) * kInt4RowsPerWarp;
   const uint16_t* xh = x + head * n * D;
-  // the warp's rows are loaded first (in flight together), then coded
-  uint2 raw[kInt4RowsPerWarp];
+  const int ng = D / group;
+  const int width = group / 16;                       // lanes per group: 8 (group 128) or 4 (64)
+  // both passes' rows are loaded first (four 16-byte loads in flight)
+  uint4 raw[kPasses][2];
+  int row[kPasses];
 #pragma unroll
-  for (int i = 0; i < kInt4RowsPerWarp; ++i)
-    raw[i] = r0 + i < n ? *reinterpret_cast<const uint2*>(xh + static_cast<int64_t>(r0 + i) * D + lane * 4)
-                        : make_uint2(0, 0);
+  for (int ps = 0; ps < kPasses; ++ps) {
+    row[ps] = static_cast<int>(blockIdx.x) * kInt4RowsPerCta + ps * (kAppendThreads / 8) + (threadIdx.x >> 3);
+    const bool in = row[ps] < n;
+    const uint4* src = reinterpret_cast<const uint4*>(xh + static_cast<int64_t>(row[ps]) * D + q * 16);
+    raw[ps][0] = in ? __ldcs(src) : make_uint4(0, 0, 0, 0);
+    raw[ps][1] = in ? __ldcs(src + 1) : make_uint4(0, 0, 0, 0);
+  }
 #pragma unroll
-  for (int i = 0; i < kInt4RowsPerWarp; ++i) {
-    if (r0 + i >= n) break;                             // (uniform per warp)
-    const int t = L + r0 + i;
-    const float f[4] = {bf16_bits_to_f32(raw[i].x & 0xFFFFu), bf16_bits_to_f32(raw[i].x >> 16),
-                        bf16_bits_to_f32(raw[i].y & 0xFFFFu), bf16_bits_to_f32(raw[i].y >> 16)};
-    float m = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
-    // reduce over the lanes of this lane's group (16 lanes for group 64)
-    const int width = group / 4;
+  for (int ps = 0; ps < kPasses; ++ps) {
+    const uint32_t w[8] = {raw[ps][0].x, raw[ps][0].y, raw[ps][0].z, raw[ps][0].w,
+                           raw[ps][1].x, raw[ps][1].y, raw[ps][1].z, raw[ps][1].w};
+    float f[16];
+    uint32_t mb = 0;                                  // max |x| on the bf16 bits (sign cleared)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int k = 0; k < 8; ++k) {
+      f[2 * k] = bf16_bits_to_f32(w[k] & 0xFFFFu);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      mb = __vmaxu2(mb, w[k] & 0x7FFF7FFFu);
+    }
+    float m = bf16_bits_to_f32(max(mb & 0xFFFFu, mb >> 16));
+    // maximum over the lanes of this lane's group (within the octet)
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
       const float other = __shfl_xor_sync(0xffffffffu, m, o);
       if (o < width) m = fmaxf(m, other);
     }
     const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
     const float s = __half2float(s16);
-    uint32_t packed = 0;
-    if (s != 0.0f) {
+    uint2 codes = make_uint2(0, 0);
+    if (s != 0.0f) {                                  // (fp16 scales are never subnormal in float32)
       const float rcp = __frcp_rn(s);
-      const bool slow = s < 1.17549435e-38f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) packed |= (static_cast<uint32_t>(code_fast(f[e], s, rcp, slow, 7)) & 0xFu) << (4 * e);
+      codes = int4_codes16(f, s, rcp, m * rcp >= 7.5f);
     }
-    *reinterpret_cast<uint16_t*>(cache + (head * Lmax + t) * (D / 2) + lane * 2) = static_cast<uint16_t>(packed);
-    const int ng = D / group;
-    if ((lane % width) == 0)
-      scales[(head * Lmax + t) * ng + lane / width] = __half_as_ushort(s16);
+    if (row[ps] < n) {
+      const int t = L + row[ps];
+      *reinterpret_cast<uint2*>(cache + (head * Lmax + t) * (D / 2) + q * 8) = codes;
+      if ((q % width) == 0) scales[(head * Lmax + t) * ng + q / width] = __half_as_ushort(s16);
+    }
   }
 }
 
@@ -209,8 +254,8 @@ cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st) {
                                                             a.Lmax, a.kv_block, static_cast<int8_t*>(a.cache),
                                                             static_cast<float*>(a.scales));
   } else {
-    const int per_cta = (kAppendThreads / 32) * kInt4RowsPerWarp;
-    const dim3 grid(static_cast<unsigned>((a.n + per_cta - 1) / per_cta), static_cast<unsigned>(a.B * a.Hkv));
+    const dim3 grid(static_cast<unsigned>((a.n + kInt4RowsPerCta - 1) / kInt4RowsPerCta),
+                    static_cast<unsigned>(a.B * a.Hkv));
     kv_append_int4_kernel<<<grid, kAppendThreads, 0, st>>>(static_cast<const uint16_t*>(a.x), a.n, a.L, a.Lmax,
                                                            a.group, static_cast<uint8_t*>(a.cache),
                                                            static_cast<uint16_t*>(a.scales));

@@ -248,6 +248,57 @@ qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const v
                              stream);
 }
 
+qattn_status_t qattn_dequant_bf16(const void* codes, const float* scales, qattn_dtype_t code_dtype,
+                                  qattn_layout_t layout, int B, int H, int N, int D, int block_tokens, void* out,
+                                  qattn_stream_t stream) {
+  if (B < 0 || H < 0 || N < 0 || D <= 0 || block_tokens <= 0) return QATTN_ERR_INVALID_ARG;
+  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3) return QATTN_ERR_INVALID_ARG;
+  if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
+  if (D % 16) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * N == 0) return QATTN_OK;
+  if (!codes || !scales || !out) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(out)) return QATTN_ERR_ALIGNMENT;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  DequantArgs a;
+  a.codes = codes;
+  a.scales = scales;
+  a.int8 = code_dtype == QATTN_INT8;
+  a.layout = layout;
+  a.B = B; a.H = H; a.N = N; a.D = D; a.block = block_tokens;
+  a.out = out;
+  return from_cuda(launch_dequant_bf16(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms));
+}
+
+qattn_status_t qattn_attention_bf16(const void* q, const void* k, const void* v, qattn_layout_t layout, int B, int H,
+                                    int N_q, int N_kv, int D, int causal, float softmax_scale, void* out, float* lse,
+                                    qattn_stream_t stream) {
+  if (B < 0 || H < 0 || N_q < 0 || N_kv < 0 || D <= 0) return QATTN_ERR_INVALID_ARG;
+  if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return QATTN_ERR_INVALID_ARG;
+  if (causal && N_q != N_kv) return QATTN_ERR_UNSUPPORTED;
+  if (!attn_bf16_supported(D)) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * N_q == 0) return QATTN_OK;
+  if (N_kv == 0) return QATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return QATTN_ERR_ALIGNMENT;
+  if (static_cast<int64_t>(B) * H * ((N_q + 127) / 128) >= (1LL << 31)) return QATTN_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / sqrtf(static_cast<float>(D));
+  AttnBf16Args a;
+  a.q = q; a.k = k; a.v = v;
+  a.layout = layout;
+  a.B = B; a.H = H; a.Nq = N_q; a.Nkv = N_kv; a.D = D;
+  a.causal = causal;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
+  return from_cuda(launch_attn_bf16(a, reinterpret_cast<cudaStream_t>(stream), ds->err));
+}
+
 size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D) {
   if (B <= 0 || H_q <= 0 || H_kv <= 0 || L < 0 || D <= 0 || H_q % H_kv) return 0;
   DeviceState* ds = nullptr;
@@ -280,7 +331,9 @@ qattn_status_t qattn_decode_kvq(const void* q, const void* k_cache, const void* 
   DeviceState* ds = nullptr;
   qattn_status_t s = device_state(&ds);
   if (s != QATTN_OK) return s;
-  if (workspace_bytes < decode_workspace_bytes(B, H_q, H_kv, L, D, ds->num_sms)) return QATTN_ERR_WORKSPACE;
+  // (the call's own split count: qattn_decode_workspace_size() is at least this)
+  if (workspace_bytes < decode_workspace_bytes_for(B, H_q, H_kv, L, kv_dtype == QATTN_INT4_PACKED, ds->num_sms))
+    return QATTN_ERR_WORKSPACE;
   if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / sqrtf(static_cast<float>(D));
   DecodeArgs a;
   a.q = q; a.k = k_cache; a.v = v_cache; a.ks = k_scales; a.vs = v_scales;

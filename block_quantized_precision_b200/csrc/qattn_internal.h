@@ -55,6 +55,32 @@ bool prefill_supported(int D);
 bool prefill_codes_supported(int qk_code, int v_code);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st, int num_sms, int* err);
 
+// The dequantize-first comparison path (prefill_bf16.cu).
+struct DequantArgs {
+  const void* codes;  // INT8 or e4m3, 1 byte per element, layout as the input
+  const float* scales;
+  int int8;           // 1: INT8 codes, 0: e4m3
+  int layout;
+  int B, H, N, D, block;
+  void* out;          // bf16, same layout
+};
+
+struct AttnBf16Args {
+  const void* q;      // bf16
+  const void* k;
+  const void* v;
+  int layout;
+  int B, H, Nq, Nkv, D;
+  int causal;
+  float scale_log2;
+  void* out;          // bf16
+  float* lse;         // nullable
+};
+
+bool attn_bf16_supported(int D);
+cudaError_t launch_attn_bf16(const AttnBf16Args& a, cudaStream_t st, int* err);
+cudaError_t launch_dequant_bf16(const DequantArgs& a, cudaStream_t st, int num_sms);
+
 struct DecodeArgs {
   const void* q;      // bf16 [B, Hq, 1, D]
   const void* k;
@@ -72,6 +98,9 @@ struct DecodeArgs {
 bool decode_supported(int D, int group_size_ratio);
 int decode_splits(int B, int Hkv, int L, int num_sms);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int L, int D, int num_sms);
+// The bytes one call of the given cache type writes (its own split count);
+// at most decode_workspace_bytes().
+size_t decode_workspace_bytes_for(int B, int Hq, int Hkv, int L, bool int4, int num_sms);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st, int num_sms, int* err);
 
 struct KvAppendArgs {

@@ -186,6 +186,40 @@ qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, c
                                    qattn_stream_t stream);
 
 /*
+ * The dequantize-first comparison path: the standard INT8 path that the
+ * pages contrast with quantized attention ("INT8 量化算子", ops-transformer
+ * items 1-2: INT8 is converted back to FP16 and multiplied in FP16, where the
+ * optimised path feeds INT8 to the matrix unit directly). Built to measure
+ * that contrast on B200 beside qattn_prefill; not a step of the method.
+ *
+ * qattn_dequant_bf16: out[...] = bf16(code * scale[b, h, token / block_tokens])
+ * for every element (the float32 product rounded to nearest even).
+ *   codes:  INT8 or e4m3 codes (code_dtype), [B,H,N,D] (BNSD) or [B,N,H,D]
+ *           (BSND), 16-byte aligned; scales float32 [B,H,ceil(N/block_tokens)].
+ *   out:    bfloat16, same layout and shape, 16-byte aligned, caller-owned.
+ *   D must be a multiple of 16.
+ *
+ * qattn_attention_bf16: softmax(Q K^T * softmax_scale) V over bfloat16 Q/K/V
+ * with float32 accumulation on the 16-bit tensor-core path; probabilities
+ * are not quantized (they are rounded to bfloat16 only as the operand of the
+ * P.V product; the row sums use their float32 values). Running softmax over
+ * tiles of 64 keys.
+ *   q/k/v:  bfloat16 [B,H,N,D] or [B,N,H,D], 16-byte aligned; N_q rows of Q,
+ *           N_kv of K and V; D in {64, 128}.
+ *   causal: 0/1 (1 needs N_q == N_kv; key j visible to query i iff j <= i).
+ *   softmax_scale: <= 0 selects 1/sqrt(D).
+ *   out:    bfloat16, layout of Q; lse: nullable float32 [B,H,N_q], natural log.
+ * Errors as qattn_prefill.
+ */
+qattn_status_t qattn_dequant_bf16(const void* codes, const float* scales, qattn_dtype_t code_dtype,
+                                  qattn_layout_t layout, int B, int H, int N, int D, int block_tokens,
+                                  void* out, qattn_stream_t stream);
+
+qattn_status_t qattn_attention_bf16(const void* q, const void* k, const void* v, qattn_layout_t layout,
+                                    int B, int H, int N_q, int N_kv, int D, int causal,
+                                    float softmax_scale, void* out, float* lse, qattn_stream_t stream);
+
+/*
  * Bytes of device workspace qattn_decode_kvq needs for these sizes on the
  * current device (0 when no scratch is needed). The value depends on the
  * device's SM count.
@@ -222,8 +256,9 @@ size_t qattn_decode_workspace_size(int B, int H_q, int H_kv, int L, int D);
  * softmax_scale: <= 0 selects 1/sqrt(D) (float32).
  * out:      bfloat16 [B, H_q, 1, D].
  * workspace / workspace_bytes: device scratch of at least
- *           qattn_decode_workspace_size(B, H_q, H_kv, L, D) bytes, 16-byte
- *           aligned; its contents need no initialisation and are
+ *           qattn_decode_workspace_size(B, H_q, H_kv, L, D) bytes (enough
+ *           for either cache type; a smaller workspace that holds this
+ *           call's own partials is accepted too), 16-byte aligned; its contents need no initialisation and are
  *           overwritten. Calls that share a workspace must not overlap.
  * L == 0 writes zeros to out.
  */
@@ -235,23 +270,27 @@ qattn_status_t qattn_decode_kvq(const void* q, const void* k_cache, const void* 
 
 /*
  * qattn_decode_kvq without a workspace argument: the split partials go to a
- * fixed 4 MiB device array inside the library (4194304 bytes, held on every
+ * fixed 16 MiB device array inside the library (16777216 bytes, held on every
  * GPU that loads the library until the process exits). No counterpart on
  * the pages; it exists for callers that cannot allocate device memory on
  * their decode path -- their memory is reserved up front by an allocator
  * they do not own, or a cudaMalloc/cudaFree there could synchronise the
  * device and stall other streams. The caller still passes inputs and output.
  *
- * Arguments and results are those of qattn_decode_kvq. Sizes whose workspace
- * (qattn_decode_workspace_size) exceeds 4 MiB are rejected with
- * QATTN_ERR_WORKSPACE before anything is launched. The first call on a
+ * Arguments and results are those of qattn_decode_kvq, bit for bit. A call
+ * whose partials (B * H_q * splits * 528 bytes, with the split count of its
+ * own cache type) exceed 16 MiB is rejected with QATTN_ERR_WORKSPACE before
+ * anything is launched; both stated decode problems fit (B=64 H_q=32 L=8192
+ * INT8: 8.25 MiB; B=16 H_q=32 L=32768 INT4: 3.4 MiB). The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current); make that first call before any stream capture.
- * Nothing is allocated or freed, ever. Every call shares the one array and
- * it keeps the last call's contents; nothing in it needs to start at zero
- * (each call writes every partial before reading it). Calls that overlap on
- * the GPU (different streams, or host threads without ordering) race on the
- * array: serialise them.
+ * that device current) and keeps it for the life of the process; make that
+ * first call before any stream capture, and do not call this entry point
+ * again on a device after cudaDeviceReset() (the kept address would be
+ * stale). Nothing is allocated or freed, ever. Every call shares the one
+ * array and it keeps the last call's contents; nothing in it needs to start
+ * at zero (each call writes every partial before reading it). Calls that
+ * overlap on the GPU (different streams, or host threads without ordering)
+ * race on the array: serialise them.
  */
 qattn_status_t qattn_decode_kvq_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                         const void* k_scales, const void* v_scales,

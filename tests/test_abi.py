@@ -137,3 +137,19 @@ def test_kv_append_validation(L):
     assert call(n=0) == qa.QATTN_OK
     assert call(c=None) == qa.QATTN_ERR_INVALID_ARG
     assert call(x=p + 2) == qa.QATTN_ERR_ALIGNMENT
+
+
+def test_dequant_path_validation(L):
+    bad = 0x1000
+    d = L.qattn_dequant_bf16
+    assert d(bad, bad, qa.QATTN_BF16, 0, 1, 1, 128, 128, 128, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert d(bad, bad, qa.QATTN_INT8, 3, 1, 1, 128, 128, 128, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert d(bad, bad, qa.QATTN_INT8, 0, 1, 1, 128, 120, 128, bad, None) == qa.QATTN_ERR_UNSUPPORTED
+    assert d(bad + 8, bad, qa.QATTN_INT8, 0, 1, 1, 128, 128, 128, bad, None) == qa.QATTN_ERR_ALIGNMENT
+    assert d(None, None, qa.QATTN_INT8, 0, 0, 1, 128, 128, 128, None, None) == qa.QATTN_OK
+    a = L.qattn_attention_bf16
+    assert a(bad, bad, bad, 0, 1, 1, 128, 128, 96, 0, 0.0, bad, None, None) == qa.QATTN_ERR_UNSUPPORTED
+    assert a(bad, bad, bad, 0, 1, 1, 128, 200, 128, 1, 0.0, bad, None, None) == qa.QATTN_ERR_UNSUPPORTED
+    assert a(bad, bad, bad, 0, 1, 1, 128, 128, 128, 2, 0.0, bad, None, None) == qa.QATTN_ERR_INVALID_ARG
+    assert a(bad, bad, bad, 0, 1, 1, 128, 0, 128, 0, 0.0, bad, None, None) == qa.QATTN_ERR_UNSUPPORTED
+    assert a(bad, bad + 8, bad, 0, 1, 1, 128, 128, 128, 0, 0.0, bad, None, None) == qa.QATTN_ERR_ALIGNMENT
