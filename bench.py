@@ -463,7 +463,7 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         res[key] = {"workload": "%s shape, K and V of a %d-token prefill into empty caches" % (p.name, n_new),
                     "ms": round(ms, 4), "GB/s": round(gbs, 1), "bytes": by,
                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                                 "frac": round(gbs / hbm_peak, 4)}}
+                                 "frac": round(gbs / hbm_peak, 4), "traffic": load_traffic(key)}}
         del xs, caches, scls
         torch.cuda.empty_cache()
 
@@ -569,9 +569,10 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         "ms_attention_bf16": round(ms_ab, 4), "TFLOPS_attention_bf16": round(ops / (ms_ab * 1e-3) / 1e12, 1),
         "ms_path": round(ms_dq + ms_ab, 4), "ms_int8_prefill": round(ms_i8, 4),
         "int8_speedup_over_path": round((ms_dq + ms_ab) / ms_i8, 3),
-        "roofline": {"bound": "tensor", "peak": pk_bf16, "unit": "TFLOP/s",
+        "roofline": {"kernel": "attn_bf16", "bound": "tensor", "peak": pk_bf16, "unit": "TFLOP/s",
+                     "achieved": round(ops / (ms_ab * 1e-3) / 1e12, 1),
                      "frac": round(ops / (ms_ab * 1e-3) / 1e12 / pk_bf16, 4),
-                     "peak_source": "measured bf16 burst (cuBLAS)"}}
+                     "traffic": load_traffic("attn_bf16"), "peak_source": "measured bf16 burst (cuBLAS)"}}
     del cq, deq
 
     # INT4 Q/K/V on the same problem (Q/K rotated), widened to INT8 on chip
