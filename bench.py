@@ -175,23 +175,29 @@ def gpu_arm(args):
         flush.zero_()
         flush.sum()
     ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
-    names = ["rotq_q", "rotq_k", "quant_v", "prefill"]
+    qkv_out = [(bufs["qc"], bufs["qs"]), (bufs["kc"], bufs["ks"]), (bufs["vc"], bufs["vs"])]
 
     def step(ev=None):
+        # one call quantizes Q, K and V (the Q and K rotations concurrently on
+        # the library's internal streams, joined back into this stream), then
+        # the prefill
         def mark(i):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, p.code_dtype, bufs["qc"], bufs["qs"])
+        qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype, out=qkv_out,
+                                        stream=stream)
         mark(1)
-        qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, p.code_dtype, bufs["kc"], bufs["ks"])
-        mark(2)
-        qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, p.code_dtype, bufs["vc"], bufs["vs"])
-        mark(3)
         qa.qattn_prefill(bufs["qc"], bufs["qs"], bufs["kc"], bufs["ks"], bufs["vc"], bufs["vs"], p.code_dtype,
                          p.layout, p.causal, out=bufs["out"])
-        mark(4)
+        mark(2)
         launches[0] += 4
+
+    def k1_alone(nm):
+        # one of the three quantizations by itself on the whole GPU: the
+        # per-kernel rooflines of the rotation and the V quantization
+        qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
+                                    p.code_dtype, bufs[nm + "c"], bufs[nm + "s"])
 
     def barrier():
         torch.cuda.synchronize()
@@ -203,7 +209,7 @@ def gpu_arm(args):
         l2_flush()
         step()
     assert qa.qattn_device_error() == qa.QATTN_OK
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     props = torch.cuda.get_device_properties(dev)
     uuid = "GPU-" + str(props.uuid) if getattr(props, "uuid", None) else None
     launches[0] = 0
@@ -215,26 +221,51 @@ def gpu_arm(args):
         barrier()
     clocks = clk.summary(pk.get("sm_max_mhz", 1965.0))
     step_launches = launches[0]
-    per = np.array([[evs[i][k].elapsed_time(evs[i][k + 1]) for k in range(4)] for i in range(args.steps)])
+    per = np.array([[evs[i][k].elapsed_time(evs[i][k + 1]) for k in range(2)] for i in range(args.steps)])
     step_ms = per.sum(axis=1)
     ms = max_over_ranks(float(step_ms.mean()), world, dev)
     value = job_rate(ops, world, ms)
     kern_ms = per.mean(axis=0)
+    # the three quantizations one at a time (outside the timed steps, same
+    # flush before each), for their own rooflines and for the gain of
+    # running them in one call
+    alone = {}
+    for nm in ("q", "k", "v"):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            l2_flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            k1_alone(nm)
+            b.record(stream)
+            b.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        alone[nm] = float(np.mean(ts))
+    assert qa.qattn_device_error() == qa.QATTN_OK
     qk_rows = p.B * p.H * p.N
+    elems = qk_rows * p.D
+    k1_bytes, k1_flop = 3 * 3 * elems, 2 * 2 * elems * p.D
+    k1_floor_ms = max(k1_bytes / (hbm_peak * 1e9), k1_flop / (fp32_peak * 1e12)) * 1e3
     kernels = {
-        "rotq_q": {"ms": kern_ms[0], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (kern_ms[0] * 1e-3) / 1e12,
-                   "peak": fp32_peak, "unit": "TFLOP/s"},
-        "rotq_k": {"ms": kern_ms[1], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (kern_ms[1] * 1e-3) / 1e12,
-                   "peak": fp32_peak, "unit": "TFLOP/s"},
-        "quant_v": {"ms": kern_ms[2], "bound": "hbm", "achieved": qk_rows * p.D * 3 / (kern_ms[2] * 1e-3) / 1e9,
-                    "peak": hbm_peak, "unit": "GB/s"},
-        "prefill": {"ms": kern_ms[3], "bound": "tensor", "achieved": ops / (kern_ms[3] * 1e-3) / 1e12,
-                    "peak": int8_peak, "unit": "TOPS"},
+        "rotq_q": {"ms": alone["q"], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (alone["q"] * 1e-3) / 1e12,
+                   "peak": fp32_peak, "unit": "TFLOP/s", "timed": "alone"},
+        "rotq_k": {"ms": alone["k"], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (alone["k"] * 1e-3) / 1e12,
+                   "peak": fp32_peak, "unit": "TFLOP/s", "timed": "alone"},
+        "quant_v": {"ms": alone["v"], "bound": "hbm", "achieved": qk_rows * p.D * 3 / (alone["v"] * 1e-3) / 1e9,
+                    "peak": hbm_peak, "unit": "GB/s", "timed": "alone"},
+        "quant_qkv": {"ms": kern_ms[0], "bound": "alu (FP32 FMA) / hbm, the larger time", "floor_ms": k1_floor_ms,
+                      "frac": k1_floor_ms / kern_ms[0], "timed": "in the step (three launches, one call)",
+                      "ms_three_alone": sum(alone.values())},
+        "prefill": {"ms": kern_ms[1], "bound": "tensor", "achieved": ops / (kern_ms[1] * 1e-3) / 1e12,
+                    "peak": int8_peak, "unit": "TOPS", "timed": "in the step"},
     }
     for k in kernels.values():
-        k["frac"] = k["achieved"] / k["peak"]
+        if "frac" not in k:
+            k["frac"] = k["achieved"] / k["peak"]
         k["ms"] = float(k["ms"])
-    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+        k["frac"] = float(k["frac"])
+    dom = max((n for n in kernels if n != "quant_qkv"), key=lambda n: kernels[n]["ms"])
     traffic = load_traffic(dom)
     roof = {"kernel": dom, "bound": kernels[dom]["bound"], "achieved": round(kernels[dom]["achieved"], 2),
             "peak": kernels[dom]["peak"], "unit": kernels[dom]["unit"], "frac": round(kernels[dom]["frac"], 4),
@@ -484,10 +515,12 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
             x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256, p.code_dtype, codes[nm][0],
             codes[nm][1]), n)
 
+    qkv = lambda: qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype,
+                                                  out=[codes["q"], codes["k"], codes["v"]], stream=stream)
+    ms_qkv = timeit(qkv, n)
+
     def full():
-        for nm in ("q", "k", "v"):
-            qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
-                                        p.code_dtype, codes[nm][0], codes[nm][1])
+        qkv()
         pf()
     ms_full = timeit(full, n)
     ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
@@ -507,12 +540,14 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                                             "peak_source": "measured bf16 burst x 2 (FP8:bf16 nominal ratio)"},
                                "k1": {"ms_rotq_q": round(k1_ms["q"], 4), "ms_rotq_k": round(k1_ms["k"], 4),
                                       "ms_quant_v": round(k1_ms["v"], 4), "ms_total": round(k1_total, 4),
+                                      "ms_one_call": round(ms_qkv, 4),
                                       "bytes": k1_bytes, "fma": k1_fma,
                                       "GB/s": round(k1_bytes / (k1_total * 1e-3) / 1e9, 1),
                                       "TFLOP/s_rotation": round(2 * k1_fma / ((k1_ms["q"] + k1_ms["k"]) * 1e-3) / 1e12, 2),
                                       "roofline": {"bound": "alu (FP32 FMA) / hbm, the larger time",
                                                    "floor_ms": round(k1_floor_ms, 4),
-                                                   "frac": round(k1_floor_ms / k1_total, 4)}}}
+                                                   "frac": round(k1_floor_ms / ms_qkv, 4),
+                                                   "frac_one_at_a_time": round(k1_floor_ms / k1_total, 4)}}}
     keep["prefill_fp8_long"] = {"problem": p, "data": d, "out": out.view(torch.int16).cpu().numpy().view(np.uint16)}
     del x, codes, out
 

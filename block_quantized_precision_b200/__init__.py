@@ -6,7 +6,8 @@ memory and streams. There is no fallback: if libqattn.so is missing or a call
 fails, an exception is raised.
 
 Function names follow the C ABI:
-    qattn_rotate_block_quant, qattn_prefill, qattn_prefill_mixed, qattn_dequant_bf16,
+    qattn_rotate_block_quant, qattn_rotate_block_quant_qkv, qattn_prefill, qattn_prefill_mixed,
+    qattn_dequant_bf16,
     qattn_attention_bf16, qattn_decode_workspace_size,
     qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_kv_append, qattn_device_error,
     qattn_selftest_wait_timeout,
@@ -33,7 +34,8 @@ QATTN_ERR_TIMEOUT = 6
 QATTN_BNSD, QATTN_BSND = 0, 1
 QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 3, 4
 
-EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_prefill",
+EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_rotate_block_quant_qkv",
+            "qattn_prefill",
             "qattn_prefill_mixed", "qattn_dequant_bf16", "qattn_attention_bf16",
             "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc", "qattn_kv_append",
             "qattn_attention_path_host_workspace_size", "qattn_attention_path_host",
@@ -63,6 +65,8 @@ def lib() -> C.CDLL:
         L.qattn_status_string.argtypes, L.qattn_status_string.restype = [i], C.c_char_p
         L.qattn_rotate_block_quant.argtypes = [P, i, i, i, i, i, i, P, i, i, P, P, P]
         L.qattn_rotate_block_quant.restype = i
+        L.qattn_rotate_block_quant_qkv.argtypes = [P, P, P, i, i, i, i, i, i, P, i, P, P, P, P, P, P, P]
+        L.qattn_rotate_block_quant_qkv.restype = i
         L.qattn_prefill.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
         L.qattn_prefill.restype = i
         L.qattn_prefill_mixed.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
@@ -143,6 +147,31 @@ def qattn_rotate_block_quant(x, layout: int, rot, block_tokens: int, code_dtype:
                                         code_dtype, _ptr(codes), _ptr(scales), _stream(stream))
     _check(st, "qattn_rotate_block_quant")
     return codes, scales
+
+
+def qattn_rotate_block_quant_qkv(q, k, v, layout: int, rot, code_dtype: int, out=None, stream=None):
+    """The quantizations of one prefill at once: Q (blocks of 128) and K
+    (256) rotated by rot (or not, rot=None), V (256) not rotated; the two
+    rotations run concurrently. Returns ((q codes, scales), (k ...), (v ...));
+    `out` may pass those six tensors to fill instead."""
+    import torch
+    B, H, N, D = _dims(q, layout)
+    x_dtype = {torch.bfloat16: QATTN_BF16, torch.float16: QATTN_F16}[q.dtype]
+    for t in (k, v):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must have one shape and dtype")
+    if out is None:
+        shape = tuple(q.shape[:-1]) + ((D // 2,) if code_dtype == QATTN_INT4_PACKED else (D,))
+        out = []
+        for blk in (128, 256, 256):
+            out.append((torch.empty(shape, dtype=torch.uint8, device=q.device),
+                        torch.empty((B, H, -(-N // blk)), dtype=torch.float32, device=q.device)))
+    (qc, qs), (kc, ks), (vc, vs) = out
+    st = lib().qattn_rotate_block_quant_qkv(_ptr(q), _ptr(k), _ptr(v), x_dtype, layout, B, H, N, D, _ptr(rot),
+                                            code_dtype, _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(vc), _ptr(vs),
+                                            _stream(stream))
+    _check(st, "qattn_rotate_block_quant_qkv")
+    return out
 
 
 def qattn_prefill(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, code_dtype: int, layout: int,

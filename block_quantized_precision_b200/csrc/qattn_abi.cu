@@ -148,6 +148,76 @@ cudaError_t launch_wait_selftest(int timeout_ms, cudaStream_t st, int* err) {
 
 using namespace qattn;
 
+namespace {
+
+// Argument checks of one rotate/quantize call; QATTN_OK also for an empty
+// problem (nothing to launch: *empty is set).
+qattn_status_t check_rotq(const void* x, qattn_dtype_t x_dtype, qattn_layout_t layout, int B, int H, int N, int D,
+                          const float* rot, int block_tokens, qattn_dtype_t code_dtype, const void* codes,
+                          const float* scales, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0 || D <= 0 || block_tokens <= 0) return QATTN_ERR_INVALID_ARG;
+  if (x_dtype != QATTN_F16 && x_dtype != QATTN_BF16) return QATTN_ERR_INVALID_ARG;
+  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3 && code_dtype != QATTN_INT4_PACKED)
+    return QATTN_ERR_INVALID_ARG;
+  if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
+  if (!rotate_block_quant_supported(D, block_tokens)) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * N == 0) {
+    *empty = true;
+    return QATTN_OK;
+  }
+  if (!x || !codes || !scales) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || (rot && !aligned16(rot))) return QATTN_ERR_ALIGNMENT;
+  return QATTN_OK;
+}
+
+RotQuantArgs rotq_args(const void* x, qattn_dtype_t x_dtype, qattn_layout_t layout, int B, int H, int N, int D,
+                       const float* rot, int block_tokens, qattn_dtype_t code_dtype, void* codes, float* scales) {
+  RotQuantArgs a;
+  a.x = x;
+  a.is_bf16 = x_dtype == QATTN_BF16;
+  a.layout = layout;
+  a.B = B; a.H = H; a.N = N; a.D = D; a.T = block_tokens;
+  a.rot = rot;
+  a.int8 = code_dtype == QATTN_INT8 || code_dtype == QATTN_INT4_PACKED;
+  a.int4 = code_dtype == QATTN_INT4_PACKED;
+  a.codes = codes;
+  a.scales = scales;
+  return a;
+}
+
+// Two internal streams and three events per device for
+// qattn_rotate_block_quant_qkv, created on first use and kept; `enqueue`
+// serialises the calls' enqueueing (they share the streams).
+struct QkvStreams {
+  bool ready = false;
+  cudaStream_t sq = nullptr, sk = nullptr;
+  cudaEvent_t fork = nullptr, done_q = nullptr, done_k = nullptr;
+  std::mutex enqueue;
+};
+QkvStreams g_qkv[kMaxDevices];
+std::mutex g_qkv_mu;
+
+qattn_status_t qkv_streams(QkvStreams** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_qkv_mu);
+  QkvStreams& S = g_qkv[dev];
+  if (!S.ready) {
+    if (cudaStreamCreateWithFlags(&S.sq, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&S.sk, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&S.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&S.done_q, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&S.done_k, cudaEventDisableTiming) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+    S.ready = true;
+  }
+  *out = &S;
+  return QATTN_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int qattn_abi_version(void) { return QATTN_ABI_VERSION; }
@@ -169,29 +239,61 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype, qa
                                         int H, int N, int D, const float* rot, int block_tokens,
                                         qattn_dtype_t code_dtype, void* codes, float* scales,
                                         qattn_stream_t stream) {
-  if (B < 0 || H < 0 || N < 0 || D <= 0 || block_tokens <= 0) return QATTN_ERR_INVALID_ARG;
-  if (x_dtype != QATTN_F16 && x_dtype != QATTN_BF16) return QATTN_ERR_INVALID_ARG;
-  if (code_dtype != QATTN_INT8 && code_dtype != QATTN_FP8_E4M3 && code_dtype != QATTN_INT4_PACKED)
-    return QATTN_ERR_INVALID_ARG;
-  if (layout != QATTN_BNSD && layout != QATTN_BSND) return QATTN_ERR_INVALID_ARG;
-  if (!rotate_block_quant_supported(D, block_tokens)) return QATTN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * H * N == 0) return QATTN_OK;
-  if (!x || !codes || !scales) return QATTN_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(codes) || (rot && !aligned16(rot))) return QATTN_ERR_ALIGNMENT;
+  bool empty = false;
+  const qattn_status_t c = check_rotq(x, x_dtype, layout, B, H, N, D, rot, block_tokens, code_dtype, codes, scales,
+                                      &empty);
+  if (c != QATTN_OK || empty) return c;
   DeviceState* ds = nullptr;
   qattn_status_t s = device_state(&ds);
   if (s != QATTN_OK) return s;
-  RotQuantArgs a;
-  a.x = x;
-  a.is_bf16 = x_dtype == QATTN_BF16;
-  a.layout = layout;
-  a.B = B; a.H = H; a.N = N; a.D = D; a.T = block_tokens;
-  a.rot = rot;
-  a.int8 = code_dtype == QATTN_INT8 || code_dtype == QATTN_INT4_PACKED;
-  a.int4 = code_dtype == QATTN_INT4_PACKED;
-  a.codes = codes;
-  a.scales = scales;
+  const RotQuantArgs a = rotq_args(x, x_dtype, layout, B, H, N, D, rot, block_tokens, code_dtype, codes, scales);
   return from_cuda(launch_rotate_block_quant(a, reinterpret_cast<cudaStream_t>(stream), ds->num_sms, ds->err));
+}
+
+qattn_status_t qattn_rotate_block_quant_qkv(const void* q, const void* k, const void* v, qattn_dtype_t x_dtype,
+                                            qattn_layout_t layout, int B, int H, int N, int D, const float* rot,
+                                            qattn_dtype_t code_dtype, void* q_codes, float* q_scales, void* k_codes,
+                                            float* k_scales, void* v_codes, float* v_scales,
+                                            qattn_stream_t stream) {
+  bool empty = false;
+  qattn_status_t c = check_rotq(q, x_dtype, layout, B, H, N, D, rot, 128, code_dtype, q_codes, q_scales, &empty);
+  if (c == QATTN_OK) c = check_rotq(k, x_dtype, layout, B, H, N, D, rot, 256, code_dtype, k_codes, k_scales, &empty);
+  if (c == QATTN_OK) c = check_rotq(v, x_dtype, layout, B, H, N, D, nullptr, 256, code_dtype, v_codes, v_scales, &empty);
+  if (c != QATTN_OK || empty) return c;
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const RotQuantArgs aq = rotq_args(q, x_dtype, layout, B, H, N, D, rot, 128, code_dtype, q_codes, q_scales);
+  const RotQuantArgs ak = rotq_args(k, x_dtype, layout, B, H, N, D, rot, 256, code_dtype, k_codes, k_scales);
+  const RotQuantArgs av = rotq_args(v, x_dtype, layout, B, H, N, D, nullptr, 256, code_dtype, v_codes, v_scales);
+  if (rot == nullptr) {
+    // three memory-bound passes: one after the other on the whole GPU
+    cudaError_t e = launch_rotate_block_quant(aq, st, ds->num_sms, ds->err);
+    if (e == cudaSuccess) e = launch_rotate_block_quant(ak, st, ds->num_sms, ds->err);
+    if (e == cudaSuccess) e = launch_rotate_block_quant(av, st, ds->num_sms, ds->err);
+    return from_cuda(e);
+  }
+  QkvStreams* S = nullptr;
+  s = qkv_streams(&S);
+  if (s != QATTN_OK) return s;
+  // The rotations of Q and K (FMA-bound, one persistent CTA per SM) run at
+  // the same time on two internal streams, each on half of the SMs; V's
+  // memory-bound quantization is enqueued on the caller's stream and takes
+  // SMs as they free up. The caller's stream waits for both rotations.
+  const int half = ds->num_sms / 2 > 0 ? ds->num_sms / 2 : 1;
+  std::lock_guard<std::mutex> lock(S->enqueue);
+  cudaError_t e = cudaEventRecord(S->fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(S->sq, S->fork, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(S->sk, S->fork, 0);
+  if (e == cudaSuccess) e = launch_rotate_block_quant(aq, S->sq, half, ds->err);
+  if (e == cudaSuccess) e = launch_rotate_block_quant(ak, S->sk, ds->num_sms - half, ds->err);
+  if (e == cudaSuccess) e = launch_rotate_block_quant(av, st, ds->num_sms, ds->err);
+  if (e == cudaSuccess) e = cudaEventRecord(S->done_q, S->sq);
+  if (e == cudaSuccess) e = cudaEventRecord(S->done_k, S->sk);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, S->done_q, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, S->done_k, 0);
+  return from_cuda(e);
 }
 
 qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, const void* k_codes,

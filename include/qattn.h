@@ -122,6 +122,37 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype,
                                         qattn_stream_t stream);
 
 /*
+ * The three quantizations of one prefill at once: Q (blocks of 128 tokens)
+ * and K (blocks of 256) rotated by the same R, V (blocks of 256) not rotated,
+ * all to code_dtype -- the same codes and scales, bit for bit, as three
+ * qattn_rotate_block_quant calls ("MindIE-SD quantization", FA量化 / 技术特点:
+ * rotation of Q and K, then block quantization of Q/K/V).
+ *
+ * With rot != NULL the two rotations (bound by float32 FMA throughput, one
+ * persistent CTA per SM) run concurrently, each on half of the SMs, on two
+ * streams internal to the library (created on first use per device and
+ * kept); the quantization of V is enqueued on `stream` and takes SMs as they
+ * free up; `stream` then waits for both rotations, so the call behaves as an
+ * ordinary stream-ordered operation. Concurrent calls on one device
+ * serialise their enqueueing. With rot == NULL the three passes run one after
+ * the other on `stream`.
+ *
+ * Arguments as qattn_rotate_block_quant, for three tensors of one shape:
+ *   q, k, v:            F16/BF16 [B,H,N,D] (BNSD) or [B,N,H,D] (BSND).
+ *   q_codes, q_scales:  codes like q (D/2 bytes per row for INT4), float32
+ *                       [B,H,ceil(N/128)].
+ *   k_codes/v_codes, k_scales/v_scales: likewise with [B,H,ceil(N/256)].
+ * Errors: those of qattn_rotate_block_quant for any of the three; nothing is
+ * launched on an argument error.
+ */
+qattn_status_t qattn_rotate_block_quant_qkv(const void* q, const void* k, const void* v,
+                                            qattn_dtype_t x_dtype, qattn_layout_t layout, int B,
+                                            int H, int N, int D, const float* rot,
+                                            qattn_dtype_t code_dtype, void* q_codes,
+                                            float* q_scales, void* k_codes, float* k_scales,
+                                            void* v_codes, float* v_scales, qattn_stream_t stream);
+
+/*
  * Quantized attention over block-quantized codes (prefill).
  *
  * Defined by: "MindIE-SD quantization", FA量化 / FP8 Attention (attention in

@@ -153,3 +153,17 @@ def test_dequant_path_validation(L):
     assert a(bad, bad, bad, 0, 1, 1, 128, 128, 128, 2, 0.0, bad, None, None) == qa.QATTN_ERR_INVALID_ARG
     assert a(bad, bad, bad, 0, 1, 1, 128, 0, 128, 0, 0.0, bad, None, None) == qa.QATTN_ERR_UNSUPPORTED
     assert a(bad, bad + 8, bad, 0, 1, 1, 128, 128, 128, 0, 0.0, bad, None, None) == qa.QATTN_ERR_ALIGNMENT
+
+
+def test_rotate_block_quant_qkv_validation(L):
+    bad = 0x1000
+    f = L.qattn_rotate_block_quant_qkv
+    args = lambda **kw: [kw.get("q", bad), bad, bad, kw.get("x", qa.QATTN_BF16), 0, kw.get("B", 1), 1, 128, kw.get("D", 128),
+                         None, kw.get("code", qa.QATTN_INT8), bad, bad, bad, bad, kw.get("vc", bad), bad, None]
+    assert f(*args(B=-1)) == qa.QATTN_ERR_INVALID_ARG
+    assert f(*args(x=qa.QATTN_INT8)) == qa.QATTN_ERR_INVALID_ARG
+    assert f(*args(code=qa.QATTN_BF16)) == qa.QATTN_ERR_INVALID_ARG
+    assert f(*args(D=96)) == qa.QATTN_ERR_UNSUPPORTED
+    assert f(*args(q=bad + 8)) == qa.QATTN_ERR_ALIGNMENT
+    assert f(*args(vc=None)) == qa.QATTN_ERR_INVALID_ARG          # V codes missing
+    assert f(*args(B=0)) == qa.QATTN_OK                            # empty problem

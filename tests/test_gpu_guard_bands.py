@@ -189,3 +189,21 @@ def test_dequant_path(N, D, layout):
     assert qa.qattn_device_error() == qa.QATTN_OK
     out.check("output")
     lse.check("lse")
+
+
+@pytest.mark.parametrize("N", [1, 300])
+@pytest.mark.parametrize("code", [synth.INT8, synth.INT4_PACKED])
+def test_rotate_block_quant_qkv(N, code):
+    """The three quantizations in one call, two of them on internal streams:
+    six outputs, each inside its own guard bands."""
+    p = _problem(N, 128, synth.BSND, synth.INT8, False, 7500 + N + code)
+    d = synth.make_prefill(p)
+    x = [dev_bits(d[n], p.in_dtype) for n in ("q", "k", "v")]
+    shape = tuple(x[0].shape[:-1]) + ((64,) if code == synth.INT4_PACKED else (128,))
+    outs = [(Guarded(shape, torch.uint8), Guarded((p.B, p.H, -(-N // blk)), torch.float32)) for blk in (128, 256, 256)]
+    qa.qattn_rotate_block_quant_qkv(*x, p.layout, dev(d["rot"]), code, out=[(c.t, s.t) for c, s in outs])
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    for name, (c, s) in zip("qkv", outs):
+        c.check("%s codes" % name)
+        s.check("%s scales" % name)
