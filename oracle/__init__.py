@@ -126,8 +126,7 @@ def int4_unpack(b: int):
 # ---------------------------------------------------------------------------
 
 def rotate_row(x: np.ndarray, rot) -> np.ndarray:
-    """float32 y = x R for one row: the exact products summed in float64,
-    rounded once to float32."""
+    """float32 y = x R for one row (sequential float32 FMA chain)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     R = None if rot is None else np.ascontiguousarray(rot, dtype=np.float32)
     y = np.empty_like(x)

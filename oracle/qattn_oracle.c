@@ -34,15 +34,11 @@
  *    per block of tokens like the INT8/e4m3 ones (absmax / 7, codes in
  *    [-7, 7], packed as above).
  *
- * Precision: the rotation is the matrix product X R as the page states it,
- * each entry summed in float64 from the exact products (an input has at
- * most 11 significant bits and R 24, so every product is exact in float64)
- * and rounded once to float32, the type of the rotated values; the steps
- * after it that decide an integer code (block absmax, scale, code rounding,
- * the probabilities that are rounded to 8-bit codes) are carried out in IEEE
- * float32, one rounding per operation, in the order written here; everything
- * else (dot products of codes, the softmax sums, the output accumulation) is
- * exact or float64.
+ * Precision: every step whose result decides an integer code (rotation,
+ * block absmax, scale, code rounding, the probabilities that are rounded to
+ * 8-bit codes) is carried out in IEEE float32, one rounding per operation, in
+ * the order written here; everything else (dot products of codes, the
+ * softmax sums, the output accumulation) is exact or float64.
  *
  * Built with: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC.
  */
@@ -193,23 +189,23 @@ static float in_to_f32(const uint16_t* x, int dtype, int64_t i) {
 /* ------------------------------------------------------------------------ */
 
 /*
- * Rotation of one row: y[j] = sum_k x[k] R[k][j] (R row-major D x D). Each
- * product is exact in float64; they are added in float64 in ascending k
- * starting from +0, and the sum is rounded once to float32. R == NULL: y = x.
+ * Rotation of one row: y[j] = sum_k x[k] R[k][j] (R row-major D x D), as a
+ * chain of float32 fused multiply-adds in ascending k starting from +0, one
+ * rounding per step. R == NULL: y = x.
  */
 void orc_rotate_row(const float* x, const float* R, int D, float* y) {
   for (int j = 0; j < D; ++j) {
     if (!R) { y[j] = x[j]; continue; }
-    double acc = 0.0;
-    for (int k = 0; k < D; ++k) acc += (double)x[k] * (double)R[(int64_t)k * D + j];
-    y[j] = (float)acc;
+    float acc = 0.0f;
+    for (int k = 0; k < D; ++k) acc = fmaf(x[k], R[(int64_t)k * D + j], acc);
+    y[j] = acc;
   }
 }
 
 /*
  * One block of one (b, h): rows n in [blk*T, min(N, (blk+1)*T)).
- *   y = x R           (y[j] = sum_k x[k] R[k][j]: exact products summed in
- *                      float64, rounded once to float32; R == NULL: y = x)
+ *   y = x R           (y[j] = sum_k x[k] R[k][j], float32 fused multiply-adds
+ *                      in ascending k starting from +0; R == NULL: y = x)
  *   amax = max |y|    over the block's valid rows and all D columns
  *   s = amax / qmax   (one float32 division; qmax 127 for INT8, 448 for e4m3)
  *   code = RNE(y / s) (float32 division, then round half to even; INT8

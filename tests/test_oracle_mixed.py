@@ -64,7 +64,7 @@ def test_int4_codes_match_torch_division(orc, layout, block):
 
 
 def test_int4_rotation_by_permutation_is_exact(orc):
-    """A permutation matrix rotates exactly (every sum adds zeros and one
+    """A permutation matrix rotates exactly (every FMA chain adds zeros and one
     product by 1), so the codes are the unrotated codes with permuted columns."""
     rng = np.random.default_rng(3)
     x = _bf16(rng, (1, 2, 256, 64))
