@@ -176,28 +176,25 @@ def gpu_arm(args):
         flush.sum()
     ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
     qkv_out = [(bufs["qc"], bufs["qs"]), (bufs["kc"], bufs["ks"]), (bufs["vc"], bufs["vs"])]
+    # The step runs as one CUDA graph (captured once): the launches of a step
+    # reach the GPU back to back, with no host time between them. An event
+    # node between the quantization and the prefill times both in every step.
+    ev_mid = torch.cuda.Event(enable_timing=True, external=True)
 
-    def step(ev=None):
+    def step_body(st):
         # one call quantizes Q, K and V (the Q and K rotations concurrently on
         # the library's internal streams, joined back into this stream), then
         # the prefill
-        def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
-        mark(0)
-        qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype, out=qkv_out,
-                                        stream=stream)
-        mark(1)
+        qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype, out=qkv_out, stream=st)
+        ev_mid.record(st)
         qa.qattn_prefill(bufs["qc"], bufs["qs"], bufs["kc"], bufs["ks"], bufs["vc"], bufs["vs"], p.code_dtype,
-                         p.layout, p.causal, out=bufs["out"])
-        mark(2)
-        launches[0] += 4
+                         p.layout, p.causal, out=bufs["out"], stream=st)
 
-    def k1_alone(nm):
+    def k1_alone(nm, st):
         # one of the three quantizations by itself on the whole GPU: the
         # per-kernel rooflines of the rotation and the V quantization
         qa.qattn_rotate_block_quant(x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256,
-                                    p.code_dtype, bufs[nm + "c"], bufs[nm + "s"])
+                                    p.code_dtype, bufs[nm + "c"], bufs[nm + "s"], stream=st)
 
     def barrier():
         torch.cuda.synchronize()
@@ -205,43 +202,38 @@ def gpu_arm(args):
             dist.barrier()
         torch.cuda.synchronize()
 
+    g_step = capture_graph(step_body, args.warmup)
+    g_alone = {nm: capture_graph(lambda st, nm=nm: k1_alone(nm, st), 2) for nm in ("q", "k", "v")}
     for _ in range(args.warmup):
         l2_flush()
-        step()
+        g_step.replay()
+    torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
     uuid = "GPU-" + str(props.uuid) if getattr(props, "uuid", None) else None
-    launches[0] = 0
+    per = []
     with ClockSampler(uuid) as clk:
         barrier()
         for i in range(args.steps):
             l2_flush()
-            step(evs[i])
+            e0.record(stream)
+            g_step.replay()
+            e1.record(stream)
+            e1.synchronize()
+            per.append((e0.elapsed_time(ev_mid), ev_mid.elapsed_time(e1)))
         barrier()
     clocks = clk.summary(pk.get("sm_max_mhz", 1965.0))
-    step_launches = launches[0]
-    per = np.array([[evs[i][k].elapsed_time(evs[i][k + 1]) for k in range(2)] for i in range(args.steps)])
+    step_launches = 4 * args.steps                  # 3 quantization kernels + the prefill per step
+    per = np.array(per)
     step_ms = per.sum(axis=1)
     ms = max_over_ranks(float(step_ms.mean()), world, dev)
     value = job_rate(ops, world, ms)
     kern_ms = per.mean(axis=0)
-    # the three quantizations one at a time (outside the timed steps, same
-    # flush before each), for their own rooflines and for the gain of
+    # the three quantizations one at a time (graphs of one call each, the
+    # same flush before each), for their own rooflines and for the gain of
     # running them in one call
-    alone = {}
-    for nm in ("q", "k", "v"):
-        ts = []
-        for i in range(args.warmup + args.steps):
-            l2_flush()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            k1_alone(nm)
-            b.record(stream)
-            b.synchronize()
-            if i >= args.warmup:
-                ts.append(a.elapsed_time(b))
-        alone[nm] = float(np.mean(ts))
+    alone = {nm: time_graph(g_alone[nm], args.steps, args.warmup, stream, l2_flush) for nm in ("q", "k", "v")}
     assert qa.qattn_device_error() == qa.QATTN_OK
     qk_rows = p.B * p.H * p.N
     elems = qk_rows * p.D
@@ -249,16 +241,16 @@ def gpu_arm(args):
     k1_floor_ms = max(k1_bytes / (hbm_peak * 1e9), k1_flop / (fp32_peak * 1e12)) * 1e3
     kernels = {
         "rotq_q": {"ms": alone["q"], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (alone["q"] * 1e-3) / 1e12,
-                   "peak": fp32_peak, "unit": "TFLOP/s", "timed": "alone"},
+                   "peak": fp32_peak, "unit": "TFLOP/s", "timed": "alone (graph of one call)"},
         "rotq_k": {"ms": alone["k"], "bound": "alu", "achieved": qk_rows * p.D * p.D * 2 / (alone["k"] * 1e-3) / 1e12,
-                   "peak": fp32_peak, "unit": "TFLOP/s", "timed": "alone"},
+                   "peak": fp32_peak, "unit": "TFLOP/s", "timed": "alone (graph of one call)"},
         "quant_v": {"ms": alone["v"], "bound": "hbm", "achieved": qk_rows * p.D * 3 / (alone["v"] * 1e-3) / 1e9,
-                    "peak": hbm_peak, "unit": "GB/s", "timed": "alone"},
+                    "peak": hbm_peak, "unit": "GB/s", "timed": "alone (graph of one call)"},
         "quant_qkv": {"ms": kern_ms[0], "bound": "alu (FP32 FMA) / hbm, the larger time", "floor_ms": k1_floor_ms,
-                      "frac": k1_floor_ms / kern_ms[0], "timed": "in the step (three launches, one call)",
+                      "frac": k1_floor_ms / kern_ms[0], "timed": "in the step graph (three launches, one call)",
                       "ms_three_alone": sum(alone.values())},
         "prefill": {"ms": kern_ms[1], "bound": "tensor", "achieved": ops / (kern_ms[1] * 1e-3) / 1e12,
-                    "peak": int8_peak, "unit": "TOPS", "timed": "in the step"},
+                    "peak": int8_peak, "unit": "TOPS", "timed": "in the step graph"},
     }
     for k in kernels.values():
         if "frac" not in k:
@@ -509,20 +501,29 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
     pf = lambda: qa.qattn_prefill(codes["q"][0], codes["q"][1], codes["k"][0], codes["k"][1], codes["v"][0],
                                   codes["v"][1], p.code_dtype, p.layout, p.causal, out=out)
     ms_pf = timeit(pf, n)
+    # the quantizations and the path as CUDA graphs (no host time between launches)
     k1_ms = {}
     for nm in ("q", "k", "v"):
-        k1_ms[nm] = timeit(lambda nm=nm: qa.qattn_rotate_block_quant(
+        g = capture_graph(lambda st, nm=nm: qa.qattn_rotate_block_quant(
             x[nm], p.layout, rot if nm != "v" else None, 128 if nm == "q" else 256, p.code_dtype, codes[nm][0],
-            codes[nm][1]), n)
+            codes[nm][1], stream=st), 2)
+        k1_ms[nm] = time_graph(g, n, 3, stream)
+        del g
 
-    qkv = lambda: qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype,
-                                                  out=[codes["q"], codes["k"], codes["v"]], stream=stream)
-    ms_qkv = timeit(qkv, n)
+    def qkv(st):
+        qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype,
+                                        out=[codes["q"], codes["k"], codes["v"]], stream=st)
+    g = capture_graph(qkv, 2)
+    ms_qkv = time_graph(g, n, 3, stream)
+    del g
 
-    def full():
-        qkv()
-        pf()
-    ms_full = timeit(full, n)
+    def full(st):
+        qkv(st)
+        qa.qattn_prefill(codes["q"][0], codes["q"][1], codes["k"][0], codes["k"][1], codes["v"][0], codes["v"][1],
+                         p.code_dtype, p.layout, p.causal, out=out, stream=st)
+    g = capture_graph(full, 2)
+    ms_full = time_graph(g, n, 3, stream)
+    del g
     ops = prefill_ops(p.B, p.H, p.N, p.D, p.causal)
     tf = ops / (ms_pf * 1e-3) / 1e12
     # K1 (rotate + quantize Q and K, quantize V): 3 bytes per element of each
@@ -821,6 +822,42 @@ def reference_arm(args):
             "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
+
+
+def capture_graph(fn, warm):
+    """A CUDA graph of the launches fn(stream) makes, captured after `warm`
+    eager runs on a side stream (capture wants warmed-up callers)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(max(1, warm)):
+            fn(side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, reps, warm, stream, flush=None):
+    """Mean device time (ms) of graph replays, each after flush(): CUDA events
+    on the replaying stream around each replay."""
+    import torch
+    ts = []
+    for i in range(warm + reps):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        b.synchronize()
+        if i >= warm:
+            ts.append(a.elapsed_time(b))
+    return float(np.mean(ts))
 
 def profile_case(args):
     """Runs one workload (warmup + steps launches, no timing, no JSON): the

@@ -49,21 +49,22 @@ def test_dequant_pass_bit_exact(orc, code_dtype, layout):
         assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), want)
 
 
-def _oracle_bf16_inputs(orc, p, d, heads):
-    """The oracle's codes and scales of Q, K, V dequantized and rounded to
-    bfloat16 (bit patterns, the layout of the problem)."""
-    oq = orc.rotate_block_quant(d["q"], p.in_dtype, p.layout, d["rot"], 128, p.code_dtype, heads=heads)
-    ok_ = orc.rotate_block_quant(d["k"], p.in_dtype, p.layout, d["rot"], 256, p.code_dtype, heads=heads)
-    ov = orc.rotate_block_quant(d["v"], p.in_dtype, p.layout, None, 256, p.code_dtype, heads=heads)
-    return (_dequant_ref(oq[0], oq[1], p.code_dtype, p.layout, 128, orc),
-            _dequant_ref(ok_[0], ok_[1], p.code_dtype, p.layout, 256, orc),
-            _dequant_ref(ov[0], ov[1], p.code_dtype, p.layout, 256, orc))
+def _oracle_codes(orc, p, d, heads):
+    return (orc.rotate_block_quant(d["q"], p.in_dtype, p.layout, d["rot"], 128, p.code_dtype, heads=heads),
+            orc.rotate_block_quant(d["k"], p.in_dtype, p.layout, d["rot"], 256, p.code_dtype, heads=heads),
+            orc.rotate_block_quant(d["v"], p.in_dtype, p.layout, None, 256, p.code_dtype, heads=heads))
 
 
-def _gpu_path(p, d):
-    (qc, qs), (kc, ks), (vc, vs) = gpu_quant_all(d)
-    deq = [qa.qattn_dequant_bf16(c, s, p.code_dtype, p.layout, blk)
-           for (c, s), blk in (((qc, qs), 128), ((kc, ks), 256), ((vc, vs), 256))]
+def _bf16_inputs(orc, p, codes):
+    """Codes and scales of Q, K, V dequantized and rounded to bfloat16 (bit
+    patterns, the layout of the problem)."""
+    return tuple(_dequant_ref(c, s, p.code_dtype, p.layout, blk, orc) for (c, s), blk in zip(codes, (128, 256, 256)))
+
+
+def _gpu_path(p, codes):
+    """The GPU's dequantize pass and bfloat16 attention on the given codes."""
+    deq = [qa.qattn_dequant_bf16(torch.from_numpy(c).cuda(), torch.from_numpy(s).cuda(), p.code_dtype, p.layout, blk)
+           for (c, s), blk in zip(codes, (128, 256, 256))]
     lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device="cuda")
     out = qa.qattn_attention_bf16(*deq, p.layout, p.causal, lse=lse)
     torch.cuda.synchronize()
@@ -72,16 +73,18 @@ def _gpu_path(p, d):
 
 
 def _run(orc, p, d, rows=None):
-    """The GPU path against float64 attention on the bfloat16 inputs it
-    receives (the oracle's codes x scales rounded to bfloat16): what the
+    """The GPU's dequantize pass and bfloat16 attention, fed the oracle's
+    codes, against float64 attention on the bfloat16 inputs they make (the
+    oracle's codes x scales rounded to bfloat16): what the
     dequantize-first path computes, exactly up to its float32 accumulation
     and the bfloat16 rounding of P as an MMA operand. (The bfloat16 rounding
     of the dequantized inputs itself moves large scores -- the outlier
     channels -- by O(1), so the quantized-attention oracle is not the
     reference here.)"""
-    out_bits, lse_np = _gpu_path(p, d)
     heads = [(b, h) for b in range(p.B) for h in range(p.H)] if rows is None else list(rows)
-    qb_bits, kb_bits, vb_bits = _oracle_bf16_inputs(orc, p, d, heads)
+    codes = _oracle_codes(orc, p, d, heads)
+    out_bits, lse_np = _gpu_path(p, codes)
+    qb_bits, kb_bits, vb_bits = _bf16_inputs(orc, p, codes)
     rbh = {bh: list(range(p.N)) for bh in heads} if rows is None else rows
     ref = orc.exact_rows(qb_bits, kb_bits, vb_bits, synth.BF16, p.layout, p.causal, rbh)
     qb, kb, vb = bf16_to_f64(qb_bits), bf16_to_f64(kb_bits), bf16_to_f64(vb_bits)

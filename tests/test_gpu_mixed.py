@@ -122,8 +122,8 @@ def test_mixed_int4_full_size(orc):
 @pytest.mark.parametrize("layout", [synth.BNSD, synth.BSND])
 @pytest.mark.parametrize("D,block", [(64, 128), (128, 128), (128, 256)])
 def test_int4_rotated_block_quant_bit_exact(orc, layout, D, block):
-    """Rotation + INT4 codes (the float32 FMA chain of the rotation decides
-    the codes as for INT8)."""
+    """Rotation + INT4 codes (the rotated values decide the codes as for
+    INT8)."""
     N = 300
     rng = np.random.default_rng(D + block + 11 * layout)
     shape = (1, 3, N, D) if layout == synth.BNSD else (1, N, 3, D)

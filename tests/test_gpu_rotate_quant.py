@@ -1,5 +1,5 @@
-"""GPU parity of the fused rotation + block quantization kernel: codes and
-scales must equal the oracle's bit for bit."""
+"""GPU parity of the rotation + block quantization kernels: codes and scales
+must equal the oracle's bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -36,7 +36,7 @@ def _check_all(orc, x_bits, in_dtype, layout, rot, block, code_dtype, blocks=Non
 
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("layout", [synth.BNSD, synth.BSND])
-@pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3])
+@pytest.mark.parametrize("code_dtype", [synth.INT8, synth.FP8_E4M3, synth.INT4_PACKED])
 @pytest.mark.parametrize("rotate", [False, True])
 @pytest.mark.parametrize("block", [128, 256])
 def test_small_shapes_bit_exact(orc, D, layout, code_dtype, rotate, block):
@@ -110,3 +110,32 @@ def test_full_size_sampled_blocks(orc, prob):
             blocks = [(0, int(h), int(k)) for h, k in zip(rng.integers(0, p.H, 6), rng.integers(0, nblk, 6))]
             blocks += [(0, p.H - 1, nblk - 1), (0, 0, 0)]
         _check_all(orc, d[name], p.in_dtype, p.layout, rot, blk, p.code_dtype, blocks=blocks)
+
+
+def test_signed_permutation_rotation_all_shapes(orc):
+    """A signed permutation moves every value exactly: at both block sizes,
+    both D and every code type."""
+    rng = np.random.default_rng(21)
+    for D in (64, 128):
+        x = synth.f32_to_bf16_bits(rng.standard_normal((1, 2, 300, D)) * 4)
+        P = np.zeros((D, D), dtype=np.float32)
+        P[np.arange(D), rng.permutation(D)] = rng.choice([-1.0, 1.0], D)
+        for T in (128, 256):
+            for code in (synth.INT8, synth.FP8_E4M3, synth.INT4_PACKED):
+                _check_all(orc, x, synth.BF16, synth.BNSD, P, T, code)
+
+
+@pytest.mark.parametrize("in_dtype", [synth.BF16, synth.F16])
+def test_wide_range_inputs_and_matrix(orc, in_dtype):
+    """Inputs spanning many binades (f16 ones with subnormals) and a
+    non-orthogonal R whose entries span many binades too, some far below the
+    largest: the FMA chain of the rotation is reproduced bit for bit."""
+    rng = np.random.default_rng(23 + in_dtype)
+    D = 128
+    mag = np.exp2(rng.integers(-16, 6, (1, 2, 300, D)))
+    vals = rng.standard_normal((1, 2, 300, D)) * mag
+    x = synth.f32_to_bf16_bits(vals) if in_dtype == synth.BF16 else synth.f64_to_f16_bits(vals)
+    R = (rng.standard_normal((D, D)) * np.exp2(rng.integers(-30, 3, (D, D)))).astype(np.float32)
+    for code in (synth.INT8, synth.FP8_E4M3, synth.INT4_PACKED):
+        for T in (128, 256):
+            _check_all(orc, x, in_dtype, synth.BNSD, R, T, code)
