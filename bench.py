@@ -883,6 +883,25 @@ def profile_case(args):
             scl = torch.zeros((p.B, p.Hkv, 4096, p.D // p.group), dtype=torch.float16, device=dev)
         for _ in range(args.warmup + args.steps):
             qa.qattn_kv_append(xn, cache, scl, 0, kvt, group=p.group)
+    elif c == "step_int8":
+        # the benchmark step as bench.py times it: one quantization call and
+        # the prefill, captured as a CUDA graph after eager warm-up runs
+        p = synth.INT8_CAUSAL
+        d = synth.make_prefill(p)
+        x = {n: torch.from_numpy(d[n].view(np.int16)).to(dev).view(torch.bfloat16) for n in ("q", "k", "v")}
+        rot = torch.from_numpy(d["rot"]).to(dev)
+        shp = p.shape()
+        nqb, nkb = -(-p.N // 128), -(-p.N // 256)
+        c3 = [(torch.empty(shp, dtype=torch.uint8, device=dev), torch.empty((p.B, p.H, nb), device=dev))
+              for nb in (nqb, nkb, nkb)]
+        out = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+
+        def body(st):
+            qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype, out=c3, stream=st)
+            qa.qattn_prefill(*c3[0], *c3[1], *c3[2], p.code_dtype, p.layout, p.causal, out=out, stream=st)
+        g = capture_graph(body, args.warmup)
+        for _ in range(args.warmup + args.steps):
+            g.replay()
     elif c == "ablation_bf16":
         # the dequantize-first comparison path on the INT8 causal problem
         p = synth.INT8_CAUSAL
@@ -938,7 +957,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-heads", type=int, default=4, help="heads per reference-arm step")
-    ap.add_argument("--case", default=None, choices=["prefill_int8", "prefill_fp8", "prefill_int4v", "prefill_int4", "decode_int8kv",
+    ap.add_argument("--case", default=None, choices=["step_int8", "prefill_int8", "prefill_fp8", "prefill_int4v", "prefill_int4", "decode_int8kv",
                                                            "decode_int4kv", "kv_append_int8", "kv_append_int4",
                                                            "ablation_bf16"],
                     help="run one workload only (for profiler captures); prints no JSON")
