@@ -134,7 +134,10 @@ qattn_status_t qattn_rotate_block_quant(const void* x, qattn_dtype_t x_dtype,
  * kept); the quantization of V is enqueued on `stream` and takes SMs as they
  * free up; `stream` then waits for both rotations, so the call behaves as an
  * ordinary stream-ordered operation. Concurrent calls on one device
- * serialise their enqueueing. With rot == NULL the three passes run one after
+ * serialise their enqueueing. The call can be captured in a CUDA graph (the
+ * internal streams join the capture through events recorded on `stream`);
+ * the first call on a device creates those streams and events and should
+ * come before any capture. With rot == NULL the three passes run one after
  * the other on `stream`.
  *
  * Arguments as qattn_rotate_block_quant, for three tensors of one shape:
