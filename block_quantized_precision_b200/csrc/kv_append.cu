@@ -16,9 +16,10 @@
 //     [-127, 127].
 // Packed INT4 cache, one fp16 scale per token per group:
 //   kv_append_int4_kernel: eight lanes per new token of one (b, h_kv), 16
-//     channels each; s16 = fp16(absmax_group / 7), codes RNE(x / s16)
-//     clamped to [-7, 7] (the product with RN(1/s16) unless it is within
-//     1e-4 of a half-integer), packed two per byte.
+//     channels each; s16 = fp16(absmax_group / 7) (the quotient IEEE-
+//     rounded to float32 first), codes RNE(x / s16) clamped to [-7, 7] (the
+//     product with 1/s16 unless it is within 1e-4 of a half-integer),
+//     packed two per byte.
 // Both are small, memory-bound kernels (the new rows are read once, the
 // codes written once; a growing INT8 block also rewrites its earlier codes).
 #include <cuda_bf16.h>
@@ -47,6 +48,41 @@ __device__ __forceinline__ int code_fast(float y, float s, float rcp, bool slow,
   const float r = (v + 12582912.0f) - 12582912.0f;
   if (slow || fabsf(v - r) > 0.4999f) v = __fdiv_rn(y, s);
   return rne_clamp(v, lim);
+}
+
+// INT8 codes of the 8 bf16 values of v (two's complement bytes, value e in
+// byte e): the magic-number rounding of y * rcp in f32x2 pairs, the integer
+// landing in the low mantissa byte (|y / s| <= 127 here), with d = y * rcp -
+// RNE(y * rcp) from the exact product; when any |d| comes within 1e-4 of
+// 0.5, or the scale is below the smallest normal float32, all 8 are decided
+// by code_fast (the IEEE quotient where the product cannot decide).
+__device__ __forceinline__ uint2 codes8_i8(uint4 v, float s, float rcp, bool slow) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float f[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f[2 * k] = __uint_as_float(w[k] << 16);
+    f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+  const float2 rc = make_float2(rcp, rcp);
+  const float2 mg = make_float2(12582912.0f, 12582912.0f);
+  uint32_t t[8];
+  float dmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 y = make_float2(f[2 * i], f[2 * i + 1]);
+    const float2 m = ffma2(y, rc, mg);                                        // RNE(y * rcp) in the low bits
+    const float2 d = ffma2(y, rc, ffma2(m, make_float2(-1.0f, -1.0f), mg));   // y * rcp - that integer
+    dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+    t[2 * i] = __float_as_uint(m.x);
+    t[2 * i + 1] = __float_as_uint(m.y);
+  }
+  if (slow || dmax > 0.4999f) {                                               // rare: value by value
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = static_cast<uint32_t>(code_fast(f[e], s, rcp, slow, 127));
+  }
+  return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+                    __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
 }
 
 // x: bf16 [B, H_kv, n, D]; cache int8 [B, H_kv, L_max, D]; scales float32
@@ -129,17 +165,8 @@ __global__ void __launch_bounds__(kAppendThreads)
     for (int u = 0; u < 4; ++u) {
       const int64_t i = i0 + u * kAppendThreads;
       if (i >= total) break;
-      const uint32_t w[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
-      uint32_t o[2] = {0, 0};
-      if (s != 0.0f) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t lo = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] & 0xFFFFu), s, rcp, slow, 127)) & 0xFFu;
-          const uint32_t hi = static_cast<uint32_t>(code_fast(bf16_bits_to_f32(w[k] >> 16), s, rcp, slow, 127)) & 0xFFu;
-          o[k >> 1] |= (lo | (hi << 8)) << (16 * (k & 1));
-        }
-      }
-      *reinterpret_cast<uint2*>(cn + i * 8) = make_uint2(o[0], o[1]);
+      const uint2 o = s != 0.0f ? codes8_i8(vv[u], s, rcp, slow) : make_uint2(0, 0);
+      *reinterpret_cast<uint2*>(cn + i * 8) = o;
     }
   }
   if (threadIdx.x == 0) scales[head * nblk + blk] = s;
@@ -152,9 +179,15 @@ __global__ void __launch_bounds__(kAppendThreads)
 // work (group maximum, scale, reciprocal) is shared by them.
 constexpr int kInt4RowsPerCta = 64;                 // 32 rows per pass of 256 threads, two passes
 
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Codes RNE(y / s) clamped to [-7, 7] of 16 values, packed two per byte
 // (element 2i in the low nibble of byte i) into 8 bytes. The product with
-// rcp = RN(1/s) decides unless it lies within 1e-4 of a half-integer, or
+// rcp (1/s within 2^-22) decides unless it lies within 1e-4 of a half-integer, or
 // `wide` says a product may exceed 7.5 in magnitude (an fp16 scale in the
 // subnormal range can round well below absmax / 7); those take the IEEE
 // quotient, clamped.
@@ -224,12 +257,23 @@ __global__ void __launch_bounds__(kAppendThreads)
       const float other = __shfl_xor_sync(0xffffffffu, m, o);
       if (o < width) m = fmaxf(m, other);
     }
-    const __half s16 = __float2half_rn(__fdiv_rn(m, 7.0f));
+    // s16 = fp16(m / 7), the quotient IEEE-rounded to float32 first. m *
+    // RN(1/7) is within 1.75 float32 units of that quotient, so its fp16
+    // rounding is the same unless it lies within 3 units of an fp16 rounding
+    // midpoint (float32 mantissa bits 12..0 = 0x1000) or in the fp16
+    // subnormal range; those take the IEEE division.
+    float q7 = m * 0.142857149f;
+    if (q7 < 6.103515625e-05f || abs(static_cast<int>(__float_as_uint(q7) & 0x1FFFu) - 0x1000) <= 3)
+      q7 = __fdiv_rn(m, 7.0f);
+    const __half s16 = __float2half_rn(q7);
     const float s = __half2float(s16);
     uint2 codes = make_uint2(0, 0);
     if (s != 0.0f) {                                  // (fp16 scales are never subnormal in float32)
-      const float rcp = __frcp_rn(s);
-      codes = int4_codes16(f, s, rcp, m * rcp >= 7.5f);
+      // the approximate reciprocal (relative error below 2^-22) keeps every
+      // product within 2e-6 of the quotient (|y / s| <= 7.5), far inside the
+      // codes' 1e-4 margin; `wide` is decided with room for it
+      const float rcp = rcp_approx(s);
+      codes = int4_codes16(f, s, rcp, m * rcp >= 7.4999f);
     }
     if (row[ps] < n) {
       const int t = L + row[ps];

@@ -74,3 +74,33 @@ def test_ordered_on_the_callers_stream():
     assert qa.qattn_device_error() == qa.QATTN_OK
     for o in outs:
         assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
+
+
+def test_captured_in_a_cuda_graph():
+    """The call and a prefill captured as one CUDA graph (the internal
+    streams join the capture) and replayed: the same bytes as eager calls,
+    replay after replay, on new inputs copied into the captured buffers."""
+    p = synth.scaled(synth.INT8_CAUSAL, H=4, N=1024, seed=820)
+    d = synth.make_prefill(p)
+    x = {n: dev_bits(d[n], p.in_dtype) for n in ("q", "k", "v")}
+    rot = dev(d["rot"])
+    codes = qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype)   # creates the streams
+    out = qa.qattn_prefill(*codes[0], *codes[1], *codes[2], p.code_dtype, p.layout, p.causal)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = torch.cuda.current_stream()
+        qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, p.code_dtype, out=codes, stream=st)
+        qa.qattn_prefill(*codes[0], *codes[1], *codes[2], p.code_dtype, p.layout, p.causal, out=out, stream=st)
+    for seed in (821, 822):
+        d2 = synth.make_prefill(synth.scaled(p, seed=seed))
+        x2 = {n: dev_bits(d2[n], p.in_dtype) for n in ("q", "k", "v")}
+        want_codes = _three_calls(x2, rot, p, p.code_dtype)
+        want = qa.qattn_prefill(*want_codes[0], *want_codes[1], *want_codes[2], p.code_dtype, p.layout, p.causal)
+        for n in ("q", "k", "v"):
+            x[n].copy_(x2[n])
+        g.replay()
+        torch.cuda.synchronize()
+        assert qa.qattn_device_error() == qa.QATTN_OK
+        _same(codes, want_codes)
+        assert torch.equal(out.view(torch.int16), want.view(torch.int16))
