@@ -597,12 +597,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
   for (int64_t id = blockIdx.x; id < total; id += gridDim.x, ++it) {
     const int slot = it % kQStages;
     const uint32_t parity = (it / kQStages) & 1;
-    // One thread waits (bounded); the barrier releases the others, whose own
-    // completed test of the phase then orders their reads after the copy.
-    bool ok = true;
-    if (tid == 0) ok = mbar_wait(&full[slot], parity, &abort_flag, err);
-    if (!__syncthreads_and(ok)) break;
-    mbar_try_wait(&full[slot], parity);
+    // Every thread waits for the copy itself (bounded); the CTA decides on a
+    // timeout together at the barrier of the block maximum below.
+    const bool ok = mbar_wait(&full[slot], parity, &abort_flag, err);
     const int blk = static_cast<int>(id % nblk);
     const int bh = static_cast<int>(id / nblk);
     const int b = bh / H, h = bh % H;
@@ -614,7 +611,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     uint32_t mb0 = 0, mb1 = 0;
 #pragma unroll
     for (int i = 0; i < kVec; ++i) {
-      v[i] = src[tid + i * kQThreads];
+      v[i] = ok ? src[tid + i * kQThreads] : make_uint4(0, 0, 0, 0);
       mb0 = max_u16x2(mb0, max_u16x2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu));
       mb1 = max_u16x2(mb1, max_u16x2(v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu));
     }
@@ -624,7 +621,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((tid & 31) == 0) red[it & 1][tid >> 5] = m;
-    __syncthreads();  // also: every thread is done with the slot of block it - 1
+    if (!__syncthreads_and(ok)) break;  // also: every thread is done with the slot of block it - 1
     float amax = 0.0f;
 #pragma unroll
     for (int w = 0; w < kQThreads / 32; ++w) amax = fmaxf(amax, red[it & 1][w]);
