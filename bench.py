@@ -586,6 +586,19 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
                     "ms_prefill": round(ms_pf, 4), "TOPS_prefill": round(tops, 1),
                     "ms_quant_v": round(ms_qv, 4), "GB/s_quant_v": round(v_bytes / (ms_qv * 1e-3) / 1e9, 1),
                     "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TOPS", "frac": round(tops / int8_peak, 4)}}
+        if vt == qa.QATTN_INT4_PACKED:
+            # the other order: V widened to INT8 codes by its own HBM-bound
+            # pass, then the INT8 prefill (both timed, one flush before)
+            vw = qa.qattn_widen_int4(vcodes[0])
+            pw = lambda: (qa.qattn_widen_int4(vcodes[0], out=vw),
+                          qa.qattn_prefill(qk["q"][0], qk["q"][1], qk["k"][0], qk["k"][1], vw, vcodes[1],
+                                           qa.QATTN_INT8, p.layout, p.causal, out=out))
+            ms_pw = timeit(pw, n, flush)
+            tops_w = ops / (ms_pw * 1e-3) / 1e12
+            res[key]["widened_first"] = {"ms": round(ms_pw, 4), "TOPS": round(tops_w, 1),
+                                         "frac": round(tops_w / int8_peak, 4),
+                                         "calls": "qattn_widen_int4(V), qattn_prefill INT8"}
+            del vw
 
     # The dequantize-first comparison path on the same codes: bf16 = code x
     # scale written to HBM, then attention on the 16-bit tensor-core path
@@ -625,11 +638,40 @@ def extra_measurements(args, dev, stream, qa, synth, hbm_peak, int8_peak, fp32_p
         pf4()
     ms_full4 = timeit(full4, n, flush)
     tops4 = ops / (ms_pf4 * 1e-3) / 1e12
-    res["prefill_int4_qkv"] = {"workload": "%s, Q/K/V int4 packed" % p.name, "ms_prefill": round(ms_pf4, 4),
-                               "TOPS_prefill": round(tops4, 1), "ms_path": round(ms_full4, 4),
-                               "TOPS_path": round(ops / (ms_full4 * 1e-3) / 1e12, 1),
+    # The other order: each packed tensor widened to INT8 codes by its own
+    # HBM-bound pass (the widened codes stay in L2), then the INT8 prefill;
+    # its path quantizes Q/K/V in one call
+    w4 = {nm: qa.qattn_widen_int4(c4[nm][0]) for nm in ("q", "k", "v")}
+
+    def widen4():
+        for nm in ("q", "k", "v"):
+            qa.qattn_widen_int4(c4[nm][0], out=w4[nm])
+
+    def pw4():
+        widen4()
+        qa.qattn_prefill(w4["q"], c4["q"][1], w4["k"], c4["k"][1], w4["v"], c4["v"][1], qa.QATTN_INT8, p.layout,
+                         p.causal, out=out)
+
+    def full4w():
+        qa.qattn_rotate_block_quant_qkv(x["q"], x["k"], x["v"], p.layout, rot, qa.QATTN_INT4_PACKED,
+                                        out=[c4["q"], c4["k"], c4["v"]])
+        pw4()
+    ms_w4, ms_pw4, ms_full4w = timeit(widen4, n, flush), timeit(pw4, n, flush), timeit(full4w, n, flush)
+    w_bytes = 3 * sum(c4[nm][0].numel() for nm in ("q", "k", "v"))
+    tops4w = ops / (ms_pw4 * 1e-3) / 1e12
+    res["prefill_int4_qkv"] = {"workload": "%s, Q/K/V int4 packed" % p.name,
+                               "order": "widen to INT8 first (qattn_widen_int4 x3), then the INT8 prefill",
+                               "ms_prefill": round(ms_pw4, 4), "TOPS_prefill": round(tops4w, 1),
+                               "ms_widen": round(ms_w4, 4), "GB/s_widen": round(w_bytes / (ms_w4 * 1e-3) / 1e9, 1),
+                               "ms_path": round(ms_full4w, 4),
+                               "TOPS_path": round(ops / (ms_full4w * 1e-3) / 1e12, 1),
                                "roofline": {"bound": "tensor", "peak": int8_peak, "unit": "TOPS",
-                                            "frac": round(tops4 / int8_peak, 4)}}
+                                            "frac": round(tops4w / int8_peak, 4)},
+                               "on_chip": {"ms_prefill": round(ms_pf4, 4), "TOPS_prefill": round(tops4, 1),
+                                           "frac": round(tops4 / int8_peak, 4), "ms_path": round(ms_full4, 4),
+                                           "calls": "qattn_prefill_mixed INT4/INT4 (widened inside the kernel); "
+                                                    "path: three qattn_rotate_block_quant calls"}}
+    del w4
     return res
 
 
@@ -931,9 +973,11 @@ def profile_case(args):
     else:
         p = synth.FP8_LONG if c == "prefill_fp8" else synth.INT8_CAUSAL
         # prefill_int4v: the INT8 causal problem with V in packed INT4;
-        # prefill_int4: with Q, K and V in packed INT4
-        vt = qa.QATTN_INT4_PACKED if c in ("prefill_int4v", "prefill_int4") else p.code_dtype
-        qkt = qa.QATTN_INT4_PACKED if c == "prefill_int4" else p.code_dtype
+        # prefill_int4: with Q, K and V in packed INT4; prefill_int4_widened:
+        # the same codes widened to INT8 first, then the INT8 prefill
+        int4 = ("prefill_int4v", "prefill_int4", "prefill_int4_widened")
+        vt = qa.QATTN_INT4_PACKED if c in int4 else p.code_dtype
+        qkt = qa.QATTN_INT4_PACKED if c in int4[1:] else p.code_dtype
         d = synth.make_prefill(p)
         x = {n: torch.from_numpy(d[n].view(np.int16)).to(dev).view(torch.bfloat16) for n in ("q", "k", "v")}
         rot = torch.from_numpy(d["rot"]).to(dev)
@@ -941,7 +985,11 @@ def profile_case(args):
             qc = qa.qattn_rotate_block_quant(x["q"], p.layout, rot, 128, qkt)
             kc = qa.qattn_rotate_block_quant(x["k"], p.layout, rot, 256, qkt)
             vc = qa.qattn_rotate_block_quant(x["v"], p.layout, None, 256, vt)
-            qa.qattn_prefill_mixed(*qc, *kc, *vc, qkt, vt, p.layout, p.causal)
+            if c == "prefill_int4_widened":
+                qa.qattn_prefill(qa.qattn_widen_int4(qc[0]), qc[1], qa.qattn_widen_int4(kc[0]), kc[1],
+                                 qa.qattn_widen_int4(vc[0]), vc[1], qa.QATTN_INT8, p.layout, p.causal)
+            else:
+                qa.qattn_prefill_mixed(*qc, *kc, *vc, qkt, vt, p.layout, p.causal)
     torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
     print("case %s: ok" % c)
@@ -957,9 +1005,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-heads", type=int, default=4, help="heads per reference-arm step")
-    ap.add_argument("--case", default=None, choices=["step_int8", "prefill_int8", "prefill_fp8", "prefill_int4v", "prefill_int4", "decode_int8kv",
-                                                           "decode_int4kv", "kv_append_int8", "kv_append_int4",
-                                                           "ablation_bf16"],
+    ap.add_argument("--case", default=None,
+                    choices=["step_int8", "prefill_int8", "prefill_fp8", "prefill_int4v", "prefill_int4",
+                             "prefill_int4_widened", "decode_int8kv", "decode_int4kv", "kv_append_int8",
+                             "kv_append_int4", "ablation_bf16"],
                     help="run one workload only (for profiler captures); prints no JSON")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -7,7 +7,7 @@ fails, an exception is raised.
 
 Function names follow the C ABI:
     qattn_rotate_block_quant, qattn_rotate_block_quant_qkv, qattn_prefill, qattn_prefill_mixed,
-    qattn_dequant_bf16,
+    qattn_widen_int4, qattn_dequant_bf16,
     qattn_attention_bf16, qattn_decode_workspace_size,
     qattn_decode_kvq, qattn_decode_kvq_noalloc, qattn_kv_append, qattn_device_error,
     qattn_selftest_wait_timeout,
@@ -36,7 +36,7 @@ QATTN_F16, QATTN_BF16, QATTN_INT8, QATTN_FP8_E4M3, QATTN_INT4_PACKED = 0, 1, 2, 
 
 EXPORTED = ("qattn_abi_version", "qattn_status_string", "qattn_rotate_block_quant", "qattn_rotate_block_quant_qkv",
             "qattn_prefill",
-            "qattn_prefill_mixed", "qattn_dequant_bf16", "qattn_attention_bf16",
+            "qattn_prefill_mixed", "qattn_widen_int4", "qattn_dequant_bf16", "qattn_attention_bf16",
             "qattn_decode_workspace_size", "qattn_decode_kvq", "qattn_decode_kvq_noalloc", "qattn_kv_append",
             "qattn_attention_path_host_workspace_size", "qattn_attention_path_host",
             "qattn_device_error", "qattn_selftest_wait_timeout")
@@ -71,6 +71,7 @@ def lib() -> C.CDLL:
         L.qattn_prefill.restype = i
         L.qattn_prefill_mixed.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, f, P, P, P]
         L.qattn_prefill_mixed.restype = i
+        L.qattn_widen_int4.argtypes, L.qattn_widen_int4.restype = [P, C.c_int64, P, P], i
         L.qattn_dequant_bf16.argtypes = [P, P, i, i, i, i, i, i, i, P, P]
         L.qattn_dequant_bf16.restype = i
         L.qattn_attention_bf16.argtypes = [P, P, P, i, i, i, i, i, i, i, f, P, P, P]
@@ -207,6 +208,21 @@ def qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales,
                                    kv_block, int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse),
                                    _stream(stream))
     _check(st, "qattn_prefill_mixed")
+    return out
+
+
+def qattn_widen_int4(packed, out=None, stream=None):
+    """Packed INT4 codes ([..., D/2] bytes) widened to INT8 codes ([..., D]
+    bytes, int8 values -8..7, the same block scales apply)."""
+    import torch
+    if out is None:
+        out = torch.empty(tuple(packed.shape[:-1]) + (2 * packed.shape[-1],), dtype=torch.uint8,
+                          device=packed.device)
+    n = packed.numel() * packed.element_size()
+    if not (packed.is_contiguous() and out.is_contiguous()) or out.numel() * out.element_size() != 2 * n:
+        raise ValueError("qattn_widen_int4: contiguous tensors of n and 2n bytes expected")
+    st = lib().qattn_widen_int4(_ptr(packed), n, _ptr(out), _stream(stream))
+    _check(st, "qattn_widen_int4")
     return out
 
 

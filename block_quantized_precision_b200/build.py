@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqattn.so")
 SOURCES = ["qattn_abi.cu", "rotate_quant.cu", "prefill.cu", "prefill_bf16.cu", "decode.cu", "decode_noalloc.cu", "kv_append.cu",
-           "path_host.cu"]
+           "path_host.cu", "widen_int4.cu"]
 HEADERS = ["qattn_device.cuh", "qattn_internal.h", "prefill_common.cuh"]
 
 NVCC_FLAGS = [

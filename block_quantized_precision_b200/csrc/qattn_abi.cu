@@ -350,6 +350,20 @@ qattn_status_t qattn_prefill(const void* q_codes, const float* q_scales, const v
                              stream);
 }
 
+qattn_status_t qattn_widen_int4(const void* packed, int64_t n_packed, void* out, qattn_stream_t stream) {
+  if (n_packed < 0) return QATTN_ERR_INVALID_ARG;
+  if (n_packed == 0) return QATTN_OK;
+  if (!packed || !out) return QATTN_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(out)) return QATTN_ERR_ALIGNMENT;
+  const uintptr_t p0 = reinterpret_cast<uintptr_t>(packed), o0 = reinterpret_cast<uintptr_t>(out);
+  const uintptr_t n = static_cast<uintptr_t>(n_packed);
+  if (p0 < o0 + 2 * n && o0 < p0 + n) return QATTN_ERR_INVALID_ARG;   // overlapping ranges
+  DeviceState* ds = nullptr;
+  qattn_status_t s = device_state(&ds);
+  if (s != QATTN_OK) return s;
+  return from_cuda(launch_widen_int4(packed, n_packed, out, reinterpret_cast<cudaStream_t>(stream), ds->num_sms));
+}
+
 qattn_status_t qattn_dequant_bf16(const void* codes, const float* scales, qattn_dtype_t code_dtype,
                                   qattn_layout_t layout, int B, int H, int N, int D, int block_tokens, void* out,
                                   qattn_stream_t stream) {

@@ -55,6 +55,10 @@ bool prefill_supported(int D);
 bool prefill_codes_supported(int qk_code, int v_code);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t st, int num_sms, int* err);
 
+// Packed INT4 codes (n bytes) to INT8 codes (2n bytes), element order kept
+// (widen_int4.cu).
+cudaError_t launch_widen_int4(const void* packed, int64_t n, void* out, cudaStream_t st, int num_sms);
+
 // The dequantize-first comparison path (prefill_bf16.cu).
 struct DequantArgs {
   const void* codes;  // INT8 or e4m3, 1 byte per element, layout as the input

@@ -220,6 +220,38 @@ qattn_status_t qattn_prefill_mixed(const void* q_codes, const float* q_scales, c
                                    qattn_stream_t stream);
 
 /*
+ * Packed INT4 codes widened to INT8 codes of the same values.
+ *
+ * Defined by: "FlashAttention 的 INT8/INT4 量化", 第二层 (INT4 codes are
+ * widened to INT8 before the integer matmul); packing as in
+ * "ops-transformer INT8/INT4 量化推理", 5.2.
+ *
+ * out[2i] = the low nibble of packed[i], out[2i + 1] = its high nibble, each
+ * as a signed 4-bit value (-8..7) stored in one INT8 byte. A packed code
+ * tensor [B,H,N,D/2] or [B,N,H,D/2] thus becomes the INT8 code tensor
+ * [B,H,N,D] or [B,N,H,D] with the same block scales, and
+ *   qattn_widen_int4(q), (k), (v) then qattn_prefill(..., QATTN_INT8, ...)
+ * computes what qattn_prefill_mixed(..., QATTN_INT4_PACKED,
+ * QATTN_INT4_PACKED, ...) computes: the same integer scores and P.V sums
+ * (qattn_prefill_mixed widens each nibble on chip as code + 8 and removes
+ * the offset in float32, so the two outputs can differ in the last bits;
+ * both stay within the prefill's tolerance). Widening V alone does the same
+ * for INT8 Q/K with INT4 V. On B200 this order is the faster one: this pass
+ * is bound by HBM (n_packed bytes read, 2 n_packed written, the output left
+ * in L2), the prefill by instruction issue, where qattn_prefill_mixed
+ * widens inside the pipeline that feeds the softmax warps and needs no
+ * extra memory.
+ *
+ *   packed:   n_packed bytes, device memory, 16-byte aligned.
+ *   out:      2 * n_packed bytes, device memory, 16-byte aligned,
+ *             caller-owned; must not overlap packed.
+ * Errors: QATTN_ERR_INVALID_ARG (n_packed < 0, null pointer with
+ * n_packed > 0, overlapping ranges), QATTN_ERR_ALIGNMENT, QATTN_ERR_CUDA.
+ * n_packed == 0 does nothing. Asynchronous on `stream`; allocates nothing.
+ */
+qattn_status_t qattn_widen_int4(const void* packed, int64_t n_packed, void* out, qattn_stream_t stream);
+
+/*
  * The dequantize-first comparison path: the standard INT8 path that the
  * pages contrast with quantized attention ("INT8 量化算子", ops-transformer
  * items 1-2: INT8 is converted back to FP16 and multiplied in FP16, where the

@@ -167,3 +167,16 @@ def test_rotate_block_quant_qkv_validation(L):
     assert f(*args(q=bad + 8)) == qa.QATTN_ERR_ALIGNMENT
     assert f(*args(vc=None)) == qa.QATTN_ERR_INVALID_ARG          # V codes missing
     assert f(*args(B=0)) == qa.QATTN_OK                            # empty problem
+
+
+def test_widen_int4_validation(L):
+    bad = 0x1000
+    w = L.qattn_widen_int4
+    assert w(bad, -1, bad + 4096, None) == qa.QATTN_ERR_INVALID_ARG
+    assert w(None, 0, None, None) == qa.QATTN_OK                      # nothing to widen
+    assert w(None, 16, bad, None) == qa.QATTN_ERR_INVALID_ARG
+    assert w(bad, 16, None, None) == qa.QATTN_ERR_INVALID_ARG
+    assert w(bad + 8, 16, bad + 4096, None) == qa.QATTN_ERR_ALIGNMENT
+    assert w(bad, 16, bad + 4104, None) == qa.QATTN_ERR_ALIGNMENT
+    assert w(bad, 64, bad + 48, None) == qa.QATTN_ERR_INVALID_ARG    # out overlaps the input's tail
+    assert w(bad + 64, 64, bad, None) == qa.QATTN_ERR_INVALID_ARG    # input inside the output

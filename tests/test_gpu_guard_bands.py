@@ -207,3 +207,15 @@ def test_rotate_block_quant_qkv(N, code):
     for name, (c, s) in zip("qkv", outs):
         c.check("%s codes" % name)
         s.check("%s scales" % name)
+
+
+@pytest.mark.parametrize("n", [17, 4096 + 7, 300 * 64])
+def test_widen_int4(n):
+    """The INT4 -> INT8 widening pass writes its 2n bytes and nothing else
+    (byte tail beyond the last 16-byte vector included)."""
+    rng = np.random.default_rng(n)
+    packed = torch.from_numpy(rng.integers(0, 256, n, dtype=np.uint8)).cuda()
+    out = Guarded((2 * n,), torch.uint8)
+    qa.qattn_widen_int4(packed, out=out.t)
+    torch.cuda.synchronize()
+    out.check("widened codes")

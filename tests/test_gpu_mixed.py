@@ -65,6 +65,13 @@ def _mixed(orc, p, d, v_dtype, rows_by_head, check_codes=True):
     vc, vs = qa.qattn_rotate_block_quant(v, p.layout, None, 256, v_dtype)
     lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device="cuda")
     out = qa.qattn_prefill_mixed(qc, qs, kc, ks, vc, vs, qa.QATTN_INT8, v_dtype, p.layout, p.causal, lse=lse)
+    runs = [(out, lse, "on chip")]
+    if v_dtype == synth.INT4_PACKED:
+        # V widened to INT8 codes first, then the INT8 prefill
+        lse_w = torch.empty_like(lse)
+        out_w = qa.qattn_prefill(qc, qs, kc, ks, qa.qattn_widen_int4(vc), vs, qa.QATTN_INT8, p.layout, p.causal,
+                                 lse=lse_w)
+        runs.append((out_w, lse_w, "widened first"))
     torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
     heads = sorted(rows_by_head)
@@ -79,13 +86,18 @@ def _mixed(orc, p, d, v_dtype, rows_by_head, check_codes=True):
                 assert np.array_equal(gsc[b, h], o[1][b, h])
     ref = orc.prefill_rows(*oq, *ok_, *ov, synth.INT8, p.layout, p.causal, rows_by_head, want_lse=True,
                            v_dtype=v_dtype)
-    out_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
-    lse_np = lse.cpu().numpy()
-    for (b, h), rows in rows_by_head.items():
-        got = bf16_to_f64(head_rows(out_bits, p.layout, b, h)[rows])
-        vmax = dequant_v_max(ov[0], ov[1], v_dtype, p.layout, b, h, orc)
-        assert_close(got, bf16_to_f64(ref[(b, h)][0]), vmax, "head (%d,%d)" % (b, h))
-        assert np.abs(lse_np[b, h, rows] - ref[(b, h)][2]).max() < 1e-2
+    _check_runs(orc, p, runs, ref, ov, v_dtype, rows_by_head)
+
+
+def _check_runs(orc, p, runs, ref, ov, v_dtype, rows_by_head):
+    for (out, lse, how) in runs:
+        out_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+        lse_np = lse.cpu().numpy()
+        for (b, h), rows in rows_by_head.items():
+            got = bf16_to_f64(head_rows(out_bits, p.layout, b, h)[rows])
+            vmax = dequant_v_max(ov[0], ov[1], v_dtype, p.layout, b, h, orc)
+            assert_close(got, bf16_to_f64(ref[(b, h)][0]), vmax, "head (%d,%d), %s" % (b, h, how))
+            assert np.abs(lse_np[b, h, rows] - ref[(b, h)][2]).max() < 1e-2, how
 
 
 @pytest.mark.parametrize("v_dtype", [synth.INT4_PACKED, synth.FP8_E4M3])
@@ -146,9 +158,13 @@ def _int4_all(orc, p, d, rows_by_head, check_codes=True):
     lse = torch.empty((p.B, p.H, p.N), dtype=torch.float32, device="cuda")
     out = qa.qattn_prefill_mixed(*c["q"], *c["k"], *c["v"], qa.QATTN_INT4_PACKED, qa.QATTN_INT4_PACKED, p.layout,
                                  p.causal, lse=lse)
+    # every operand widened to INT8 codes first, then the INT8 prefill
+    w = {nm: (qa.qattn_widen_int4(c[nm][0]), c[nm][1]) for nm in "qkv"}
+    lse_w = torch.empty_like(lse)
+    out_w = qa.qattn_prefill(*w["q"], *w["k"], *w["v"], qa.QATTN_INT8, p.layout, p.causal, lse=lse_w)
     torch.cuda.synchronize()
     assert qa.qattn_device_error() == qa.QATTN_OK
-    assert out.shape == tuple(p.shape())
+    assert out.shape == tuple(p.shape()) and out_w.shape == tuple(p.shape())
     heads = sorted(rows_by_head)
     o = {nm: orc.rotate_block_quant(d[nm], p.in_dtype, p.layout, d["rot"] if nm != "v" else None,
                                     128 if nm == "q" else 256, synth.INT4_PACKED, heads=heads) for nm in "qkv"}
@@ -160,13 +176,8 @@ def _int4_all(orc, p, d, rows_by_head, check_codes=True):
                 assert np.array_equal(gsc[b, h], o[nm][1][b, h])
     ref = orc.prefill_rows(*o["q"], *o["k"], *o["v"], synth.INT4_PACKED, p.layout, p.causal, rows_by_head,
                            want_lse=True)
-    out_bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
-    lse_np = lse.cpu().numpy()
-    for (b, h), rows in rows_by_head.items():
-        got = bf16_to_f64(head_rows(out_bits, p.layout, b, h)[rows])
-        vmax = dequant_v_max(o["v"][0], o["v"][1], synth.INT4_PACKED, p.layout, b, h, orc)
-        assert_close(got, bf16_to_f64(ref[(b, h)][0]), vmax, "head (%d,%d)" % (b, h))
-        assert np.abs(lse_np[b, h, rows] - ref[(b, h)][2]).max() < 1e-2
+    _check_runs(orc, p, [(out, lse, "on chip"), (out_w, lse_w, "widened first")], ref, o["v"], synth.INT4_PACKED,
+                rows_by_head)
 
 
 @pytest.mark.parametrize("D", [64, 128])
