@@ -185,16 +185,16 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// Codes RNE(y / s) clamped to [-7, 7] of 16 values, packed two per byte
-// (element 2i in the low nibble of byte i) into 8 bytes. The product with
-// rcp (1/s within 2^-22) decides unless it lies within 1e-4 of a half-integer, or
-// `wide` says a product may exceed 7.5 in magnitude (an fp16 scale in the
-// subnormal range can round well below absmax / 7); those take the IEEE
-// quotient, clamped.
-__device__ __forceinline__ uint2 int4_codes16(const float (&f)[16], float s, float rcp, bool wide) {
+// Codes RNE(y / s) of 16 values, packed two per byte (element 2i in the low
+// nibble of byte i) into 8 bytes: the product with rcp (1/s within 2^-22)
+// rounded by the 1.5 * 2^23 addend. That decides the code unless the product
+// lies within 1e-4 of a half-integer; `redo` is then set (it may already be
+// set when a product can exceed 7.5, see the caller) and the caller
+// completes the codes with int4_codes16_exact.
+__device__ __forceinline__ uint2 int4_codes16(const float (&f)[16], float rcp, bool& redo) {
   const float2 rc = make_float2(rcp, rcp);
   const float2 mg = make_float2(12582912.0f, 12582912.0f);
-  uint32_t t[16];
+  uint32_t b[8];                                  // byte i: codes 2i (low nibble) and 2i + 1
   float dmax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -202,19 +202,50 @@ __device__ __forceinline__ uint2 int4_codes16(const float (&f)[16], float s, flo
     const float2 m = ffma2(y, rc, mg);                               // RNE(y * rcp) in the low bits
     const float2 d = ffma2(y, rc, ffma2(m, make_float2(-1.0f, -1.0f), mg));   // y * rcp - that integer
     dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-    t[2 * i] = __float_as_uint(m.x);
-    t[2 * i + 1] = __float_as_uint(m.y);
+    b[i] = (__float_as_uint(m.x) & 0xFu) | ((__float_as_uint(m.y) & 0xFu) << 4);
   }
-  if (wide || dmax > 0.4999f) {                                      // rare: decide exactly
-#pragma unroll
-    for (int e = 0; e < 16; ++e)
-      t[e] = static_cast<uint32_t>(max(-7, min(7, __float2int_rn(__fdiv_rn(f[e], s)))));
-  }
-  uint32_t w[2] = {0, 0};
-#pragma unroll
-  for (int e = 0; e < 16; ++e) w[e >> 3] |= (t[e] & 0xFu) << (4 * (e & 7));
-  return make_uint2(w[0], w[1]);
+  redo = redo || dmax > 0.4999f;
+  return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                    __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
 }
+
+// Completes the codes of int4_codes16 where it could not decide them all
+// (the values come as their bf16 bits, two per word, element 2k in the low
+// half): each value's product is formed and checked again, and only the
+// values within 1e-4 of a half-integer (every value when `wide`) take the
+// IEEE quotient, clamped to [-7, 7], one division per such value; with bf16
+// inputs that is about one value in a thousand. Out of line, so that the
+// common path carries none of this.
+__device__ __noinline__ uint2 int4_codes16_exact(uint4 lo, uint4 hi, float s, float rcp, bool wide, uint2 codes) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  const float mg = 12582912.0f;
+  uint32_t redo = 0;                                  // bit e: value e takes the quotient
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float y = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+    const float m = __fmaf_rn(y, rcp, mg);                           // as in int4_codes16
+    const float d = __fmaf_rn(y, rcp, mg - m);
+    if (wide || fabsf(d) > 0.4999f) redo |= 1u << e;
+  }
+#pragma unroll 1
+  while (redo != 0) {
+    const int e = __ffs(static_cast<int>(redo)) - 1;
+    redo &= redo - 1;
+    const int k = e >> 1;
+    const uint4 v = k < 4 ? lo : hi;
+    const uint32_t wd = (k & 3) == 0 ? v.x : (k & 3) == 1 ? v.y : (k & 3) == 2 ? v.z : v.w;
+    const float y = __uint_as_float((e & 1) ? (wd & 0xFFFF0000u) : (wd << 16));
+    const uint32_t c = static_cast<uint32_t>(max(-7, min(7, __float2int_rn(__fdiv_rn(y, s))))) & 0xFu;
+    const int sh = 4 * (e & 7);
+    if (e < 8) codes.x = (codes.x & ~(0xFu << sh)) | (c << sh);
+    else codes.y = (codes.y & ~(0xFu << sh)) | (c << sh);
+  }
+  return codes;
+}
+
+// RN(m / 7) for the rare group maxima whose fp16 rounding the product with
+// RN(1/7) cannot decide; out of line for the same reason.
+__device__ __noinline__ float div7_exact(float m) { return __fdiv_rn(m, 7.0f); }
 
 // Grid (ceil(n / kInt4RowsPerCta), B * H_kv): blockIdx.y is the (b, h_kv) head.
 __global__ void __launch_bounds__(kAppendThreads)
@@ -264,7 +295,7 @@ __global__ void __launch_bounds__(kAppendThreads)
     // subnormal range; those take the IEEE division.
     float q7 = m * 0.142857149f;
     if (q7 < 6.103515625e-05f || abs(static_cast<int>(__float_as_uint(q7) & 0x1FFFu) - 0x1000) <= 3)
-      q7 = __fdiv_rn(m, 7.0f);
+      q7 = div7_exact(m);
     const __half s16 = __float2half_rn(q7);
     const float s = __half2float(s16);
     uint2 codes = make_uint2(0, 0);
@@ -273,7 +304,10 @@ __global__ void __launch_bounds__(kAppendThreads)
       // product within 2e-6 of the quotient (|y / s| <= 7.5), far inside the
       // codes' 1e-4 margin; `wide` is decided with room for it
       const float rcp = rcp_approx(s);
-      codes = int4_codes16(f, s, rcp, m * rcp >= 7.4999f);
+      const bool wide = m * rcp >= 7.4999f;
+      bool redo = wide;
+      codes = int4_codes16(f, rcp, redo);
+      if (redo) codes = int4_codes16_exact(raw[ps][0], raw[ps][1], s, rcp, wide, codes);
     }
     if (row[ps] < n) {
       const int t = L + row[ps];

@@ -90,3 +90,33 @@ def test_int8_decode_problem_size(orc):
         L += n
     assert np.array_equal(gc.cpu().numpy(), cache)
     assert np.array_equal(gs.cpu().numpy().view(np.uint32), sc.view(np.uint32))
+
+
+@pytest.mark.parametrize("group", [128, 64])
+def test_int4_ties_and_near_ties(orc, group):
+    """Rows whose every group has maximum |x| = 7 exactly (fp16 scale exactly
+    1) holding half-integers k + 1/2 (exact ties, decided to even) and their
+    bf16 neighbours one unit away: every code as the IEEE quotient decides
+    it, against the oracle."""
+    B, H, n, D, Lmax = 1, 2, 64, 128, 128
+    rng = np.random.default_rng(group)
+    half = (rng.integers(-7, 7, (B, H, n, D)) + 0.5).astype(np.float32)
+    x = np.where(rng.random((B, H, n, D)) < 0.6, half, rng.uniform(-6.9, 6.9, (B, H, n, D))).astype(np.float32)
+    for g0 in range(0, D, group):
+        x[..., g0] = np.where(rng.random((B, H, n)) < 0.5, 7.0, -7.0)
+    bits = synth.f32_to_bf16_bits(x)
+    step = np.where(rng.random(bits.shape) < 0.5, 1, -1).astype(np.int32)
+    near = (rng.random(bits.shape) < 0.2) & (np.abs(x) < 6.9)
+    bits = np.where(near, (bits.astype(np.int32) + step).astype(np.uint16), bits)
+    oc = np.zeros((B, H, Lmax, D // 2), np.uint8)
+    osc = np.zeros((B, H, Lmax, D // group), np.uint16)
+    gc = dev(oc.copy())
+    gs = dev(osc.copy()).view(torch.float16)
+    xg = dev(bits.view(np.int16)).view(torch.bfloat16)
+    qa.qattn_kv_append(xg, gc, gs, 0, synth.INT4_PACKED, group=group)
+    torch.cuda.synchronize()
+    assert qa.qattn_device_error() == qa.QATTN_OK
+    oc, osc = orc.kv_append(bits, oc, osc, 0, synth.INT4_PACKED, group=group)
+    assert np.array_equal(osc[:, :, :n], np.full((B, H, n, D // group), 0x3C00, np.uint16))   # scale 1.0
+    assert np.array_equal(gc.cpu().numpy(), oc)
+    assert np.array_equal(gs.view(torch.int16).cpu().numpy().view(np.uint16), osc)
