@@ -110,7 +110,21 @@ def _check(status: int, where: str):
 
 
 def _ptr(t) -> Optional[int]:
+    """Address of a host tensor (or None)."""
     return None if t is None else t.data_ptr()
+
+
+def _dptr(t) -> Optional[int]:
+    """Address of a device tensor (or None). The kernels read and write the
+    dense row-major extent from that address, so a tensor on the host or a
+    strided view is refused here instead of being read out of bounds."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor, got one on %s" % t.device)
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor (shape %s, strides %s)" % (tuple(t.shape), t.stride()))
+    return t.data_ptr()
 
 
 def _stream(stream) -> Optional[int]:
@@ -144,8 +158,8 @@ def qattn_rotate_block_quant(x, layout: int, rot, block_tokens: int, code_dtype:
         codes = torch.empty(shape, dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((B, H, nblk), dtype=torch.float32, device=x.device)
-    st = lib().qattn_rotate_block_quant(_ptr(x), x_dtype, layout, B, H, N, D, _ptr(rot), block_tokens,
-                                        code_dtype, _ptr(codes), _ptr(scales), _stream(stream))
+    st = lib().qattn_rotate_block_quant(_dptr(x), x_dtype, layout, B, H, N, D, _dptr(rot), block_tokens,
+                                        code_dtype, _dptr(codes), _dptr(scales), _stream(stream))
     _check(st, "qattn_rotate_block_quant")
     return codes, scales
 
@@ -168,8 +182,8 @@ def qattn_rotate_block_quant_qkv(q, k, v, layout: int, rot, code_dtype: int, out
             out.append((torch.empty(shape, dtype=torch.uint8, device=q.device),
                         torch.empty((B, H, -(-N // blk)), dtype=torch.float32, device=q.device)))
     (qc, qs), (kc, ks), (vc, vs) = out
-    st = lib().qattn_rotate_block_quant_qkv(_ptr(q), _ptr(k), _ptr(v), x_dtype, layout, B, H, N, D, _ptr(rot),
-                                            code_dtype, _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(vc), _ptr(vs),
+    st = lib().qattn_rotate_block_quant_qkv(_dptr(q), _dptr(k), _dptr(v), x_dtype, layout, B, H, N, D, _dptr(rot),
+                                            code_dtype, _dptr(qc), _dptr(qs), _dptr(kc), _dptr(ks), _dptr(vc), _dptr(vs),
                                             _stream(stream))
     _check(st, "qattn_rotate_block_quant_qkv")
     return out
@@ -184,9 +198,9 @@ def qattn_prefill(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, code_
     Nkv = _dims(k_codes, layout)[2]
     if out is None:
         out = torch.empty(q_codes.shape, dtype=torch.bfloat16, device=q_codes.device)
-    st = lib().qattn_prefill(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
-                             _ptr(v_scales), code_dtype, layout, B, H, Nq, Nkv, D, q_block, kv_block,
-                             int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    st = lib().qattn_prefill(_dptr(q_codes), _dptr(q_scales), _dptr(k_codes), _dptr(k_scales), _dptr(v_codes),
+                             _dptr(v_scales), code_dtype, layout, B, H, Nq, Nkv, D, q_block, kv_block,
+                             int(bool(causal)), float(softmax_scale), _dptr(out), _dptr(lse), _stream(stream))
     _check(st, "qattn_prefill")
     return out
 
@@ -203,9 +217,9 @@ def qattn_prefill_mixed(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales,
     Nkv = _dims(k_codes, layout)[2]
     if out is None:
         out = torch.empty(tuple(q_codes.shape[:-1]) + (D,), dtype=torch.bfloat16, device=q_codes.device)
-    st = lib().qattn_prefill_mixed(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
-                                   _ptr(v_scales), qk_dtype, v_dtype, layout, B, H, Nq, Nkv, D, q_block,
-                                   kv_block, int(bool(causal)), float(softmax_scale), _ptr(out), _ptr(lse),
+    st = lib().qattn_prefill_mixed(_dptr(q_codes), _dptr(q_scales), _dptr(k_codes), _dptr(k_scales), _dptr(v_codes),
+                                   _dptr(v_scales), qk_dtype, v_dtype, layout, B, H, Nq, Nkv, D, q_block,
+                                   kv_block, int(bool(causal)), float(softmax_scale), _dptr(out), _dptr(lse),
                                    _stream(stream))
     _check(st, "qattn_prefill_mixed")
     return out
@@ -221,7 +235,7 @@ def qattn_widen_int4(packed, out=None, stream=None):
     n = packed.numel() * packed.element_size()
     if not (packed.is_contiguous() and out.is_contiguous()) or out.numel() * out.element_size() != 2 * n:
         raise ValueError("qattn_widen_int4: contiguous tensors of n and 2n bytes expected")
-    st = lib().qattn_widen_int4(_ptr(packed), n, _ptr(out), _stream(stream))
+    st = lib().qattn_widen_int4(_dptr(packed), n, _dptr(out), _stream(stream))
     _check(st, "qattn_widen_int4")
     return out
 
@@ -233,7 +247,7 @@ def qattn_dequant_bf16(codes, scales, code_dtype: int, layout: int, block_tokens
     B, H, N, D = _dims(codes, layout)
     if out is None:
         out = torch.empty(codes.shape, dtype=torch.bfloat16, device=codes.device)
-    st = lib().qattn_dequant_bf16(_ptr(codes), _ptr(scales), code_dtype, layout, B, H, N, D, block_tokens, _ptr(out),
+    st = lib().qattn_dequant_bf16(_dptr(codes), _dptr(scales), code_dtype, layout, B, H, N, D, block_tokens, _dptr(out),
                                   _stream(stream))
     _check(st, "qattn_dequant_bf16")
     return out
@@ -248,8 +262,8 @@ def qattn_attention_bf16(q, k, v, layout: int, causal: bool, softmax_scale: floa
     Nkv = _dims(k, layout)[2]
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
-    st = lib().qattn_attention_bf16(_ptr(q), _ptr(k), _ptr(v), layout, B, H, Nq, Nkv, D, int(bool(causal)),
-                                    float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream))
+    st = lib().qattn_attention_bf16(_dptr(q), _dptr(k), _dptr(v), layout, B, H, Nq, Nkv, D, int(bool(causal)),
+                                    float(softmax_scale), _dptr(out), _dptr(lse), _stream(stream))
     _check(st, "qattn_attention_bf16")
     return out
 
@@ -277,9 +291,9 @@ def qattn_attention_path_host(q, k, v, rot, layout: int, code_dtype: int, causal
     need = qattn_attention_path_host_workspace_size(B, H, N, D, layout, groups)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-    st = lib().qattn_attention_path_host(_ptr(q), _ptr(k), _ptr(v), x_dtype, layout, B, H, N, D, _ptr(rot),
+    st = lib().qattn_attention_path_host(_ptr(q), _ptr(k), _ptr(v), x_dtype, layout, B, H, N, D, _dptr(rot),
                                          code_dtype, int(bool(causal)), float(softmax_scale), _ptr(out),
-                                         int(groups), _ptr(workspace), workspace.numel(), _stream(stream))
+                                         int(groups), _dptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "qattn_attention_path_host")
     return out
 
@@ -302,9 +316,9 @@ def qattn_decode_kvq(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: int, kv_
     need = qattn_decode_workspace_size(B, Hq, Hkv, L, D)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    st = lib().qattn_decode_kvq(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales), kv_dtype,
-                                B, Hq, Hkv, L, D, kv_block, group, float(softmax_scale), _ptr(out),
-                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    st = lib().qattn_decode_kvq(_dptr(q), _dptr(k_cache), _dptr(v_cache), _dptr(k_scales), _dptr(v_scales), kv_dtype,
+                                B, Hq, Hkv, L, D, kv_block, group, float(softmax_scale), _dptr(out),
+                                _dptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "qattn_decode_kvq")
     return out
 
@@ -322,9 +336,9 @@ def qattn_decode_kvq_noalloc(q, k_cache, v_cache, k_scales, v_scales, kv_dtype: 
     Hkv, L = k_cache.shape[1], k_cache.shape[2]
     if out is None:
         out = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=q.device)
-    st = lib().qattn_decode_kvq_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+    st = lib().qattn_decode_kvq_noalloc(_dptr(q), _dptr(k_cache), _dptr(v_cache), _dptr(k_scales), _dptr(v_scales),
                                         kv_dtype, B, Hq, Hkv, L, D, kv_block, group, float(softmax_scale),
-                                        _ptr(out), _stream(stream))
+                                        _dptr(out), _stream(stream))
     _check(st, "qattn_decode_kvq_noalloc")
     return out
 
@@ -337,7 +351,7 @@ def qattn_kv_append(x_new, cache, scales, L: int, kv_dtype: int, kv_block: int =
     [B, H_kv, L_max, D/2], scales float16 [B, H_kv, L_max, D/group]."""
     B, Hkv, n, D = x_new.shape
     Lmax = cache.shape[2]
-    st = lib().qattn_kv_append(_ptr(x_new), B, Hkv, n, D, kv_dtype, int(L), Lmax, _ptr(cache), _ptr(scales),
+    st = lib().qattn_kv_append(_dptr(x_new), B, Hkv, n, D, kv_dtype, int(L), Lmax, _dptr(cache), _dptr(scales),
                                kv_block, group, _stream(stream))
     _check(st, "qattn_kv_append")
     return cache, scales
